@@ -1,0 +1,342 @@
+/*
+ * NSA forward oracle: a plain, slow, fp64 CPU statement of what the
+ * Native Sparse Attention forward pass computes.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the tests, the package smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header or constant with the
+ * CUDA path.
+ *
+ * Sources (web pages on Native Sparse Attention):
+ *  - "DeepSeek NSA ... config.toml" (qwbw.cn/news/106443), section 1: three
+ *    parallel branches per query (compressed coarse attention, selected
+ *    fine-grained blocks, sliding window) aggregated by a gate; section 3:
+ *    the knobs compress_block_size, select_block_size, select_top_k,
+ *    sliding_window, gate_type = learned, dtype = bfloat16.
+ *  - "DeepSeek NSA in manufacturing" (chencunli.com), section "动态稀疏到底稀疏了什么":
+ *    every block gets a learned compressed representation, the query attends
+ *    coarsely to all compressed blocks and the highest-scoring blocks are
+ *    selected; inside the selected blocks it attends token by token; the
+ *    illustrative selector flattens each key block and applies one linear map.
+ *  - "NSA vs MoBA" (gtnt.cn/news/122266), section 1: block compression,
+ *    dynamic top-k selection, sliding-window local attention.
+ *
+ * Readings taken where the pages are silent (each one is listed in the design
+ * notes of the repository):
+ *  - compressor: one linear map per KV head, W[h] of shape [D, l*D], applied
+ *    to the flattened block (element p*D + c is token p, channel c), no bias;
+ *    separate maps for keys and values; the compressed tensor is stored in
+ *    bf16 (round to nearest even), and steps 2-3 use that stored tensor;
+ *  - a compressed block is visible to query t once its last token is <= t;
+ *  - block score = sum over the query heads of the KV group of the compressed
+ *    softmax probabilities (l == d == l'), the incomplete block holding t is a
+ *    candidate with score 0; ties go to the lower block index; if there are at
+ *    most n candidates, all are taken;
+ *  - window = the w tokens ending at t (t included);
+ *  - scale 1/sqrt(D) by default for all three branches;
+ *  - an empty branch contributes 0;
+ *  - gates are given per token, head and branch (order cmp, slc, win) and are
+ *    applied as given.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+  int D;      /* head dim (d_k = d_v) */
+  int Hq;     /* query heads */
+  int Hkv;    /* key/value heads; G = Hq / Hkv query heads per group */
+  int l;      /* compression block length */
+  int d;      /* compression stride */
+  int lsel;   /* selection block length l' */
+  int n;      /* top-n selected blocks */
+  int w;      /* sliding-window length */
+  double scale;
+} nsa_oracle_params;
+
+/* ------------------------------------------------------------ bf16 <-> f64 */
+double oracle_bf16_to_f64(uint16_t b) {
+  uint32_t u = ((uint32_t)b) << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* Round an fp64 value to the nearest bf16 (ties to even), single rounding. */
+uint16_t oracle_f64_to_bf16(double x) {
+  if (x != x) return 0x7FC0;
+  double ax = fabs(x);
+  double r;
+  if (ax == 0.0) {
+    r = 0.0;
+  } else if (ax < ldexp(1.0, -126)) {
+    /* subnormal range: spacing 2^-133 */
+    r = nearbyint(ax * ldexp(1.0, 133)) * ldexp(1.0, -133);
+  } else {
+    int e;
+    double m = frexp(ax, &e);          /* ax = m * 2^e, m in [0.5, 1) */
+    double q = nearbyint(m * 256.0);   /* 8 significant bits, ties to even */
+    r = ldexp(q, e - 8);
+    if (r >= ldexp(1.0, 128)) r = INFINITY;
+  }
+  float f = (float)r; /* exact: r is representable in bf16 */
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  uint16_t b = (uint16_t)(u >> 16);
+  if (x < 0) b |= 0x8000;
+  return b;
+}
+
+/* ------------------------------------------------------------ step 1 */
+int oracle_num_cmp_blocks(const nsa_oracle_params* P, int T) {
+  if (T < P->l) return 0;
+  return (T - P->l) / P->d + 1;
+}
+
+/*
+ * Compressed keys (or values) of one sequence.
+ *   X   [T, Hkv, D] bf16 bits
+ *   W   [Hkv, D, l*D] fp32
+ *   out [C, Hkv, D] fp64 (unrounded) and bf16 (rounded), either may be NULL.
+ */
+void oracle_compress(const nsa_oracle_params* P, int T, const uint16_t* X, const float* W,
+                     double* out_f64, uint16_t* out_bf16) {
+  const int C = oracle_num_cmp_blocks(P, T);
+  const int D = P->D, H = P->Hkv, L = P->l;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int i = 0; i < C; ++i) {
+    for (int h = 0; h < H; ++h) {
+      for (int c = 0; c < D; ++c) {
+        const float* wrow = W + ((size_t)h * D + c) * (size_t)L * D;
+        double acc = 0.0;
+        for (int p = 0; p < L; ++p) {
+          const uint16_t* x = X + ((size_t)(i * P->d + p) * H + h) * D;
+          for (int cc = 0; cc < D; ++cc) acc += (double)wrow[p * D + cc] * oracle_bf16_to_f64(x[cc]);
+        }
+        size_t o = ((size_t)i * H + h) * D + c;
+        if (out_f64) out_f64[o] = acc;
+        if (out_bf16) out_bf16[o] = oracle_f64_to_bf16(acc);
+      }
+    }
+  }
+}
+
+/* ------------------------------------------------------------ softmax attention */
+/*
+ * Softmax attention of one query head over an explicit list of key rows.
+ *   q [D] fp64; keys/vals: bf16 rows of a [*, Hkv, D] tensor, head h.
+ *   Writes o[D], the probabilities p[nk] (may be NULL) and returns the
+ *   log-sum-exp of the scaled logits (-INFINITY when nk == 0, o = 0).
+ */
+static double attend(const nsa_oracle_params* P, const double* q, const uint16_t* keys,
+                     const uint16_t* vals, int h, const int* rows, int nk, double* o, double* p,
+                     double* scratch) {
+  const int D = P->D, H = P->Hkv;
+  for (int c = 0; c < D; ++c) o[c] = 0.0;
+  if (nk == 0) return -INFINITY;
+  double* z = scratch;
+  double zmax = -INFINITY;
+  for (int j = 0; j < nk; ++j) {
+    const uint16_t* k = keys + ((size_t)rows[j] * H + h) * D;
+    double s = 0.0;
+    for (int c = 0; c < D; ++c) s += q[c] * oracle_bf16_to_f64(k[c]);
+    z[j] = P->scale * s;
+    if (z[j] > zmax) zmax = z[j];
+  }
+  double sum = 0.0;
+  for (int j = 0; j < nk; ++j) sum += exp(z[j] - zmax);
+  for (int j = 0; j < nk; ++j) {
+    double pj = exp(z[j] - zmax) / sum;
+    if (p) p[j] = pj;
+    const uint16_t* v = vals + ((size_t)rows[j] * H + h) * D;
+    for (int c = 0; c < D; ++c) o[c] += pj * oracle_bf16_to_f64(v[c]);
+  }
+  return zmax + log(sum);
+}
+
+/* ------------------------------------------------------------ step 4 */
+/*
+ * Top-n of S[0..ncand) under the order (score descending, index ascending).
+ * Writes the chosen indices in ascending order to sel[0..n), -1 padded, and
+ * returns the gap S_(n) - S_(n+1) between the n-th and (n+1)-th ranked
+ * candidates (+INFINITY when every candidate is taken).
+ */
+double oracle_select(const double* S, int ncand, int n, int* sel) {
+  int taken = 0;
+  if (ncand <= n) {
+    for (int j = 0; j < ncand; ++j) sel[taken++] = j;
+    for (int j = taken; j < n; ++j) sel[j] = -1;
+    return INFINITY;
+  }
+  /* selection by repeated maximum; ties keep the lower index */
+  char* used = (char*)calloc((size_t)ncand, 1);
+  double last = 0.0;
+  for (int r = 0; r < n; ++r) {
+    int best = -1;
+    for (int j = 0; j < ncand; ++j) {
+      if (used[j]) continue;
+      if (best < 0 || S[j] > S[best]) best = j;
+    }
+    used[best] = 1;
+    last = S[best];
+  }
+  int next = -1;
+  for (int j = 0; j < ncand; ++j) {
+    if (used[j]) continue;
+    if (next < 0 || S[j] > S[next]) next = j;
+  }
+  for (int j = 0; j < ncand; ++j)
+    if (used[j]) sel[taken++] = j;
+  free(used);
+  return last - S[next];
+}
+
+/* ------------------------------------------------------------ one query */
+/*
+ * The whole forward pass for one query token at (0-based) position t of a
+ * sequence whose keys/values are k, v ([>= t+1, Hkv, D]) and whose stored
+ * compressed keys/values are kc, vc ([>= C(t+1), Hkv, D], bf16).
+ *   q      [Hq, D] bf16 bits, gates [Hq, 3] fp32 (cmp, slc, win)
+ * Outputs (any may be NULL):
+ *   o_cmp, o_slc, o_win, out  [Hq, D]
+ *   lse    [Hq]               log-sum-exp of the compressed branch
+ *   scores [Hkv, cmax]        block scores (entries >= C(t) left 0)
+ *   sel    [Hkv, n]           selected block indices (ascending, -1 pad)
+ *   gap    [Hkv]              n-th minus (n+1)-th ranked score
+ * Returns 0, or -1 on an unsupported geometry.
+ */
+int oracle_nsa_query(const nsa_oracle_params* P, int t, const uint16_t* q, const uint16_t* k,
+                     const uint16_t* v, const uint16_t* kc, const uint16_t* vc,
+                     const float* gates, double* o_cmp, double* o_slc, double* o_win,
+                     double* out, double* lse, double* scores, int cmax, int* sel,
+                     double* gap) {
+  const int D = P->D, Hq = P->Hq, Hkv = P->Hkv, G = Hq / Hkv;
+  if (P->l != P->d || P->lsel != P->l || Hq % Hkv != 0) return -1;
+  /* visible compressed blocks: i*d + l - 1 <= t */
+  const int ncmp = (t + 1 >= P->l) ? (t + 1 - P->l) / P->d + 1 : 0;
+  /* selection candidates: blocks j with j*l' <= t */
+  const int ncand = t / P->lsel + 1;
+  const int maxk = ncmp + P->n * P->lsel + P->w + 1;
+  int* cmp_rows = (int*)malloc(sizeof(int) * (size_t)(ncmp + 1));
+  int* sel_rows = (int*)malloc(sizeof(int) * (size_t)(P->n * P->lsel + 1));
+  int* win_rows = (int*)malloc(sizeof(int) * (size_t)(P->w + 1));
+  double* scratch = (double*)malloc(sizeof(double) * (size_t)maxk);
+  double* prob = (double*)malloc(sizeof(double) * (size_t)(ncmp + 1));
+  double* S = (double*)malloc(sizeof(double) * (size_t)ncand);
+  int* chosen = (int*)malloc(sizeof(int) * (size_t)P->n);
+  double* qh = (double*)malloc(sizeof(double) * (size_t)D);
+  double* oc = (double*)malloc(sizeof(double) * (size_t)G * D);
+  double* os = (double*)malloc(sizeof(double) * (size_t)D);
+  double* ow = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int i = 0; i < ncmp; ++i) cmp_rows[i] = i;
+
+  for (int g = 0; g < Hkv; ++g) {
+    /* step 2 and 3: compressed branch of every head of the group, and the
+       block scores summed over those heads */
+    for (int j = 0; j < ncand; ++j) S[j] = 0.0;
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      for (int c = 0; c < D; ++c) qh[c] = oracle_bf16_to_f64(q[(size_t)h * D + c]);
+      double L = attend(P, qh, kc, vc, g, cmp_rows, ncmp, oc + (size_t)hh * D, prob, scratch);
+      if (lse) lse[h] = L;
+      for (int i = 0; i < ncmp; ++i) S[i] += prob[i]; /* l == d == l' */
+    }
+    if (scores) {
+      for (int j = 0; j < cmax; ++j) scores[(size_t)g * cmax + j] = (j < ncmp) ? S[j] : 0.0;
+    }
+    /* step 4 */
+    double gp = oracle_select(S, ncand, P->n, chosen);
+    if (gap) gap[g] = gp;
+    if (sel) memcpy(sel + (size_t)g * P->n, chosen, sizeof(int) * (size_t)P->n);
+    /* step 5 keys: tokens u <= t inside the chosen blocks */
+    int nsel = 0;
+    for (int r = 0; r < P->n; ++r) {
+      int j = chosen[r];
+      if (j < 0) continue;
+      for (int u = j * P->lsel; u < (j + 1) * P->lsel; ++u)
+        if (u <= t) sel_rows[nsel++] = u;
+    }
+    /* step 6 keys: the w tokens ending at t */
+    int nwin = 0;
+    for (int u = (t - P->w + 1 > 0 ? t - P->w + 1 : 0); u <= t; ++u) win_rows[nwin++] = u;
+
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      for (int c = 0; c < D; ++c) qh[c] = oracle_bf16_to_f64(q[(size_t)h * D + c]);
+      attend(P, qh, k, v, g, sel_rows, nsel, os, NULL, scratch);
+      attend(P, qh, k, v, g, win_rows, nwin, ow, NULL, scratch);
+      /* step 7 */
+      const double g0 = gates[h * 3 + 0], g1 = gates[h * 3 + 1], g2 = gates[h * 3 + 2];
+      for (int c = 0; c < D; ++c) {
+        const size_t o = (size_t)h * D + c;
+        const double ocv = oc[(size_t)hh * D + c];
+        if (o_cmp) o_cmp[o] = ocv;
+        if (o_slc) o_slc[o] = os[c];
+        if (o_win) o_win[o] = ow[c];
+        if (out) out[o] = g0 * ocv + g1 * os[c] + g2 * ow[c];
+      }
+    }
+  }
+  free(cmp_rows);
+  free(sel_rows);
+  free(win_rows);
+  free(scratch);
+  free(prob);
+  free(S);
+  free(chosen);
+  free(qh);
+  free(oc);
+  free(os);
+  free(ow);
+  return 0;
+}
+
+/*
+ * oracle_nsa_query for a list of rows of one packed sequence (prefill):
+ *   q [T, Hq, D], k, v [T, Hkv, D], kc, vc [C, Hkv, D], gates [T, Hq, 3];
+ *   output arrays are indexed by the position in `rows`.
+ */
+int oracle_nsa_rows(const nsa_oracle_params* P, int T, const uint16_t* q, const uint16_t* k,
+                    const uint16_t* v, const uint16_t* kc, const uint16_t* vc,
+                    const float* gates, const int* rows, int nrows, double* o_cmp,
+                    double* o_slc, double* o_win, double* out, double* lse, double* scores,
+                    int cmax, int* sel, double* gap) {
+  const int D = P->D, Hq = P->Hq, Hkv = P->Hkv;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int r = 0; r < nrows; ++r) {
+    const int t = rows[r];
+    if (t < 0 || t >= T) {
+      bad |= 1;
+      continue;
+    }
+    const size_t hd = (size_t)Hq * D;
+    int rc = oracle_nsa_query(
+        P, t, q + (size_t)t * hd, k, v, kc, vc, gates + (size_t)t * Hq * 3,
+        o_cmp ? o_cmp + r * hd : NULL, o_slc ? o_slc + r * hd : NULL,
+        o_win ? o_win + r * hd : NULL, out ? out + r * hd : NULL,
+        lse ? lse + (size_t)r * Hq : NULL, scores ? scores + (size_t)r * Hkv * cmax : NULL, cmax,
+        sel ? sel + (size_t)r * Hkv * P->n : NULL, gap ? gap + (size_t)r * Hkv : NULL);
+    bad |= (rc != 0);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * Step 4 alone over a batch of score rows given in fp32 (used to replay the
+ * selection on scores produced elsewhere): S [nrows, cstride], candidate
+ * counts ncand [nrows]; entries at or beyond the complete-block count cmp_n
+ * [nrows] are treated as 0 (the incomplete block).
+ */
+void oracle_select_f32(const float* S, int nrows, int cstride, const int* ncand,
+                       const int* cmp_n, int n, int* sel, double* gap) {
+#pragma omp parallel for schedule(static)
+  for (int r = 0; r < nrows; ++r) {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(ncand[r] > 0 ? ncand[r] : 1));
+    for (int j = 0; j < ncand[r]; ++j) s[j] = (j < cmp_n[r]) ? (double)S[(size_t)r * cstride + j] : 0.0;
+    double gp = oracle_select(s, ncand[r], n, sel + (size_t)r * n);
+    if (gap) gap[r] = gp;
+    free(s);
+  }
+}
