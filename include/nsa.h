@@ -1,0 +1,183 @@
+/*
+ * nsa.h - C ABI of the B200 (sm_100a) Native Sparse Attention forward pass.
+ *
+ * What is computed (for every query token t of every sequence, every query
+ * head h of KV group g = h / G, G = Hq / Hkv; positions restart at 0 in each
+ * sequence; s = softmax_scale):
+ *   1. compression ("DeepSeek NSA config.toml" page, section 3,
+ *      compress_block_size; "DeepSeek NSA in manufacturing" page, section on
+ *      what dynamic sparsity sparsifies: one learned linear map over each
+ *      flattened key block):
+ *        Kc[i,g,:] = W_K[g] . vec(K[i*l .. i*l+l-1, g, :]),  Vc likewise,
+ *      vec index p*D + c (token p of the block, channel c), stored in bf16;
+ *   2. compressed branch (config page, section 1): softmax over the complete
+ *      blocks i (i*l + l - 1 <= t) of s * q_h . Kc[i,g]; O_cmp = sum p Vc;
+ *   3. block scores (manufacturing page, same section: coarse attention of
+ *      the query to every compressed block ranks the blocks):
+ *        S[t,g,j] = sum over the G heads of group g of p_h[j];
+ *   4. selection (config page, section 3, select_top_k): the top_n blocks
+ *      among j*l <= t by (score descending, index ascending); the block
+ *      holding t, while incomplete, competes with score 0;
+ *   5. selected branch (config page, section 3, select_block_size): softmax
+ *      attention over the tokens u <= t of the chosen blocks;
+ *   6. window branch (config page, section 3, sliding_window): softmax
+ *      attention over u in [max(0, t-w+1), t];
+ *   7. gate (config page, sections 1 and 3, gate_type learned):
+ *        out = g_cmp * O_cmp + g_slc * O_slc + g_win * O_win,
+ *      with the gate values given per token and head (post-sigmoid).
+ * An empty branch contributes 0.  This version supports l == d == l'
+ * (compress block == stride == select block) in {32, 64}, head_dim in
+ * {64, 128}, G in {1, 2, 4, 8, 16}, 1 <= top_n <= 64, window >= 1.
+ *
+ * Memory: every pointer except the plan is caller-owned device memory (bf16
+ * is passed as raw 16-bit storage).  The library never allocates device
+ * memory in nsa_prefill / nsa_decode; scratch lives in the caller's workspace
+ * (nsa_workspace_size).  Device pointers must be 16-byte aligned; row strides
+ * are the dense strides implied by the shapes.
+ *
+ * Errors: every call returns an nsa_status.  Arguments are validated on the
+ * host before anything is launched; on error nothing is launched.  Launches
+ * are asynchronous on `stream` (a cudaStream_t; NULL is the legacy default
+ * stream) and never synchronise the host.  Faults found on the device (a
+ * bounded wait that gave up, inconsistent sequence lengths) are recorded in a
+ * status word inside the workspace, read back with nsa_read_device_status.
+ * There is no fallback path: an unsupported geometry is an error.
+ */
+#ifndef NSA_B200_H
+#define NSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NSA_OK = 0,
+  NSA_ERR_INVALID_ARG = 1,    /* null pointer, negative size, inconsistent shape */
+  NSA_ERR_UNSUPPORTED = 2,    /* valid NSA geometry this build does not implement */
+  NSA_ERR_MISALIGNED = 3,     /* a device pointer is not 16-byte aligned */
+  NSA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than nsa_workspace_size */
+  NSA_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+  NSA_ERR_DEVICE_TIMEOUT = 6, /* device status: a bounded wait gave up */
+  NSA_ERR_DEVICE_BAD_INPUT = 7 /* device status: sequence lengths out of range */
+} nsa_status;
+
+typedef enum { NSA_OUT_BF16 = 0, NSA_OUT_F32 = 1 } nsa_out_dtype;
+typedef enum { NSA_MODE_PREFILL = 0, NSA_MODE_DECODE = 1 } nsa_mode;
+
+typedef struct {
+  int head_dim;          /* D = d_k = d_v: 64 or 128 */
+  int num_q_heads;       /* Hq */
+  int num_kv_heads;      /* Hkv; Hq / Hkv must be 1, 2, 4, 8 or 16 */
+  int cmp_block;         /* l  (compress_block_size) */
+  int cmp_stride;        /* d  (compression stride; must equal l here) */
+  int sel_block;         /* l' (select_block_size; must equal l here) */
+  int top_n;             /* n  (select_top_k) */
+  int window;            /* w  (sliding_window) */
+  float softmax_scale;   /* s; 0 selects 1/sqrt(D) */
+  int max_batch;         /* upper bound on sequences per call */
+  int max_seqlen;        /* upper bound on one sequence's length (prefill) or
+                            on the cache capacity (decode) */
+  int max_total_tokens;  /* upper bound on packed tokens per prefill call */
+  int out_dtype;         /* nsa_out_dtype of `out` */
+} nsa_params;
+
+typedef struct nsa_plan_s* nsa_plan_t;
+
+/* Validates `params` and creates a plan (host memory only, no GPU work).
+ * Returns NSA_ERR_INVALID_ARG / NSA_ERR_UNSUPPORTED without creating one.
+ * A plan is immutable; it may be shared by calls on several streams as long
+ * as each concurrent call has its own workspace. */
+int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out);
+void nsa_plan_destroy(nsa_plan_t plan);
+
+/* Bytes of device workspace a call of `mode` needs under the plan's bounds
+ * (0 for an invalid plan or mode). */
+size_t nsa_workspace_size(nsa_plan_t plan, int mode);
+
+/* Named regions of the prefill workspace, for inspection by tests and
+ * debugging.  Valid after a completed nsa_prefill on that workspace. */
+typedef enum {
+  NSA_WS_STATUS = 0,  /* int32 status word */
+  NSA_WS_O_CMP = 1,   /* fp32 [T_total, Hq, D] compressed-branch output */
+  NSA_WS_LSE = 2,     /* fp32 [T_total, Hq] compressed-branch log-sum-exp (natural log) */
+  NSA_WS_SCORES = 3,  /* fp32 [T_total, Hkv, max_seqlen / l] block scores; entry j
+                         of row t is defined for j < number of complete blocks */
+  NSA_WS_SEL = 4      /* int32 [T_total, Hkv, top_n] selection (when sel_idx is NULL) */
+} nsa_ws_region;
+int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, size_t* bytes);
+
+/* Rows of the packed compressed-KV output of a prefill over `total_tokens`
+ * tokens: floor(total_tokens / l), an upper bound on sum_b floor(T_b / l). */
+int nsa_cmp_rows(nsa_plan_t plan, int total_tokens);
+
+/*
+ * Causal prefill over a packed batch (steps 1-7 for every token).
+ *   q          [T_total, Hq, D]  bf16
+ *   k, v       [T_total, Hkv, D] bf16
+ *   gates      [T_total, Hq, 3]  fp32, order (cmp, slc, win)
+ *   w_k, w_v   [Hkv, D, l*D]     fp32 compressor weights
+ *   cu_seqlens [batch + 1]       int32 device, cu_seqlens[0] = 0, non-decreasing,
+ *                                cu_seqlens[batch] = total_tokens, each length <= max_seqlen
+ *   out        [T_total, Hq, D]  bf16 or fp32 (plan out_dtype)
+ *   k_cmp, v_cmp [nsa_cmp_rows, Hkv, D] bf16, written: the compressed keys and
+ *              values of sequence b occupy rows sum_{b'<b} floor(T_b'/l) onward
+ *   sel_idx    [T_total, Hkv, top_n] int32 or NULL: selected block indices of
+ *              each token, ascending, -1 padded
+ *   workspace  >= nsa_workspace_size(plan, NSA_MODE_PREFILL) bytes, 256-byte aligned
+ */
+int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,
+                const float* gates, const float* w_k, const float* w_v,
+                const int* cu_seqlens, int batch, int total_tokens, void* out, void* k_cmp,
+                void* v_cmp, int* sel_idx, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/*
+ * One decode step for a batch of sequences (steps 1-7 for the newest token of
+ * each sequence, which the caller has already written into the caches).
+ *   q           [batch, Hq, D]             bf16, query of the newest token
+ *   k_cache, v_cache [batch, cache_capacity, Hkv, D] bf16
+ *   k_cmp_cache, v_cmp_cache [batch, cache_capacity / l, Hkv, D] bf16: the
+ *               compressed blocks of every complete block before the newest
+ *               token; when the newest token completes a block (len % l == 0)
+ *               that block is compressed here from the cache and written back
+ *   seqlens     [batch] int32 device, tokens in the cache including the newest,
+ *               1 <= len <= cache_capacity
+ *   cache_capacity  multiple of l, <= plan max_seqlen
+ *   gates       [batch, Hq, 3] fp32
+ *   w_k, w_v    [Hkv, D, l*D] fp32
+ *   out         [batch, Hq, D] bf16 or fp32
+ *   sel_idx     [batch, Hkv, top_n] int32 or NULL
+ *   workspace   >= nsa_workspace_size(plan, NSA_MODE_DECODE) bytes
+ */
+int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* v_cache,
+               void* k_cmp_cache, void* v_cmp_cache, const int* seqlens, int batch,
+               int cache_capacity, const float* gates, const float* w_k, const float* w_v,
+               void* out, int* sel_idx, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, returns the device status word of the last call that
+ * used `workspace` (NSA_OK or NSA_ERR_DEVICE_*), and clears it.  Meant for
+ * tests and debugging; returns NSA_ERR_CUDA if the stream itself failed. */
+int nsa_read_device_status(const void* workspace, void* stream);
+
+/* Launches one CTA whose bounded wait on an mbarrier that nothing signals
+ * gives up after about `cycles` SM cycles and records NSA_ERR_DEVICE_TIMEOUT
+ * in the workspace status word.  Exercises the timeout path without faulting
+ * or hanging the GPU (tests only). */
+int nsa_selftest_timeout(void* workspace, size_t workspace_bytes, long long cycles,
+                         void* stream);
+
+/* Static description of a status code. */
+const char* nsa_strerror(int status);
+
+/* Number of kernel launches made by the last successful nsa_prefill /
+ * nsa_decode call on this thread (for launch accounting in benchmarks). */
+int nsa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_B200_H */

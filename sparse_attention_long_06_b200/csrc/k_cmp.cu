@@ -1,0 +1,437 @@
+// Compressed-branch attention and block scores (steps 2 and 3).
+//
+//   step 2 ("DeepSeek NSA config.toml" page, section 1: the compressed branch
+//   gives coarse global context): per query head, softmax over the complete
+//   compressed blocks of s * q . Kc, output O_cmp = sum p Vc;
+//   step 3 ("DeepSeek NSA in manufacturing" page, section on what dynamic
+//   sparsity sparsifies: the query's coarse attention to every compressed
+//   block ranks the blocks): S[t, g, j] = sum over the heads of group g of p.
+//
+// One persistent CTA per SM walks dense tiles of 128 MMA rows = (128 / G)
+// consecutive tokens x the G query heads of one KV group.  The compressed
+// keys are shared by all rows, so every product is a full 128 x 128 tcgen05
+// tile.  Two passes over the compressed keys of the tile:
+//   pass 1: S = Q Kc^T (rows = (token, head) on TMEM lanes): running max and
+//           sum per row -> log-sum-exp;
+//   pass 2: S^T = Kc Q^T (keys on TMEM lanes, (token, head) on columns):
+//           p = exp(s - lse) is exact, the G columns of a token sum to its
+//           block score inside one thread, P^T goes to shared memory as the
+//           MN-major A operand of O = P Vc (accumulated in TMEM).
+// Warp roles: 0 = TMA producer, 1 = tcgen05.mma issuer, 2..5 = softmax and
+// epilogue (thread i of warp w owns TMEM lane 32 * (w % 4) + i).
+#include <cuda_bf16.h>
+
+#include "nsa_internal.cuh"
+#include "sm100.cuh"
+
+namespace nsa {
+using namespace sm100;
+
+namespace {
+
+template <int D>
+struct CmpLayout {
+  static constexpr int kStages = 3;
+  static constexpr int kQBytes = kTileRows * D * 2;   // 128 rows
+  static constexpr int kChunkBytes = kChunk * D * 2;  // 128 keys
+  static constexpr int kPBytes = kChunk * kTileRows * 2;
+  static constexpr int kQ = 0;                                   // 2 buffers
+  static constexpr int kRing = kQ + 2 * kQBytes;                 // kStages
+  static constexpr int kP = kRing + kStages * kChunkBytes;       // P^T
+  static constexpr int kLse = kP + kPBytes;                      // float[128]
+  static constexpr int kBars = kLse + 128 * 4;                   // barriers
+  static constexpr int kEnd = kBars + 32 * 8 + 16;
+  // at least 116 KB so that one CTA owns an SM (it allocates all 512 TMEM columns)
+  static constexpr int kSmem = (kEnd + 1024 > 118 * 1024) ? kEnd + 1024 : 118 * 1024;
+};
+
+struct CmpItem {
+  int valid, b, g, t0, T, row0, nc, cmp0;
+};
+
+__device__ __forceinline__ CmpItem cmp_item(const PrefillArgs& a, int k) {
+  CmpItem it{};
+  const int tiles = a.meta->tiles_total, H = a.geo.Hkv;
+  if (k >= tiles * H) return it;
+  it.valid = 1;
+  const int tau = tiles - 1 - k / H;  // heaviest (latest) tiles first
+  it.g = k % H;
+  it.b = seq_of_offset(a.tile_off, a.batch, tau);
+  it.t0 = (tau - a.tile_off[it.b]) * a.geo.tpt;
+  const int c0 = __ldg(a.cu + it.b);
+  it.T = __ldg(a.cu + it.b + 1) - c0;
+  it.row0 = c0 + it.t0;
+  const int tend = min(it.t0 + a.geo.tpt, it.T);
+  const int ncmp_max = tend / a.geo.l;  // (t + 1) / l at t = tend - 1
+  it.nc = (ncmp_max + kChunk - 1) / kChunk;
+  it.cmp0 = a.cmp_off[it.b];
+  return it;
+}
+
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    nsa_cmp_attn_kernel(const __grid_constant__ PrefillArgs a,
+                        const __grid_constant__ PrefillMaps maps) {
+  using L = CmpLayout<D>;
+  constexpr int KSTEPS = D / 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
+  uint64_t* q_full = bars + 0;     // [2]
+  uint64_t* q_empty = bars + 2;    // [2]
+  uint64_t* st_full = bars + 4;    // [3]
+  uint64_t* st_empty = bars + 7;   // [3]
+  uint64_t* s_full = bars + 10;    // [2]
+  uint64_t* s_empty = bars + 12;   // [2]
+  uint64_t* p_full = bars + 14;
+  uint64_t* p_empty = bars + 15;
+  uint64_t* o_full = bars + 16;
+  uint64_t* o_empty = bars + 17;
+  uint64_t* fin = bars + 18;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
+  float* lse_s = reinterpret_cast<float*>(sm + L::kLse);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (a.meta->bad) return;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(q_full + i, 1);
+      mbar_init(q_empty + i, 1);
+      mbar_init(s_full + i, 1);
+      mbar_init(s_empty + i, 4);
+    }
+    for (int i = 0; i < L::kStages; ++i) {
+      mbar_init(st_full + i, 1);
+      mbar_init(st_empty + i, 1);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(p_empty, 1);
+    mbar_init(o_full, 1);
+    mbar_init(o_empty, 4);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(sm);
+  int* status = a.status;
+  const int G = a.geo.G, l = a.geo.l;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.kc);
+      tma_prefetch_desc(&maps.vc);
+      int qc = 0, sc = 0;
+      bool ok = true;
+      auto load_chunk = [&](const CUtensorMap* map, const CmpItem& it, int c) {
+        const int s = sc % L::kStages, u = sc / L::kStages;
+        if (u > 0 && !mbar_wait(st_empty + s, (u - 1) & 1, abort_flag, status, kWaitCycles)) {
+          ok = false;
+          return;
+        }
+        uint8_t* dst = sm + L::kRing + s * L::kChunkBytes;
+        mbar_arrive_expect_tx(st_full + s, L::kChunkBytes);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(dst + h * 16384, map, st_full + s, h * 64, it.g, it.cmp0 + c * kChunk);
+        ++sc;
+      };
+      for (int k = blockIdx.x; ok; k += gridDim.x) {
+        const CmpItem it = cmp_item(a, k);
+        if (!it.valid) break;
+        if (it.nc == 0) continue;
+        const int qb = qc & 1, u = qc >> 1;
+        if (u > 0 && !mbar_wait(q_empty + qb, (u - 1) & 1, abort_flag, status, kWaitCycles)) break;
+        mbar_arrive_expect_tx(q_full + qb, L::kQBytes);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_3d(sm + L::kQ + qb * L::kQBytes + h * 16384, &maps.q, q_full + qb, h * 64,
+                      it.g * G, it.row0);
+        ++qc;
+        for (int c = 0; c < it.nc && ok; ++c) load_chunk(&maps.kc, it, c);
+        if (ok) load_chunk(&maps.kc, it, 0);
+        for (int c = 0; c < it.nc && ok; ++c) {
+          if (c + 1 < it.nc) load_chunk(&maps.kc, it, c + 1);
+          if (ok) load_chunk(&maps.vc, it, c);
+        }
+      }
+      // drain: every issued copy has landed before the CTA retires (also
+      // after an abort, hence a private never-set abort flag)
+      volatile int never = 0;
+      for (int s = 0; s < L::kStages && s < sc; ++s) {
+        const int last = sc - 1 - ((sc - 1 - s) % L::kStages);
+        mbar_wait(st_full + s, (last / L::kStages) & 1, &never, nullptr, kWaitCycles / 4);
+      }
+      for (int qb = 0; qb < 2 && qb < qc; ++qb) {
+        const int last = qc - 1 - ((qc - 1 - qb) % 2);
+        mbar_wait(q_full + qb, (last >> 1) & 1, &never, nullptr, kWaitCycles / 4);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t id_pv = idesc_bf16(128, D, true, true);
+      int qc = 0, sc = 0, sbc = 0, pc = 0, oc = 0;
+      bool ok = true;
+      // S[buf] = A . B^T with both operands K-major, 128-byte swizzled tiles
+      auto qk = [&](bool a_is_stage, int qb) {
+        const int s = sc % L::kStages;
+        if (!mbar_wait(st_full + s, (sc / L::kStages) & 1, abort_flag, status, kWaitCycles)) {
+          ok = false;
+          return;
+        }
+        const int buf = sbc & 1, u = sbc >> 1;
+        if (u > 0 && !mbar_wait(s_empty + buf, (u - 1) & 1, abort_flag, status, kWaitCycles)) {
+          ok = false;
+          return;
+        }
+        tc_fence_after();
+        const uint32_t stage = sbase + L::kRing + s * L::kChunkBytes;
+        const uint32_t qbuf = sbase + L::kQ + qb * L::kQBytes;
+        const uint32_t A = a_is_stage ? stage : qbuf;
+        const uint32_t B = a_is_stage ? qbuf : stage;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+          const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16_ss(tmem + buf * 128, smem_desc(A + off, 16, 1024, kLayoutSw128),
+                      smem_desc(B + off, 16, 1024, kLayoutSw128), id_qk, ks > 0);
+        }
+        mma_commit(st_empty + s);
+        mma_commit(s_full + buf);
+        ++sc;
+        ++sbc;
+      };
+      auto pv = [&](int c) {
+        const int s = sc % L::kStages;
+        if (!mbar_wait(st_full + s, (sc / L::kStages) & 1, abort_flag, status, kWaitCycles) ||
+            !mbar_wait(p_full, pc & 1, abort_flag, status, kWaitCycles)) {
+          ok = false;
+          return;
+        }
+        if (c == 0 && oc > 0 && !mbar_wait(o_empty, (oc - 1) & 1, abort_flag, status, kWaitCycles)) {
+          ok = false;
+          return;
+        }
+        tc_fence_after();
+        const uint32_t stage = sbase + L::kRing + s * L::kChunkBytes;
+        const uint32_t P = sbase + L::kP;
+#pragma unroll
+        for (int ks = 0; ks < kChunk / 16; ++ks)
+          mma_bf16_ss(tmem + 256, smem_desc(P + ks * 2048, 16384, 1024, kLayoutSw128),
+                      smem_desc(stage + ks * 2048, 16384, 1024, kLayoutSw128), id_pv,
+                      (c > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(st_empty + s);
+        mma_commit(p_empty);
+        ++sc;
+        ++pc;
+      };
+      for (int k = blockIdx.x; ok; k += gridDim.x) {
+        const CmpItem it = cmp_item(a, k);
+        if (!it.valid) break;
+        if (it.nc == 0) continue;
+        const int qb = qc & 1;
+        if (!mbar_wait(q_full + qb, (qc >> 1) & 1, abort_flag, status, kWaitCycles)) break;
+        for (int c = 0; c < it.nc && ok; ++c) qk(false, qb);  // pass 1: S = Q Kc^T
+        if (ok) qk(true, qb);  // pass 2: S^T = Kc Q^T
+        for (int c = 0; c < it.nc && ok; ++c) {
+          if (c + 1 < it.nc) qk(true, qb);
+          if (ok) pv(c);
+        }
+        if (!ok) break;
+        mma_commit(o_full);
+        mma_commit(q_empty + qb);
+        ++oc;
+        ++qc;
+      }
+      mma_commit(fin);
+      volatile int never = 0;
+      mbar_wait(fin, 0, &never, nullptr, kWaitCycles / 4);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;  // TMEM lane owned by this thread
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const float sl2 = a.geo.scale_log2;
+    const int Hq = a.geo.Hq, Hkv = a.geo.Hkv, cap = a.geo.cmp_cap;
+    int sbc = 0, pc = 0, oc = 0;
+    for (int k = blockIdx.x;; k += gridDim.x) {
+      const CmpItem it = cmp_item(a, k);
+      if (!it.valid) break;
+      const int i_row = r / G, h_row = r % G;
+      const int t_row = it.t0 + i_row;
+      const bool row_ok = t_row < it.T;
+      const int ncmp_row = row_ok ? (t_row + 1) / l : 0;
+      const size_t orow = ((size_t)(it.row0 + i_row) * Hq + it.g * G + h_row);
+      if (it.nc == 0) {
+        if (row_ok && !*abort_flag) {
+          float4* o = reinterpret_cast<float4*>(a.o_cmp + orow * D);
+          for (int j = 0; j < D / 4; ++j) o[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          a.lse[orow] = -INFINITY;
+        }
+        continue;
+      }
+      // ---- pass 1: running max / sum per row
+      float m = -INFINITY, lsum = 0.f;
+      for (int c = 0; c < it.nc; ++c) {
+        const int buf = sbc & 1;
+        mbar_wait(s_full + buf, (sbc >> 1) & 1, abort_flag, status, kWaitCycles);
+        tc_fence_after();
+        float x[kChunk];
+#pragma unroll
+        for (int grp = 0; grp < kChunk / 16; ++grp) {
+          float v[16];
+          tmem_ld16(lane_addr + buf * 128 + grp * 16, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[grp * 16 + j] = v[j];
+        }
+        tmem_ld_wait();
+        float cm = -INFINITY;
+        const int jmax = ncmp_row - c * kChunk;  // columns j < jmax are visible blocks
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+          x[j] = j < jmax ? x[j] * sl2 : -INFINITY;
+          cm = fmaxf(cm, x[j]);
+        }
+        const float mn = fmaxf(m, cm);
+        if (mn != -INFINITY) {
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) s += ex2(x[j] - mn);
+          lsum = lsum * ex2(m - mn) + s;
+          m = mn;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty + buf);
+        ++sbc;
+      }
+      const float lse2 = lsum > 0.f ? m + __log2f(lsum) : -INFINITY;
+      softmax_bar();  // every thread is done reading lse_s of the previous tile
+      lse_s[r] = lse2;
+      softmax_bar();
+      // ---- pass 2: this thread owns key r of every chunk
+      for (int c = 0; c < it.nc; ++c) {
+        const int buf = sbc & 1;
+        mbar_wait(s_full + buf, (sbc >> 1) & 1, abort_flag, status, kWaitCycles);
+        tc_fence_after();
+        if (pc > 0) mbar_wait(p_empty, (pc - 1) & 1, abort_flag, status, kWaitCycles);
+        const int key = c * kChunk + r;
+        // rows (token, head) that see compressed block `key`: tokens t with
+        // (t + 1) / l > key, inside the sequence
+        const int tok_lo = max(0, (key + 1) * l - 1 - it.t0);
+        const int tok_hi = min(a.geo.tpt, it.T - it.t0);
+        const int row_lo = tok_lo * G, row_hi = tok_hi * G;
+        const uint32_t prow = sbase + L::kP + (key & 127) / 8 * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int grp = 0; grp < kTileRows / 16; ++grp) {
+          float v[16];
+          tmem_ld16(lane_addr + buf * 128 + grp * 16, v);
+          tmem_ld_wait();
+          float p[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int row = grp * 16 + j;
+            p[j] = (row >= row_lo && row < row_hi) ? ex2(v[j] * sl2 - lse_s[row]) : 0.f;
+          }
+          // block score of each token whose heads lie in this group of 16 rows
+          for (int j0 = 0; j0 < 16; j0 += G) {
+            const int row = grp * 16 + j0;
+            const int tok = row / G;
+            if (row >= row_lo && row < row_hi) {
+              float s = 0.f;
+              for (int j = j0; j < j0 + G; ++j) s += p[j];
+              if (!*abort_flag)
+                a.scores[((size_t)(it.row0 + tok) * Hkv + it.g) * cap + key] = s;
+            }
+          }
+          uint32_t pk[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int cidx = grp * 2 + cc;
+            const uint32_t addr = prow + (cidx >> 3) * 16384 + (((cidx & 7) ^ (r & 7)) << 4);
+            st_shared_v4(addr, pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(s_empty + buf);
+          mbar_arrive(p_full);
+        }
+        ++sbc;
+        ++pc;
+      }
+      // ---- epilogue: O_cmp row and log-sum-exp
+      mbar_wait(o_full, oc & 1, abort_flag, status, kWaitCycles);
+      tc_fence_after();
+#pragma unroll
+      for (int grp = 0; grp < D / 16; ++grp) {
+        float v[16];
+        tmem_ld16(lane_addr + 256 + grp * 16, v);
+        tmem_ld_wait();
+        if (row_ok && !*abort_flag) {
+          float4* o = reinterpret_cast<float4*>(a.o_cmp + orow * D + grp * 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+      if (row_ok && !*abort_flag) a.lse[orow] = lse2 * 0.6931471805599453f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_empty);
+      ++oc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_cmp_attn_t(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
+                              cudaStream_t s) {
+  using L = CmpLayout<D>;
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(nsa_cmp_attn_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int grid = num_sms < kMaxPersistentCtas ? num_sms : kMaxPersistentCtas;
+  nsa_cmp_attn_kernel<D><<<grid, 192, L::kSmem, s>>>(a, m);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
+                            cudaStream_t s) {
+  return a.geo.D == 128 ? launch_cmp_attn_t<128>(a, m, num_sms, s)
+                        : launch_cmp_attn_t<64>(a, m, num_sms, s);
+}
+
+}  // namespace nsa

@@ -1,0 +1,285 @@
+// Small prefill kernels: per-call metadata, block compression (step 1) and
+// top-n block selection (step 4).
+//
+// Compression follows the NSA pages: "DeepSeek NSA config.toml" page,
+// section 3 (compress_block_size) and "DeepSeek NSA in manufacturing" page,
+// section on what dynamic sparsity sparsifies (each block is flattened and
+// mapped by one learned linear layer to a single compressed token).
+// Selection follows the config page, section 3 (select_top_k), and the
+// manufacturing page, same section (the highest-scoring blocks are kept).
+#include <cuda_bf16.h>
+
+#include "nsa_internal.cuh"
+#include "sm100.cuh"
+
+namespace nsa {
+
+// ------------------------------------------------------------------ metadata
+// One thread scans cu_seqlens: compressed-row and tile offsets per sequence,
+// and a consistency check (lengths within [0, max_seqlen], totals match).
+__global__ void nsa_meta_kernel(PrefillArgs a, int max_seqlen) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  const int B = a.batch;
+  int bad = (__ldg(a.cu) != 0);
+  int c = 0, tl = 0;
+  a.cmp_off[0] = 0;
+  a.tile_off[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    const int T = __ldg(a.cu + b + 1) - __ldg(a.cu + b);
+    if (T < 0 || T > max_seqlen) {
+      bad = 1;
+      break;
+    }
+    c += T / a.geo.l;
+    tl += (T + a.geo.tpt - 1) / a.geo.tpt;
+    a.cmp_off[b + 1] = c;
+    a.tile_off[b + 1] = tl;
+  }
+  if (!bad && __ldg(a.cu + B) != a.total_tokens) bad = 1;
+  a.meta->bad = bad;
+  a.meta->cmp_total = bad ? 0 : c;
+  a.meta->tiles_total = bad ? 0 : tl;
+  if (bad) atomicCAS(a.status, 0, sm100::kDeviceBadInputCode);
+}
+
+cudaError_t launch_meta(const PrefillArgs& a, cudaStream_t s) {
+  // max_seqlen == cmp_cap * l (the plan rounds it down to a block multiple)
+  nsa_meta_kernel<<<1, 32, 0, s>>>(a, a.geo.cmp_cap * a.geo.l);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ compression
+// Kc[r, h, c] = sum_{p < l, c' < D} W[h, c, p*D + c'] * X[tok0(r) + p, h, c']
+// for every complete block r of every sequence (tok0 = first token of the
+// block).  A tiled fp32 GEMM: CTA tile 32 blocks x D outputs, k-step 32.
+// Rows in [cmp_total, cmp_rows) are zero-filled so that later tiles reading
+// past the last sequence see finite values.
+template <int D>
+__global__ void __launch_bounds__(256) nsa_compress_kernel(PrefillArgs a) {
+  if (a.meta->bad) return;
+  constexpr int BM = 32, BK = 32, TN = D / 32;
+  const int l = a.geo.l, H = a.geo.Hkv;
+  const int h = blockIdx.y;
+  const bool is_v = blockIdx.z != 0;
+  const uint16_t* X = is_v ? a.v : a.k;
+  const float* W = (is_v ? a.w_v : a.w_k) + (size_t)h * D * l * D;
+  uint16_t* out = is_v ? a.v_cmp : a.k_cmp;
+  const int C = a.meta->cmp_total;
+  const int r0 = blockIdx.x * BM;
+  if (r0 >= a.cmp_rows) return;
+
+  __shared__ int tok0[BM];
+  __shared__ float As[BK][BM + 4];
+  __shared__ float Ws[BK][D + 4];
+  const int tid = threadIdx.x;
+  if (tid < BM) {
+    const int r = r0 + tid;
+    int t0 = -1;
+    if (r < C) {
+      const int b = seq_of_offset(a.cmp_off, a.batch, r);
+      t0 = __ldg(a.cu + b) + (r - a.cmp_off[b]) * l;
+    }
+    tok0[tid] = t0;
+  }
+  __syncthreads();
+
+  const int ty = tid / 32, tx = tid % 32;  // rows ty*4..+4, cols tx*TN..+TN
+  float acc[4][TN];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+
+  const int K = l * D;
+  for (int k0 = 0; k0 < K; k0 += BK) {
+    const int p = k0 / D, c0 = k0 % D;
+    {  // A tile: 32 rows x 32 k, 4 consecutive k per thread
+      const int row = tid / 8, kk = (tid % 8) * 4;
+      const int t0 = tok0[row];
+      float v4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (t0 >= 0) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(X + ((size_t)(t0 + p) * H + h) * D + c0 + kk);
+        v4[0] = __uint_as_float(raw.x << 16);
+        v4[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+        v4[2] = __uint_as_float(raw.y << 16);
+        v4[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) As[kk + j][row] = v4[j];
+    }
+#pragma unroll
+    for (int it = 0; it < D * BK / 4 / 256; ++it) {  // W tile: D rows x 32 k
+      const int idx = it * 256 + tid;
+      const int c = idx / 8, kq = (idx % 8) * 4;
+      const float4 w4 = __ldg(reinterpret_cast<const float4*>(W + (size_t)c * K + k0 + kq));
+      Ws[kq + 0][c] = w4.x;
+      Ws[kq + 1][c] = w4.y;
+      Ws[kq + 2][c] = w4.z;
+      Ws[kq + 3][c] = w4.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < BK; ++kk) {
+      float av[4], bv[TN];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < TN; ++j) bv[j] = Ws[kk][tx * TN + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = r0 + ty * 4 + i;
+    if (r >= a.cmp_rows) continue;
+    const bool live = r < C;
+#pragma unroll
+    for (int j = 0; j < TN; ++j) {
+      const __nv_bfloat16 bv = __float2bfloat16_rn(live ? acc[i][j] : 0.f);
+      out[((size_t)r * H + h) * D + tx * TN + j] = *reinterpret_cast<const uint16_t*>(&bv);
+    }
+  }
+}
+
+cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s) {
+  if (a.cmp_rows <= 0) return cudaSuccess;
+  dim3 grid((a.cmp_rows + 31) / 32, a.geo.Hkv, 2);
+  if (a.geo.D == 128)
+    nsa_compress_kernel<128><<<grid, 256, 0, s>>>(a);
+  else
+    nsa_compress_kernel<64><<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ top-n
+// One warp per (token, KV group).  Candidates are the blocks j with j*l <= t;
+// the complete ones (j < (t+1)/l) carry their score, the incomplete block
+// holding t competes with score 0.  The n largest under (score descending,
+// index ascending) are found by an 8-bit radix select on the score bits
+// (scores are non-negative, so their bit patterns order like the values),
+// followed by taking the lowest-index ties at the threshold.  The result is
+// written in ascending block order, padded with -1.
+__device__ __forceinline__ uint32_t score_bits(const float* S, int j, int ncmp) {
+  return j < ncmp ? __float_as_uint(S[j]) : 0u;
+}
+
+__global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
+  if (a.meta->bad) return;
+  __shared__ unsigned hist_all[8][256];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  unsigned* hist = hist_all[warp];
+  const int H = a.geo.Hkv, l = a.geo.l, n = a.geo.n;
+  const long long row = (long long)blockIdx.x * 8 + warp;
+  if (row >= (long long)a.total_tokens * H) return;
+  const int tg = (int)(row / H), g = (int)(row % H);
+  const int b = seq_of_token(a.cu, a.batch, tg);
+  const int t = tg - __ldg(a.cu + b);
+  const int ncmp = (t + 1) / l;
+  const int ncand = t / l + 1;
+  const float* S = a.scores + ((size_t)tg * H + g) * a.geo.cmp_cap;
+  int* out = a.sel + ((size_t)tg * H + g) * n;
+  const unsigned lt_mask = (1u << lane) - 1u;
+
+  if (ncand <= n) {
+    for (int j = lane; j < n; j += 32) out[j] = j < ncand ? j : -1;
+    return;
+  }
+  uint32_t prefix = 0, pmask = 0;
+  int k = n;  // rank still to be found inside the current prefix class
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) hist[i] = 0;
+    __syncwarp();
+    for (int j = lane; j < ncand; j += 32) {
+      const uint32_t x = score_bits(S, j, ncmp);
+      if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    unsigned c[8];
+    unsigned mine = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = hist[lane * 8 + e];
+      mine += c[e];
+    }
+    // suffix sum over lanes (higher lanes hold higher digits)
+    unsigned suf = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned other = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += other;
+    }
+    const unsigned above = suf - mine;  // keys with a digit above my 8 bins
+    const bool owner = (above < (unsigned)k) && ((unsigned)k <= suf);
+    const unsigned ob = __ballot_sync(0xffffffffu, owner);
+    const int src = __ffs(ob) - 1;
+    int digit = 0;
+    unsigned count_above = 0;
+    if (lane == src) {
+      unsigned acc = above;
+      for (int e = 7; e >= 0; --e) {
+        if (acc + c[e] >= (unsigned)k) {
+          digit = lane * 8 + e;
+          break;
+        }
+        acc += c[e];
+      }
+      count_above = acc;
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    count_above = __shfl_sync(0xffffffffu, count_above, src);
+    prefix |= (uint32_t)digit << shift;
+    pmask |= 255u << shift;
+    k -= (int)count_above;
+    __syncwarp();
+  }
+  // prefix is the n-th largest score; take every larger score and the k
+  // lowest-index ties.
+  int written = 0, ties_seen = 0;
+  for (int base = 0; base < ncand; base += 32) {
+    const int j = base + lane;
+    const bool valid = j < ncand;
+    const uint32_t x = valid ? score_bits(S, j, ncmp) : 0u;
+    const bool gt = valid && x > prefix;
+    const bool eq = valid && x == prefix;
+    const unsigned em = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && ties_seen + __popc(em & lt_mask) < k);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[written + __popc(tm & lt_mask)] = j;
+    written += __popc(tm);
+    ties_seen += __popc(em);
+  }
+  for (int j = written + lane; j < n; j += 32) out[j] = -1;
+}
+
+cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s) {
+  const long long rows = (long long)a.total_tokens * a.geo.Hkv;
+  if (rows == 0) return cudaSuccess;
+  nsa_topn_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ timeout self-test
+// One CTA waits on an mbarrier that nothing will ever arrive on; the bounded
+// wait gives up after `cycles` and records the timeout in the status word.
+__global__ void nsa_timeout_selftest_kernel(int* status, long long cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sm100::mbar_wait(&bar, 0, &abort_flag, status, cycles);
+}
+
+cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s) {
+  nsa_timeout_selftest_kernel<<<1, 32, 0, s>>>(status, cycles);
+  return cudaGetLastError();
+}
+
+}  // namespace nsa

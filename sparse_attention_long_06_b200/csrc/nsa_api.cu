@@ -1,0 +1,305 @@
+// Host side of the C ABI declared in include/nsa.h: plan validation,
+// workspace layout, TMA descriptor encoding and the launch sequence.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "nsa_internal.cuh"
+
+using namespace nsa;
+
+struct nsa_plan_s {
+  nsa_params p;
+  Geometry geo;
+};
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool is_pow2_le16(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+
+struct PrefillLayout {
+  size_t meta, o_cmp, lse, scores, sel, scratch, total;
+};
+
+PrefillLayout prefill_layout(const nsa_plan_s* pl) {
+  const nsa_params& p = pl->p;
+  const Geometry& g = pl->geo;
+  const size_t T = (size_t)p.max_total_tokens;
+  PrefillLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  take(kHeaderBytes);  // status word at offset 0
+  L.meta = take(sizeof(Meta) + 2 * sizeof(int) * ((size_t)p.max_batch + 1));
+  L.o_cmp = take(T * g.Hq * g.D * sizeof(float));
+  L.lse = take(T * g.Hq * sizeof(float));
+  L.scores = take(T * g.Hkv * (size_t)g.cmp_cap * sizeof(float));
+  L.sel = take(T * g.Hkv * (size_t)g.n * sizeof(int));
+  L.scratch = take((size_t)kMaxPersistentCtas * g.tpt * g.G * g.D * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- TMA encode
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor (inner D, middle heads, outer rows), 128-byte swizzled box.
+bool encode3d(CUtensorMap* m, const void* base, int D, int heads, long long rows, int box_heads,
+              int box_rows) {
+  memset(m, 0, sizeof(*m));
+  if (rows <= 0) return true;  // never dereferenced
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * heads};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms_current() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nsa_strerror(int status) {
+  switch (status) {
+    case NSA_OK: return "ok";
+    case NSA_ERR_INVALID_ARG: return "invalid argument";
+    case NSA_ERR_UNSUPPORTED: return "unsupported geometry";
+    case NSA_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case NSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case NSA_ERR_CUDA: return "CUDA runtime error";
+    case NSA_ERR_DEVICE_TIMEOUT: return "device: bounded wait gave up";
+    case NSA_ERR_DEVICE_BAD_INPUT: return "device: sequence lengths out of range";
+    default: return "unknown status";
+  }
+}
+
+int nsa_last_launch_count(void) { return g_last_launches; }
+
+int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out) {
+  if (!params || !plan_out) return NSA_ERR_INVALID_ARG;
+  *plan_out = nullptr;
+  const nsa_params& p = *params;
+  if (p.head_dim <= 0 || p.num_q_heads <= 0 || p.num_kv_heads <= 0 || p.cmp_block <= 0 ||
+      p.cmp_stride <= 0 || p.sel_block <= 0 || p.top_n <= 0 || p.window <= 0 ||
+      p.max_batch <= 0 || p.max_seqlen <= 0 || p.max_total_tokens < 0 ||
+      p.softmax_scale < 0.f || !std::isfinite(p.softmax_scale) ||
+      (p.out_dtype != NSA_OUT_BF16 && p.out_dtype != NSA_OUT_F32))
+    return NSA_ERR_INVALID_ARG;
+  if (p.num_q_heads % p.num_kv_heads != 0) return NSA_ERR_INVALID_ARG;
+  if (p.cmp_stride > p.cmp_block) return NSA_ERR_INVALID_ARG;
+  const int G = p.num_q_heads / p.num_kv_heads;
+  if (p.head_dim != 64 && p.head_dim != 128) return NSA_ERR_UNSUPPORTED;
+  if (!is_pow2_le16(G)) return NSA_ERR_UNSUPPORTED;
+  if (p.cmp_block != p.cmp_stride || p.sel_block != p.cmp_block) return NSA_ERR_UNSUPPORTED;
+  if (p.cmp_block != 32 && p.cmp_block != 64) return NSA_ERR_UNSUPPORTED;
+  // the selected branch keeps all of one token's selected keys in TMEM:
+  // at most 8 chunks of 128 keys
+  if (p.top_n > 8 * (kChunk / p.sel_block)) return NSA_ERR_UNSUPPORTED;
+  if (p.max_seqlen < p.cmp_block) return NSA_ERR_INVALID_ARG;
+  nsa_plan_s* pl = new (std::nothrow) nsa_plan_s;
+  if (!pl) return NSA_ERR_INVALID_ARG;
+  pl->p = p;
+  Geometry& g = pl->geo;
+  g.D = p.head_dim;
+  g.Hq = p.num_q_heads;
+  g.Hkv = p.num_kv_heads;
+  g.G = G;
+  g.tpt = kTileRows / G;
+  g.l = p.cmp_block;
+  g.n = p.top_n;
+  g.w = p.window;
+  g.cmp_cap = p.max_seqlen / p.cmp_block;
+  g.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / std::sqrt((float)p.head_dim);
+  g.scale_log2 = g.scale * 1.4426950408889634f;
+  g.out_f32 = p.out_dtype == NSA_OUT_F32;
+  *plan_out = pl;
+  return NSA_OK;
+}
+
+void nsa_plan_destroy(nsa_plan_t plan) { delete plan; }
+
+size_t nsa_workspace_size(nsa_plan_t plan, int mode) {
+  if (!plan) return 0;
+  if (mode == NSA_MODE_PREFILL) return prefill_layout(plan).total;
+  return 0;
+}
+
+int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, size_t* bytes) {
+  if (!plan || !offset || !bytes || mode != NSA_MODE_PREFILL) return NSA_ERR_INVALID_ARG;
+  const PrefillLayout L = prefill_layout(plan);
+  const Geometry& g = plan->geo;
+  const size_t T = (size_t)plan->p.max_total_tokens;
+  switch (region) {
+    case NSA_WS_STATUS: *offset = 0; *bytes = sizeof(int); break;
+    case NSA_WS_O_CMP: *offset = L.o_cmp; *bytes = T * g.Hq * g.D * sizeof(float); break;
+    case NSA_WS_LSE: *offset = L.lse; *bytes = T * g.Hq * sizeof(float); break;
+    case NSA_WS_SCORES: *offset = L.scores; *bytes = T * g.Hkv * (size_t)g.cmp_cap * sizeof(float); break;
+    case NSA_WS_SEL: *offset = L.sel; *bytes = T * g.Hkv * (size_t)g.n * sizeof(int); break;
+    default: return NSA_ERR_INVALID_ARG;
+  }
+  return NSA_OK;
+}
+
+int nsa_cmp_rows(nsa_plan_t plan, int total_tokens) {
+  if (!plan || total_tokens < 0) return -1;
+  return total_tokens / plan->geo.l;
+}
+
+int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, const float* gates,
+                const float* w_k, const float* w_v, const int* cu_seqlens, int batch,
+                int total_tokens, void* out, void* k_cmp, void* v_cmp, int* sel_idx,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_launches = 0;
+  if (!plan) return NSA_ERR_INVALID_ARG;
+  const nsa_params& p = plan->p;
+  const Geometry& geo = plan->geo;
+  if (batch <= 0 || batch > p.max_batch || total_tokens < 0 ||
+      total_tokens > p.max_total_tokens)
+    return NSA_ERR_INVALID_ARG;
+  if (!cu_seqlens || !workspace) return workspace ? NSA_ERR_INVALID_ARG : NSA_ERR_WORKSPACE;
+  const PrefillLayout L = prefill_layout(plan);
+  if (workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return NSA_ERR_WORKSPACE;
+  const int cmp_rows = total_tokens / geo.l;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !gates || !w_k || !w_v || !out) return NSA_ERR_INVALID_ARG;
+    if (cmp_rows > 0 && (!k_cmp || !v_cmp)) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(w_k) || !aligned16(w_v) || (cmp_rows > 0 && (!aligned16(k_cmp) || !aligned16(v_cmp))) ||
+        (reinterpret_cast<uintptr_t>(gates) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(sel_idx) & 3u))
+      return NSA_ERR_MISALIGNED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  PrefillArgs a{};
+  a.geo = geo;
+  a.batch = batch;
+  a.total_tokens = total_tokens;
+  a.cmp_rows = cmp_rows;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.gates = gates;
+  a.w_k = w_k;
+  a.w_v = w_v;
+  a.cu = cu_seqlens;
+  a.out = out;
+  a.k_cmp = static_cast<uint16_t*>(k_cmp);
+  a.v_cmp = static_cast<uint16_t*>(v_cmp);
+  a.status = reinterpret_cast<int*>(ws);
+  a.meta = reinterpret_cast<Meta*>(ws + L.meta);
+  a.cmp_off = reinterpret_cast<int*>(ws + L.meta + sizeof(Meta));
+  a.tile_off = a.cmp_off + (batch + 1);
+  a.o_cmp = reinterpret_cast<float*>(ws + L.o_cmp);
+  a.lse = reinterpret_cast<float*>(ws + L.lse);
+  a.scores = reinterpret_cast<float*>(ws + L.scores);
+  a.sel = sel_idx ? sel_idx : reinterpret_cast<int*>(ws + L.sel);
+  a.scratch = reinterpret_cast<float*>(ws + L.scratch);
+
+  // status word: cleared at the start of every call
+  if (cudaMemsetAsync(a.status, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
+  if (total_tokens == 0) {
+    if (cudaMemsetAsync(a.meta, 0, sizeof(Meta), s) != cudaSuccess) return NSA_ERR_CUDA;
+    return NSA_OK;
+  }
+  PrefillMaps m;
+  bool ok = encode3d(&m.q, q, geo.D, geo.Hq, total_tokens, geo.G, geo.tpt) &&
+            encode3d(&m.kc, k_cmp, geo.D, geo.Hkv, cmp_rows, 1, kChunk) &&
+            encode3d(&m.vc, v_cmp, geo.D, geo.Hkv, cmp_rows, 1, kChunk) &&
+            encode3d(&m.k_blk, k, geo.D, geo.Hkv, total_tokens, 1, geo.l) &&
+            encode3d(&m.v_blk, v, geo.D, geo.Hkv, total_tokens, 1, geo.l) &&
+            encode3d(&m.k_win, k, geo.D, geo.Hkv, total_tokens, 1, kChunk) &&
+            encode3d(&m.v_win, v, geo.D, geo.Hkv, total_tokens, 1, kChunk);
+  if (!ok) return NSA_ERR_CUDA;
+  const int sms = num_sms_current();
+  if (sms <= 0) return NSA_ERR_CUDA;
+
+  int launches = 0;
+  cudaError_t e = launch_meta(a, s);
+  if (e == cudaSuccess) { ++launches; e = launch_compress(a, s); }
+  if (e == cudaSuccess) { ++launches; e = launch_cmp_attn(a, m, sms, s); }
+  if (e == cudaSuccess) { ++launches; e = launch_topn(a, s); }
+  if (e == cudaSuccess) { ++launches; e = launch_slc_win(a, m, sms, s); }
+  if (e != cudaSuccess) {
+    fprintf(stderr, "nsa_prefill: launch failed: %s\n", cudaGetErrorString(e));
+    return NSA_ERR_CUDA;
+  }
+  g_last_launches = launches + 1;
+  return NSA_OK;
+}
+
+int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* v_cache,
+               void* k_cmp_cache, void* v_cmp_cache, const int* seqlens, int batch,
+               int cache_capacity, const float* gates, const float* w_k, const float* w_v,
+               void* out, int* sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)plan; (void)q; (void)k_cache; (void)v_cache; (void)k_cmp_cache; (void)v_cmp_cache;
+  (void)seqlens; (void)batch; (void)cache_capacity; (void)gates; (void)w_k; (void)w_v;
+  (void)out; (void)sel_idx; (void)workspace; (void)workspace_bytes; (void)stream;
+  g_last_launches = 0;
+  return NSA_ERR_UNSUPPORTED;
+}
+
+int nsa_read_device_status(const void* workspace, void* stream) {
+  if (!workspace) return NSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return NSA_ERR_CUDA;
+  int st = 0;
+  if (cudaMemcpy(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return NSA_ERR_CUDA;
+  if (cudaMemset(const_cast<void*>(workspace), 0, sizeof(int)) != cudaSuccess) return NSA_ERR_CUDA;
+  return st;
+}
+
+int nsa_selftest_timeout(void* workspace, size_t workspace_bytes, long long cycles,
+                         void* stream) {
+  if (!workspace || workspace_bytes < sizeof(int)) return NSA_ERR_WORKSPACE;
+  if (cycles <= 0 || cycles > (1LL << 34)) return NSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
+  if (launch_timeout_selftest(status, cycles, s) != cudaSuccess) return NSA_ERR_CUDA;
+  return NSA_OK;
+}
+
+}  // extern "C"

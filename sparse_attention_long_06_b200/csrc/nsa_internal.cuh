@@ -1,0 +1,110 @@
+// Internal structures shared by the host API (nsa_api.cu) and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/nsa.h"
+
+namespace nsa {
+
+// Tokens of one dense tile: 128 MMA rows = (128 / G) tokens x G heads.
+constexpr int kTileRows = 128;
+// Keys per MMA chunk (M of the swap-AB products, N of the dense ones).
+constexpr int kChunk = 128;
+// Fixed upper bound on persistent CTAs (scratch regions are sized for it).
+constexpr int kMaxPersistentCtas = 256;
+// Header of every workspace: status word and counters.
+constexpr size_t kHeaderBytes = 256;
+
+struct Geometry {
+  int D;        // head dim
+  int Hq, Hkv;  // heads
+  int G;        // Hq / Hkv
+  int tpt;      // tokens per dense tile = 128 / G
+  int l;        // block length (compress block == stride == select block)
+  int n;        // top-n
+  int w;        // window
+  int cmp_cap;  // row stride of the score table = max_seqlen / l
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+  int out_f32;       // output dtype
+};
+
+// Per-call device metadata derived from cu_seqlens by nsa_meta_kernel.
+struct Meta {
+  int bad;          // nonzero when cu_seqlens is inconsistent (all kernels skip)
+  int cmp_total;    // sum_b floor(T_b / l)
+  int tiles_total;  // sum_b ceil(T_b / tpt)
+  int pad_;
+  // followed in memory by: cmp_off[B+1], tile_off[B+1]
+};
+
+struct PrefillArgs {
+  Geometry geo;
+  int batch;
+  int total_tokens;
+  int cmp_rows;  // rows of k_cmp / v_cmp (floor(total / l))
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const float* gates;
+  const float* w_k;
+  const float* w_v;
+  const int* cu;
+  void* out;
+  uint16_t* k_cmp;
+  uint16_t* v_cmp;
+  int* sel;
+  // workspace views
+  int* status;
+  Meta* meta;
+  int* cmp_off;   // [B+1]
+  int* tile_off;  // [B+1]
+  float* o_cmp;   // [T, Hq, D]
+  float* lse;     // [T, Hq]
+  float* scores;  // [T, Hkv, cmp_cap]
+  float* scratch; // [kMaxPersistentCtas, tpt * G * D]
+};
+
+struct PrefillMaps {
+  CUtensorMap q;      // (D, Hq, T) box (64, G, tpt)
+  CUtensorMap kc;     // (D, Hkv, cmp_rows) box (64, 1, 128)
+  CUtensorMap vc;
+  CUtensorMap k_blk;  // (D, Hkv, T) box (64, 1, l)
+  CUtensorMap v_blk;
+  CUtensorMap k_win;  // (D, Hkv, T) box (64, 1, 128)
+  CUtensorMap v_win;
+};
+
+// Sequence of token `tok` (binary search over cu[0..B]).
+__device__ __forceinline__ int seq_of_token(const int* cu, int B, int tok) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= tok) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+// Index b with off[b] <= x < off[b+1].
+__device__ __forceinline__ int seq_of_offset(const int* off, int B, int x) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_meta(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
+                            cudaStream_t s);
+cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_slc_win(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
+                           cudaStream_t s);
+cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s);
+
+}  // namespace nsa

@@ -1,0 +1,115 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point declared in include/nsa.h, and validates arguments on the host (every
+error below is returned before anything touches the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_long_06_b200 import build as nsa_build
+from sparse_attention_long_06_b200 import nsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    nsa_build.build()
+    return nsa.lib()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "nsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert "nsa_prefill" in names and "nsa_decode" in names and "nsa_plan_create" in names
+    for name in names:
+        assert hasattr(L, name), name
+    assert sorted(names) == sorted(nsa.EXPORTED)
+
+
+def test_no_link_dependency_on_libtorch_or_libcuda(L):
+    # the library carries its own CUDA runtime and reaches the driver at run time
+    out = os.popen(f"ldd {nsa.LIB_PATH}").read()
+    assert "libtorch" not in out and "libc10" not in out
+    assert "libcuda.so" not in out
+
+
+def _params(**kw):
+    base = dict(head_dim=128, num_q_heads=64, num_kv_heads=4, cmp_block=64, cmp_stride=64,
+                sel_block=64, top_n=16, window=512, max_batch=8, max_seqlen=65536,
+                max_total_tokens=65536)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(num_q_heads=63), nsa.NSA_ERR_INVALID_ARG),
+    (dict(top_n=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(window=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(cmp_stride=128), nsa.NSA_ERR_INVALID_ARG),       # stride longer than the block
+    (dict(head_dim=96), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(num_q_heads=96, num_kv_heads=4), nsa.NSA_ERR_UNSUPPORTED),  # G = 24
+    (dict(cmp_stride=32), nsa.NSA_ERR_UNSUPPORTED),        # overlapping compression
+    (dict(sel_block=128), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(top_n=17), nsa.NSA_ERR_UNSUPPORTED),             # > 8 chunks of 128 keys
+    (dict(max_seqlen=16), nsa.NSA_ERR_INVALID_ARG),
+])
+def test_plan_validation(L, kw, code):
+    with pytest.raises(nsa.NsaError) as e:
+        nsa.Plan(**_params(**kw))
+    assert e.value.code == code
+
+
+def test_plan_sizes(L):
+    p = nsa.Plan(**_params())
+    ws = p.workspace_size(nsa.MODE_PREFILL)
+    T, Hq, Hkv, D = 65536, 64, 4, 128
+    assert ws >= T * Hq * D * 4 + T * Hkv * 1024 * 4
+    off, nb = p.workspace_region(nsa.WS_O_CMP)
+    assert off % 256 == 0 and nb == T * Hq * D * 4
+    off2, nb2 = p.workspace_region(nsa.WS_SCORES)
+    assert off2 >= off + nb and nb2 == T * Hkv * 1024 * 4 and off2 + nb2 <= ws
+    assert p.cmp_rows(65536) == 1024 and p.cmp_rows(100) == 1
+    assert nsa.Plan(**_params(head_dim=64, num_q_heads=4, num_kv_heads=1, cmp_block=32,
+                              cmp_stride=32, sel_block=32, top_n=4, window=128)).workspace_size() > 0
+
+
+def test_prefill_rejects_bad_arguments_before_launch(L):
+    p = nsa.Plan(**_params(max_total_tokens=4096))
+    fake = 1 << 20  # an aligned address that is never dereferenced
+    ws = p.workspace_size()
+    args = dict(q=fake, k=fake, v=fake, gates=fake, w_k=fake, w_v=fake, cu=fake, batch=1,
+                total=4096, out=fake, kc=fake, vc=fake, sel=None, ws=fake, wsb=ws)
+
+    def call(**over):
+        a = dict(args)
+        a.update(over)
+        return L.nsa_prefill(p.handle, a["q"], a["k"], a["v"], a["gates"], a["w_k"], a["w_v"],
+                             a["cu"], a["batch"], a["total"], a["out"], a["kc"], a["vc"], a["sel"],
+                             a["ws"], a["wsb"], None)
+
+    assert call(q=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(batch=9) == nsa.NSA_ERR_INVALID_ARG
+    assert call(total=4097) == nsa.NSA_ERR_INVALID_ARG
+    assert call(ws=None) == nsa.NSA_ERR_WORKSPACE
+    assert call(wsb=ws - 1) == nsa.NSA_ERR_WORKSPACE
+    assert call(ws=fake + 16) == nsa.NSA_ERR_WORKSPACE        # workspace not 256-byte aligned
+    assert call(q=fake + 2) == nsa.NSA_ERR_MISALIGNED
+    assert call(kc=fake + 8) == nsa.NSA_ERR_MISALIGNED
+    assert call(kc=None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_last_launch_count() == 0
+    assert L.nsa_plan_create(None, ctypes.byref(ctypes.c_void_p())) == nsa.NSA_ERR_INVALID_ARG
+
+
+def test_strerror_covers_every_code(L):
+    for code in range(8):
+        assert nsa.strerror(code) not in ("unknown status", "")
+    assert nsa.strerror(99) == "unknown status"
