@@ -169,6 +169,16 @@ int nsa_read_device_status(const void* workspace, void* stream);
 int nsa_selftest_timeout(void* workspace, size_t workspace_bytes, long long cycles,
                          void* stream);
 
+/* Per-launch timing for benchmarks.  While enabled on the calling thread,
+ * nsa_prefill / nsa_decode record a CUDA event on the call's stream before
+ * each kernel launch and after the last one (the library owns the events).
+ * nsa_profile_stage_ms synchronises the last profiled call's events and
+ * writes up to `max_stages` per-launch durations in milliseconds, in launch
+ * order; it returns the number of launches of that call, or -1 if no
+ * profiled call has been made or a CUDA call failed. */
+int nsa_profile_enable(int enable);
+int nsa_profile_stage_ms(float* ms, int max_stages);
+
 /* Static description of a status code. */
 const char* nsa_strerror(int status);
 

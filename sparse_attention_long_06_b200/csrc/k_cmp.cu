@@ -39,7 +39,8 @@ struct CmpLayout {
   static constexpr int kRing = kQ + 2 * kQBytes;                 // kStages
   static constexpr int kP = kRing + kStages * kChunkBytes;       // P^T
   static constexpr int kLse = kP + kPBytes;                      // float[128]
-  static constexpr int kBars = kLse + 128 * 4;                   // barriers
+  static constexpr int kSum = kLse + 128 * 4;                    // float[128]
+  static constexpr int kBars = kSum + 128 * 4;                   // barriers
   static constexpr int kEnd = kBars + 32 * 8 + 16;
   // at least 116 KB so that one CTA owns an SM (it allocates all 512 TMEM columns)
   static constexpr int kSmem = (kEnd + 1024 > 118 * 1024) ? kEnd + 1024 : 118 * 1024;
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   float* lse_s = reinterpret_cast<float*>(sm + L::kLse);
+  float* sum_s = reinterpret_cast<float*>(sm + L::kSum);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (a.meta->bad) return;
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(192, 1)
       const float lse2 = lsum > 0.f ? m + __log2f(lsum) : -INFINITY;
       softmax_bar();  // every thread is done reading lse_s of the previous tile
       lse_s[r] = lse2;
+      sum_s[r] = lsum;
       softmax_bar();
       // ---- pass 2: this thread owns key r of every chunk
       for (int c = 0; c < it.nc; ++c) {
@@ -342,11 +345,14 @@ __global__ void __launch_bounds__(192, 1)
           float v[16];
           tmem_ld16(lane_addr + buf * 128 + grp * 16, v);
           tmem_ld_wait();
-          float p[16];
+          // p: exact probabilities (block scores); pm = p * row sum = exp(s - row max),
+          // whose largest element is 1 and survives the bf16 rounding exactly
+          float p[16], pm[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int row = grp * 16 + j;
             p[j] = (row >= row_lo && row < row_hi) ? ex2(v[j] * sl2 - lse_s[row]) : 0.f;
+            pm[j] = p[j] * sum_s[row];
           }
           // block score of each token whose heads lie in this group of 16 rows
           for (int j0 = 0; j0 < 16; j0 += G) {
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           uint32_t pk[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
+          for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(pm[2 * j], pm[2 * j + 1]);
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             const int cidx = grp * 2 + cc;
@@ -382,6 +388,7 @@ __global__ void __launch_bounds__(192, 1)
       // ---- epilogue: O_cmp row and log-sum-exp
       mbar_wait(o_full, oc & 1, abort_flag, status, kWaitCycles);
       tc_fence_after();
+      const float inv_sum = lsum > 0.f ? 1.f / lsum : 0.f;
 #pragma unroll
       for (int grp = 0; grp < D / 16; ++grp) {
         float v[16];
@@ -390,7 +397,9 @@ __global__ void __launch_bounds__(192, 1)
         if (row_ok && !*abort_flag) {
           float4* o = reinterpret_cast<float4*>(a.o_cmp + orow * D + grp * 16);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          for (int j = 0; j < 4; ++j)
+            o[j] = make_float4(v[4 * j] * inv_sum, v[4 * j + 1] * inv_sum, v[4 * j + 2] * inv_sum,
+                               v[4 * j + 3] * inv_sum);
         }
       }
       if (row_ok && !*abort_flag) a.lse[orow] = lse2 * 0.6931471805599453f;

@@ -43,8 +43,7 @@ __global__ void nsa_meta_kernel(PrefillArgs a, int max_seqlen) {
 }
 
 cudaError_t launch_meta(const PrefillArgs& a, cudaStream_t s) {
-  // max_seqlen == cmp_cap * l (the plan rounds it down to a block multiple)
-  nsa_meta_kernel<<<1, 32, 0, s>>>(a, a.geo.cmp_cap * a.geo.l);
+  nsa_meta_kernel<<<1, 32, 0, s>>>(a, a.geo.max_seqlen);
   return cudaGetLastError();
 }
 

@@ -529,7 +529,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
-      // ---- window pass B: normalised P, O_win += P V
+      // ---- window pass B: P = exp(s - max) (largest element exactly 1), O_win += P V
       for (int c = 0; c < t.nwc; ++c) {
         const int buf = wait_s();
         wait_p_free();
@@ -544,8 +544,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int j0 = grp * 16 + 2 * j;
-            const float p0 = (row_ok && j0 >= lo && j0 <= hi) ? ex2(v[2 * j] * sl2 - m) * inv_l : 0.f;
-            const float p1 = (row_ok && j0 + 1 >= lo && j0 + 1 <= hi) ? ex2(v[2 * j + 1] * sl2 - m) * inv_l : 0.f;
+            const float p0 = (row_ok && j0 >= lo && j0 <= hi) ? ex2(v[2 * j] * sl2 - m) : 0.f;
+            const float p1 = (row_ok && j0 + 1 >= lo && j0 + 1 <= hi) ? ex2(v[2 * j + 1] * sl2 - m) : 0.f;
             pk[j] = pack_bf16x2(p0, p1);
           }
 #pragma unroll
@@ -564,7 +564,7 @@ __global__ void __launch_bounds__(192, 1)
       softmax_bar();  // token epilogues of the previous tile are done with the slab
       {
         const size_t tg = (size_t)t.row0 + i_row;
-        const float gw = row_ok ? __ldg(a.gates + (tg * Hq + t.g * G + h_row) * 3 + 2) : 0.f;
+        const float gw = row_ok ? __ldg(a.gates + (tg * Hq + t.g * G + h_row) * 3 + 2) * inv_l : 0.f;
 #pragma unroll
         for (int grp = 0; grp < D / 16; ++grp) {
           float v[16];

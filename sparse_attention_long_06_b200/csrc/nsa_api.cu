@@ -19,6 +19,27 @@ namespace {
 
 thread_local int g_last_launches = 0;
 
+// ---------------------------------------------------------------- profiling hook
+constexpr int kMaxProfEvents = 16;
+struct Profiler {
+  bool enabled = false;
+  bool created = false;
+  int marks = 0;  // events recorded by the last profiled call
+  cudaEvent_t ev[kMaxProfEvents];
+};
+thread_local Profiler g_prof;
+
+void prof_reset() { g_prof.marks = 0; }
+void prof_mark(cudaStream_t s) {
+  if (!g_prof.enabled || g_prof.marks >= kMaxProfEvents) return;
+  if (!g_prof.created) {
+    for (int i = 0; i < kMaxProfEvents; ++i)
+      if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return;
+    g_prof.created = true;
+  }
+  cudaEventRecord(g_prof.ev[g_prof.marks++], s);
+}
+
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool is_pow2_le16(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
@@ -114,6 +135,21 @@ const char* nsa_strerror(int status) {
 
 int nsa_last_launch_count(void) { return g_last_launches; }
 
+int nsa_profile_enable(int enable) {
+  g_prof.enabled = enable != 0;
+  g_prof.marks = 0;
+  return NSA_OK;
+}
+
+int nsa_profile_stage_ms(float* ms, int max_stages) {
+  if (g_prof.marks < 2) return -1;
+  if (cudaEventSynchronize(g_prof.ev[g_prof.marks - 1]) != cudaSuccess) return -1;
+  const int n = g_prof.marks - 1;
+  for (int i = 0; i < n && i < max_stages && ms; ++i)
+    if (cudaEventElapsedTime(&ms[i], g_prof.ev[i], g_prof.ev[i + 1]) != cudaSuccess) return -1;
+  return n;
+}
+
 int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out) {
   if (!params || !plan_out) return NSA_ERR_INVALID_ARG;
   *plan_out = nullptr;
@@ -148,6 +184,7 @@ int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out) {
   g.n = p.top_n;
   g.w = p.window;
   g.cmp_cap = p.max_seqlen / p.cmp_block;
+  g.max_seqlen = p.max_seqlen;
   g.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / std::sqrt((float)p.head_dim);
   g.scale_log2 = g.scale * 1.4426950408889634f;
   g.out_f32 = p.out_dtype == NSA_OUT_F32;
@@ -256,11 +293,14 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   if (sms <= 0) return NSA_ERR_CUDA;
 
   int launches = 0;
+  prof_reset();
+  prof_mark(s);
   cudaError_t e = launch_meta(a, s);
-  if (e == cudaSuccess) { ++launches; e = launch_compress(a, s); }
-  if (e == cudaSuccess) { ++launches; e = launch_cmp_attn(a, m, sms, s); }
-  if (e == cudaSuccess) { ++launches; e = launch_topn(a, s); }
-  if (e == cudaSuccess) { ++launches; e = launch_slc_win(a, m, sms, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_compress(a, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_cmp_attn(a, m, sms, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_topn(a, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_slc_win(a, m, sms, s); }
+  prof_mark(s);
   if (e != cudaSuccess) {
     fprintf(stderr, "nsa_prefill: launch failed: %s\n", cudaGetErrorString(e));
     return NSA_ERR_CUDA;

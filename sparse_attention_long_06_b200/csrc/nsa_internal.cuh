@@ -27,6 +27,7 @@ struct Geometry {
   int n;        // top-n
   int w;        // window
   int cmp_cap;  // row stride of the score table = max_seqlen / l
+  int max_seqlen;
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   int out_f32;       // output dtype

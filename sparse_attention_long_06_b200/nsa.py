@@ -28,7 +28,8 @@ WS_STATUS, WS_O_CMP, WS_LSE, WS_SCORES, WS_SEL = 0, 1, 2, 3, 4
 
 EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_workspace_region",
             "nsa_cmp_rows", "nsa_prefill", "nsa_decode", "nsa_read_device_status",
-            "nsa_selftest_timeout", "nsa_strerror", "nsa_last_launch_count"]
+            "nsa_selftest_timeout", "nsa_strerror", "nsa_last_launch_count",
+            "nsa_profile_enable", "nsa_profile_stage_ms"]
 
 
 class NsaError(RuntimeError):
@@ -83,6 +84,10 @@ def lib():
             L.nsa_strerror.restype = ctypes.c_char_p
             L.nsa_last_launch_count.argtypes = []
             L.nsa_last_launch_count.restype = i
+            L.nsa_profile_enable.argtypes = [i]
+            L.nsa_profile_enable.restype = i
+            L.nsa_profile_stage_ms.argtypes = [ctypes.POINTER(ctypes.c_float), i]
+            L.nsa_profile_stage_ms.restype = i
             _lib = L
     return _lib
 
@@ -187,3 +192,16 @@ def selftest_timeout(workspace, cycles: int, stream=None):
 
 def last_launch_count() -> int:
     return int(lib().nsa_last_launch_count())
+
+
+def profile_enable(on: bool = True):
+    lib().nsa_profile_enable(1 if on else 0)
+
+
+def profile_stage_ms(max_stages: int = 16) -> list[float]:
+    """Per-launch milliseconds of the last profiled call (synchronises)."""
+    buf = (ctypes.c_float * max_stages)()
+    n = lib().nsa_profile_stage_ms(buf, max_stages)
+    if n < 0:
+        raise NsaError(NSA_ERR_CUDA, "nsa_profile_stage_ms")
+    return [float(buf[i]) for i in range(min(n, max_stages))]

@@ -2,15 +2,17 @@
 
 Acceptance (NSA forward on the config page's knobs; tolerances from the
 bf16 arithmetic of the path):
-  * compressed KV: within one bf16 ulp of the oracle's single rounding, and
-    different in under 1 % of the elements (fp32 vs fp64 accumulation only
-    flips values that sit on a rounding boundary);
+  * compressed KV: within half a bf16 ulp of the exact fp64 value plus 1e-5
+    (the fp32 accumulation error), and bitwise different from the oracle's
+    single rounding in under 1 % of the elements;
   * stage A: the oracle's top-n replayed on the GPU's fp32 block scores gives
     the GPU's index sets bit for bit;
   * stage B: the oracle run on the GPU's compressed KV gives the same index
     sets, except rows whose fp64 gap between the n-th and (n+1)-th score is
-    below 1e-6, and outputs within max-abs 1e-2 (or half a bf16 ulp of the
-    value for bf16 output) and relative L2 5e-3;
+    below 1e-6, and fp32 outputs within max-abs 1e-2 and relative L2 5e-3;
+  * bf16 output: bit for bit the round-to-nearest-even of the fp32 output of
+    the same call (a bf16 store adds up to half a bf16 ulp, 0.0078 at |o| in
+    [2, 4), so the 1e-2 bound applies to the fp32 result);
   * end to end (oracle's own compressed KV): index sets differ only where a
     1-ulp difference of the compressed KV moves a near-tie (reported, under
     2 % of rows), and rows with equal index sets agree within 1e-2.
@@ -35,15 +37,15 @@ def _lib():
     nsa.lib()
 
 
-def _assert_report(rep, bf16_out, e2e=True):
+def _assert_report(rep, res=None, e2e=True):
     print(rep)
-    assert rep["kc_total"] == 0 or rep["kc_max_ulp"] <= 1
+    assert rep["kc_bound_fail"] == 0
     assert rep["kc_total"] == 0 or rep["kc_diff"] / rep["kc_total"] < 0.01
     assert rep["idx_bad_stageB"] == 0
-    if bf16_out:
-        assert rep["out_tol_fail"] == 0
-    else:
-        assert rep["max_abs"] <= 1e-2
+    assert rep["max_abs"] <= 1e-2
+    if res is not None and "out_bf16" in res:
+        assert res["status_bf16"] == nsa.NSA_OK
+        assert np.array_equal(res["out_bf16"], wl.bf16_bits(res["out"].astype(np.float32)))
     assert rep["rel_l2"] <= 5e-3
     if e2e and rep["e2e_rows"]:
         assert rep["e2e_idx_mismatch"] <= 0.02 * rep["e2e_rows"]
@@ -54,15 +56,14 @@ def _custom(name, D, Hq, Hkv, l, n, w, lens, seed=21):
     return wl.NsaConfig(name, seed, D, Hq, Hkv, l, l, l, n, w, seqlens=tuple(lens))
 
 
-@pytest.mark.parametrize("out_dtype", [nsa.OUT_BF16, nsa.OUT_F32])
-def test_tiny_config_all_rows(out_dtype):
+def test_tiny_config_all_rows():
     cfg = wl.CONFIGS["tiny"]
     inputs = wl.prefill_inputs(cfg)
-    res = gu.run_prefill(cfg, inputs, out_dtype=out_dtype)
+    res = gu.run_prefill(cfg, inputs, both_dtypes=True)
     assert res["status"] == nsa.NSA_OK
     assert res["launches"] == 5
     rep = gu.check_prefill(cfg, inputs, res, [np.arange(1024, dtype=np.int32)])
-    _assert_report(rep, out_dtype == nsa.OUT_BF16)
+    _assert_report(rep, res)
 
 
 @pytest.mark.parametrize("case", [
@@ -82,37 +83,37 @@ def test_edge_geometries(case):
     assert res["status"] == nsa.NSA_OK
     rows = [np.arange(T, dtype=np.int32) for T in lens]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep, False)
+    _assert_report(rep)
 
 
 def test_prefill_8k_sampled_rows():
     cfg = wl.CONFIGS["prefill_8k"]
     inputs = wl.prefill_inputs(cfg)
-    res = gu.run_prefill(cfg, inputs, out_dtype=nsa.OUT_BF16)
+    res = gu.run_prefill(cfg, inputs, both_dtypes=True)
     assert res["status"] == nsa.NSA_OK
     rows = [gu.sample_rows(8192, 384, 7, 8, 64)]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep, True)
+    _assert_report(rep, res)
 
 
 def test_varlen_planted_sampled_rows():
     cfg = wl.CONFIGS["varlen"]
     inputs = wl.prefill_inputs(cfg)
-    res = gu.run_prefill(cfg, inputs, out_dtype=nsa.OUT_BF16)
+    res = gu.run_prefill(cfg, inputs, both_dtypes=True)
     assert res["status"] == nsa.NSA_OK
     rows = [gu.sample_rows(T, 40, 100 + b, 8, 64) for b, T in enumerate(inputs["seqlens"])]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep, True)
+    _assert_report(rep, res)
 
 
 def test_prefill_64k_sampled_rows():
     cfg = wl.CONFIGS["prefill_64k"]
     inputs = wl.prefill_inputs(cfg)
-    res = gu.run_prefill(cfg, inputs, out_dtype=nsa.OUT_BF16)
+    res = gu.run_prefill(cfg, inputs, both_dtypes=True)
     assert res["status"] == nsa.NSA_OK
     rows = [gu.sample_rows(65536, 96, 11, 8, 64)]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep, True)
+    _assert_report(rep, res)
 
 
 def test_repeated_calls_are_deterministic():
