@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int k = blockIdx.x;; k += gridDim.x) {
       const CmpItem it = cmp_item(a, k);
       if (!it.valid) break;
-      const int i_row = r / G, h_row = r % G;
+      const int i_row = r >> a.geo.lg_G, h_row = r & (G - 1);
       const int t_row = it.t0 + i_row;
       const bool row_ok = t_row < it.T;
       const int ncmp_row = row_ok ? (t_row + 1) / l : 0;
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(192, 1)
           // block score of each token whose heads lie in this group of 16 rows
           for (int j0 = 0; j0 < 16; j0 += G) {
             const int row = grp * 16 + j0;
-            const int tok = row / G;
+            const int tok = row >> a.geo.lg_G;
             if (row >= row_lo && row < row_hi) {
               float s = 0.f;
               for (int j = j0; j < j0 + G; ++j) s += p[j];

@@ -475,11 +475,14 @@ __global__ void __launch_bounds__(192, 1)
       if (r < D && !*abort_flag) {
         const int co = (i * G) & 7;
         const size_t tg = (size_t)t.row0 + i;
-        for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int col = 0; col < 16; ++col) {
+          const int h = col - co;
+          if (h < 0 || h >= G) continue;
           const int gh = t.g * G + h;
           const float* gt = a.gates + (tg * Hq + gh) * 3;
           const float val = __ldg(gt + 0) * a.o_cmp[(tg * Hq + gh) * D + r] +
-                            __ldg(gt + 1) * o[(co + h) & 15] * inv[h] +
+                            __ldg(gt + 1) * o[col] * inv[col] +
                             scratch[(i * G + h) * D + r];
           const size_t oi = (tg * Hq + gh) * D + r;
           if (a.geo.out_f32) {
@@ -494,7 +497,7 @@ __global__ void __launch_bounds__(192, 1)
     for (int k = blockIdx.x;; k += gridDim.x) {
       const SwTile t = sw_tile(a, k);
       if (!t.valid) break;
-      const int i_row = r / G, h_row = r % G;
+      const int i_row = r >> a.geo.lg_G, h_row = r & (G - 1);
       const bool row_ok = i_row < t.ntok;
       // window keys of this row, as offsets into the tile's window span
       const int o_lo = max(i_row, -t.ws), o_hi = i_row + w - 1;
@@ -586,22 +589,30 @@ __global__ void __launch_bounds__(192, 1)
       softmax_bar();
       // ---- selected branch, one job per token; this thread owns key lane r
       const int* selbase = a.sel + ((size_t)t.row0 * Hkv + t.g) * n;
+      const int lg_l = a.geo.lg_l, key_in_blk = r & (l - 1), slot_in_chunk = r >> lg_l;
       for (int i = 0; i < t.ntok; ++i) {
         const int tt = t.t0 + i;
         const int* sel = selbase + (size_t)i * Hkv * n;
+        // first key of this thread's block in every chunk (-1: no block / beyond t)
+        int kfirst[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int bs = c * bpc + slot_in_chunk;
+          const int blk = (c < t.nsc && bs < n) ? __ldg(sel + bs) : -1;
+          kfirst[c] = (blk >= 0 && (blk << lg_l) + key_in_blk <= tt) ? 1 : 0;
+        }
         const int buf = wait_s();
         float mx[16];
 #pragma unroll
         for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
         // sweep 1: per-head maximum over this thread's keys
-        for (int c = 0; c < t.nsc; ++c) {
-          const int bs = c * bpc + r / l;
-          const int blk = bs < n ? __ldg(sel + bs) : -1;
-          const bool ok_key = blk >= 0 && blk * l + (r % l) <= tt;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c >= t.nsc) break;
           float v[16];
           tmem_ld16(lane_addr + buf * 128 + c * 16, v);
           tmem_ld_wait();
-          if (ok_key) {
+          if (kfirst[c]) {
 #pragma unroll
             for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[h] * sl2);
           }
@@ -613,18 +624,19 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
         const int co = (i * G) & 7;
-        for (int c = 0; c < t.nsc; ++c) {
-          const int bs = c * bpc + r / l;
-          const int blk = bs < n ? __ldg(sel + bs) : -1;
-          const bool ok_key = blk >= 0 && blk * l + (r % l) <= tt;
+        uint32_t colmask = 0;  // columns that hold this token's heads
+#pragma unroll
+        for (int h = 0; h < 16; ++h) colmask |= (h >= co && h < co + G) ? (1u << h) : 0u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (c >= t.nsc) break;
           float v[16];
           tmem_ld16(lane_addr + buf * 128 + c * 16, v);
           tmem_ld_wait();
           float p[16];
 #pragma unroll
           for (int h = 0; h < 16; ++h) {
-            const bool mine = (h >= co) && (h < co + G);
-            p[h] = (ok_key && mine) ? ex2(v[h] * sl2 - mx[h]) : 0.f;
+            p[h] = (kfirst[c] && ((colmask >> h) & 1u)) ? ex2(v[h] * sl2 - mx[h]) : 0.f;
             sm16[h] += p[h];
           }
           uint32_t pk[8];
@@ -637,11 +649,11 @@ __global__ void __launch_bounds__(192, 1)
         fence_async_smem();
         release_s(buf, true);
         reduce16(sm16, red + 64, q4, lane, false);
+        // inv_cur[col]: 1 / sum of column col (columns of other tokens get 0)
 #pragma unroll
         for (int h = 0; h < 16; ++h) {
           inv_prev[h] = inv_cur[h];
-          const float sv = sm16[(co + h) & 15];
-          inv_cur[h] = (h < G && sv > 0.f) ? 1.f / sv : 0.f;
+          inv_cur[h] = (((colmask >> h) & 1u) && sm16[h] > 0.f) ? 1.f / sm16[h] : 0.f;
         }
         if (i > 0) token_epilogue(t, i - 1, inv_prev);
       }

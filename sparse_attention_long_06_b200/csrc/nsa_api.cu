@@ -179,8 +179,10 @@ int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out) {
   g.Hq = p.num_q_heads;
   g.Hkv = p.num_kv_heads;
   g.G = G;
+  g.lg_G = __builtin_ctz(G);
   g.tpt = kTileRows / G;
   g.l = p.cmp_block;
+  g.lg_l = __builtin_ctz(p.cmp_block);
   g.n = p.top_n;
   g.w = p.window;
   g.cmp_cap = p.max_seqlen / p.cmp_block;

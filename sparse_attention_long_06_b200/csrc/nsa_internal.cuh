@@ -22,8 +22,10 @@ struct Geometry {
   int D;        // head dim
   int Hq, Hkv;  // heads
   int G;        // Hq / Hkv
+  int lg_G;     // log2(G)
   int tpt;      // tokens per dense tile = 128 / G
   int l;        // block length (compress block == stride == select block)
+  int lg_l;     // log2(l)
   int n;        // top-n
   int w;        // window
   int cmp_cap;  // row stride of the score table = max_seqlen / l

@@ -64,21 +64,40 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 constexpr int kDeviceTimeoutCode = 6;
 constexpr int kDeviceBadInputCode = 7;
 
-// Spins on `bar` reaching phase `parity`.  Gives up once `max_cycles` SM
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` nanoseconds pass, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for `bar` to reach phase `parity`.  Gives up once `max_cycles` SM
 // clock cycles have passed, or as soon as `*abort` is set by another thread of
 // the CTA.  Returns false when it gave up; a thread that gives up on its own
-// raises the CTA abort flag and records the timeout in `*status`.
+// raises the CTA abort flag and records the timeout in `*status`.  The clock
+// and the abort flag are read only every 64 polls, so a waiting warp costs
+// almost no issue slots.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* status, long long max_cycles) {
   if (mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
-  while (true) {
-    if (mbar_test(bar, parity)) return true;
-    if (*abort) return false;
-    if (clock64() - t0 > max_cycles) {
-      *abort = 1;
-      if (status) atomicCAS(status, 0, kDeviceTimeoutCode);
-      return false;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((i & 63u) == 0u) {
+      if (*abort) return false;
+      if (clock64() - t0 > max_cycles) {
+        *abort = 1;
+        if (status) atomicCAS(status, 0, kDeviceTimeoutCode);
+        return false;
+      }
     }
   }
 }
