@@ -135,6 +135,27 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,
                 void* stream);
 
 /*
+ * nsa_prefill without a caller workspace, for callers that cannot allocate
+ * device memory (code running under a memory pool it does not own, code that
+ * must avoid the device synchronisation an allocation can cause, plugins that
+ * only receive tensor pointers).  The web pages on NSA have no counterpart of
+ * this entry point: it is a deployment convenience of this library.
+ * Arguments and results are those of nsa_prefill minus the workspace; the
+ * scratch is one file-scope device array of 32 MiB per GPU, held by every GPU
+ * that loads the library until the process exits.  Returns
+ * NSA_ERR_WORKSPACE when nsa_workspace_size(plan, NSA_MODE_PREFILL) exceeds
+ * 32 MiB.  It calls no allocator.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current:
+ * make that first call before any stream capture.  All calls share the array
+ * and it keeps the last call's contents (the status word is cleared by every
+ * call); calls that overlap on the GPU race on it and must not be issued.
+ */
+int nsa_prefill_noalloc(nsa_plan_t plan, const void* q, const void* k, const void* v,
+                        const float* gates, const float* w_k, const float* w_v,
+                        const int* cu_seqlens, int batch, int total_tokens, void* out,
+                        void* k_cmp, void* v_cmp, int* sel_idx, void* stream);
+
+/*
  * One decode step for a batch of sequences (steps 1-7 for the newest token of
  * each sequence, which the caller has already written into the caches).
  *   q           [batch, Hq, D]             bf16, query of the newest token

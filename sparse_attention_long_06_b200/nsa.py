@@ -29,7 +29,7 @@ WS_STATUS, WS_O_CMP, WS_LSE, WS_SCORES, WS_SEL = 0, 1, 2, 3, 4
 EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_workspace_region",
             "nsa_cmp_rows", "nsa_prefill", "nsa_decode", "nsa_read_device_status",
             "nsa_selftest_timeout", "nsa_strerror", "nsa_last_launch_count",
-            "nsa_profile_enable", "nsa_profile_stage_ms"]
+            "nsa_profile_enable", "nsa_profile_stage_ms", "nsa_prefill_noalloc"]
 
 
 class NsaError(RuntimeError):
@@ -74,6 +74,8 @@ def lib():
             L.nsa_cmp_rows.restype = i
             L.nsa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, sz, vp]
             L.nsa_prefill.restype = i
+            L.nsa_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp]
+            L.nsa_prefill_noalloc.restype = i
             L.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
             L.nsa_decode.restype = i
             L.nsa_read_device_status.argtypes = [vp, vp]
@@ -167,6 +169,18 @@ class Plan:
                                _ptr(v_cmp), _ptr(sel_idx), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream))
         _check(rc, "nsa_prefill")
+
+    def prefill_noalloc(self, q, k, v, gates, w_k, w_v, cu_seqlens, out, k_cmp, v_cmp,
+                        sel_idx=None, stream=None):
+        """nsa_prefill on the library's static device workspace (no caller
+        workspace; for plans whose workspace fits in 32 MiB)."""
+        batch = cu_seqlens.numel() - 1
+        total = q.shape[0]
+        rc = lib().nsa_prefill_noalloc(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(gates),
+                                       _ptr(w_k), _ptr(w_v), _ptr(cu_seqlens), batch, total,
+                                       _ptr(out), _ptr(k_cmp), _ptr(v_cmp), _ptr(sel_idx),
+                                       _stream(stream))
+        _check(rc, "nsa_prefill_noalloc")
 
     def decode(self, q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, seqlens, gates, w_k, w_v,
                out, workspace, sel_idx=None, stream=None):
