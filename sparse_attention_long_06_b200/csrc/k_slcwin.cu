@@ -15,20 +15,22 @@
 // L2).  Per tile:
 //   window, as one dense 128-row tile shared by the tile's tokens:
 //     pass A  S = Q K_win^T (rows on TMEM lanes): row max and sum;
-//     pass B  S again, P = exp(S - max) / sum into shared memory (K-major
-//             A operand), O_win += P V_win in TMEM; the epilogue scales by
-//             g_win and parks the rows in a per-CTA scratch slab (L2-resident);
+//     pass B  S again, P = exp(S - max) into shared memory (K-major A
+//             operand, largest element exactly 1), O_win += P V_win in TMEM;
 //   selected, per token (its G heads share the index set): every selected
 //     block is loaded once by TMA; S^T = K_blk Q_t^T (keys on TMEM lanes,
 //     the token's heads on 16 columns), a two-sweep softmax over all of the
 //     token's keys (block-wide max and sum per head), P^T into shared
-//     memory, O_slc^T += V_blk^T P^T in TMEM; the epilogue (lane = channel)
-//     adds g_cmp O_cmp + g_slc O_slc + scratch and writes the output row.
+//     memory, O_slc^T += V_blk^T P^T in TMEM.
 // The MMA warp issues the QK^T of the next job before the PV of the current
 // one, and the TMA warp loads in the same order, so that K/V streaming
-// overlaps the softmax.
-// Warp roles: 0 = TMA producer, 1 = tcgen05.mma issuer, 2..5 = softmax and
-// epilogues.
+// overlaps the softmax.  P is double-buffered.  A separate epilogue
+// warpgroup turns O_win into g_win * O_win / sum rows of a per-CTA scratch
+// slab (L2-resident) and writes each token's output
+// g_cmp O_cmp + g_slc O_slc / sum + scratch, so that its global loads never
+// sit on the softmax warps' path.
+// Warp roles: 0 = TMA producer, 1 = tcgen05.mma issuer, 2..5 = softmax,
+// 6..9 = epilogue (warp w owns TMEM lanes 32 * (w % 4) .. + 31).
 #include <cuda_bf16.h>
 
 #include "nsa_internal.cuh"
@@ -43,20 +45,25 @@ template <int D>
 struct SwLayout {
   static constexpr int kStages = 4;
   static constexpr int kQBytes = kTileRows * D * 2;
-  static constexpr int kQPad = 2048;  // B-operand row windows may run 8 rows past the tile
   static constexpr int kChunkBytes = kChunk * D * 2;
   static constexpr int kPBytes = kChunk * kTileRows * 2;
+  // B-operand row windows of the selected branch may run 8 rows past the Q
+  // tile; they land in ring stage 0 (in bounds, and only in ignored columns)
   static constexpr int kQ = 0;
-  static constexpr int kRing = kQBytes + kQPad;
-  static constexpr int kP = kRing + kStages * kChunkBytes;
-  static constexpr int kRed = kP + kPBytes;  // float[2][4][16]
-  static constexpr int kBars = kRed + 2 * 4 * 16 * 4;
-  static constexpr int kEnd = kBars + 32 * 8 + 16;
-  static constexpr int kSmem = (kEnd + 1024 > 118 * 1024) ? kEnd + 1024 : 118 * 1024;
+  static constexpr int kRing = kQBytes;
+  static constexpr int kP = kRing + kStages * kChunkBytes;  // 2 buffers
+  static constexpr int kRed = kP + 2 * kPBytes;            // float[2][16][4]
+  static constexpr int kWstat = kRed + 2 * 16 * 4 * 4;     // float[128]
+  static constexpr int kInv = kWstat + 128 * 4;            // float[2][16]
+  static constexpr int kBars = kInv + 2 * 16 * 4;          // barriers + flags
+  static constexpr int kEnd = kBars + 34 * 8;
+  static constexpr int kSmem = kEnd + 1024;
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 constexpr uint32_t kColOwin = 256;
 constexpr uint32_t kColOslc = 384;
+constexpr int kThreads = 320;
 
 struct SwTile {
   int valid, k, b, g, t0, T, row0, ntok, nwc, ws, nsc, njobs;
@@ -69,7 +76,7 @@ __device__ __forceinline__ SwTile sw_tile(const PrefillArgs& a, int k) {
   t.valid = 1;
   t.k = k;
   t.g = k / tiles;  // group-major
-  const int tau = k % tiles;
+  const int tau = k - t.g * tiles;
   t.b = seq_of_offset(a.tile_off, a.batch, tau);
   t.t0 = (tau - a.tile_off[t.b]) * a.geo.tpt;
   const int c0 = __ldg(a.cu + t.b);
@@ -78,7 +85,7 @@ __device__ __forceinline__ SwTile sw_tile(const PrefillArgs& a, int k) {
   t.ntok = min(a.geo.tpt, t.T - t.t0);
   t.nwc = (a.geo.w + a.geo.tpt - 1 + kChunk - 1) / kChunk;
   t.ws = t.t0 - a.geo.w + 1;
-  const int bpc = kChunk / a.geo.l;
+  const int bpc = kChunk >> a.geo.lg_l;
   t.nsc = (a.geo.n + bpc - 1) / bpc;
   t.njobs = 2 * t.nwc + t.ntok;
   return t;
@@ -92,31 +99,55 @@ __device__ __forceinline__ int job_type(const SwTile& t, int jb) {
 }
 
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 // Max (is_max) or sum of 16 per-thread values over the 128 softmax threads.
-__device__ __forceinline__ void reduce16(float (&v)[16], float* red, int q4, int lane, bool is_max) {
+// A reduce-scatter butterfly leaves lane pair (2j, 2j+1) of each warp with
+// column col(lane) of its warp; the four warp partials meet in shared memory
+// laid out [column][warp], and every thread reads back all 16 columns.
+__device__ __forceinline__ void reduce16(float (&v)[16], float* red, int q4, int lane,
+                                         bool is_max) {
+  float a[8];
+  {
+    const bool up = lane & 16;
 #pragma unroll
-  for (int h = 0; h < 16; ++h) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float x = __shfl_xor_sync(0xffffffffu, v[h], o);
-      v[h] = is_max ? fmaxf(v[h], x) : v[h] + x;
+    for (int j = 0; j < 8; ++j) {
+      const float send = up ? v[j] : v[j + 8];
+      const float keep = up ? v[j + 8] : v[j];
+      const float r = __shfl_xor_sync(0xffffffffu, send, 16);
+      a[j] = is_max ? fmaxf(keep, r) : keep + r;
     }
   }
-  if (lane == 0) {
 #pragma unroll
-    for (int h = 0; h < 16; ++h) red[q4 * 16 + h] = v[h];
+  for (int o = 8, half = 4; o >= 2; o >>= 1, half >>= 1) {
+    const bool up = lane & o;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j < half) {
+        const float send = up ? a[j] : a[j + half];
+        const float keep = up ? a[j + half] : a[j];
+        const float r = __shfl_xor_sync(0xffffffffu, send, o);
+        a[j] = is_max ? fmaxf(keep, r) : keep + r;
+      }
+    }
   }
+  {
+    const float r = __shfl_xor_sync(0xffffffffu, a[0], 1);
+    a[0] = is_max ? fmaxf(a[0], r) : a[0] + r;
+  }
+  const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                  ((lane >> 1) & 1);
+  if ((lane & 1) == 0) red[col * 4 + q4] = a[0];
   softmax_bar();
 #pragma unroll
   for (int h = 0; h < 16; ++h) {
-    const float a0 = red[h], a1 = red[16 + h], a2 = red[32 + h], a3 = red[48 + h];
-    v[h] = is_max ? fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) : (a0 + a1) + (a2 + a3);
+    const float4 p = *reinterpret_cast<const float4*>(red + h * 4);
+    v[h] = is_max ? fmaxf(fmaxf(p.x, p.y), fmaxf(p.z, p.w)) : (p.x + p.y) + (p.z + p.w);
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     nsa_slc_win_kernel(const __grid_constant__ PrefillArgs a,
                        const __grid_constant__ PrefillMaps maps) {
   using L = SwLayout<D>;
@@ -127,20 +158,24 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* st_full = bars + 2;     // [4]
-  uint64_t* st_empty = bars + 6;    // [4]
-  uint64_t* s_full = bars + 10;     // [2]
-  uint64_t* s_empty = bars + 12;    // [2]
-  uint64_t* p_full = bars + 14;
-  uint64_t* p_empty = bars + 15;
-  uint64_t* owin_full = bars + 16;
-  uint64_t* owin_empty = bars + 17;
-  uint64_t* oslc_full = bars + 18;   // [2]
-  uint64_t* oslc_empty = bars + 20;  // [2]
-  uint64_t* fin = bars + 22;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 24);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
+  uint64_t* st_full = bars + 2;      // [4]
+  uint64_t* st_empty = bars + 6;     // [4]
+  uint64_t* s_full = bars + 10;      // [2]
+  uint64_t* s_empty = bars + 12;     // [2]
+  uint64_t* p_full = bars + 14;      // [2]
+  uint64_t* p_empty = bars + 16;     // [2]
+  uint64_t* owin_full = bars + 18;
+  uint64_t* owin_empty = bars + 19;  // epilogue done with O_win and the window stats
+  uint64_t* wstat_full = bars + 20;
+  uint64_t* oslc_full = bars + 21;   // [2]
+  uint64_t* tok_ready = bars + 23;   // [2] softmax wrote the token's 1/sum
+  uint64_t* tok_done = bars + 25;    // [2] epilogue done with O_slc[slot] and 1/sum
+  uint64_t* fin = bars + 27;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 30);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 31);
   float* red = reinterpret_cast<float*>(sm + L::kRed);
+  float* wstat = reinterpret_cast<float*>(sm + L::kWstat);
+  float* inv_s = reinterpret_cast<float*>(sm + L::kInv);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (a.meta->bad) return;
@@ -154,13 +189,15 @@ __global__ void __launch_bounds__(192, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
       mbar_init(s_empty + i, 4);
+      mbar_init(p_full + i, 4);
+      mbar_init(p_empty + i, 1);
       mbar_init(oslc_full + i, 1);
-      mbar_init(oslc_empty + i, 4);
+      mbar_init(tok_ready + i, 4);
+      mbar_init(tok_done + i, 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(p_empty, 1);
     mbar_init(owin_full, 1);
     mbar_init(owin_empty, 4);
+    mbar_init(wstat_full, 4);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -176,7 +213,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sbase = smem_u32(sm);
   int* status = a.status;
   const int G = a.geo.G, l = a.geo.l, n = a.geo.n, Hkv = a.geo.Hkv, Hq = a.geo.Hq;
-  const int bpc = kChunk / l;
+  const int lg_l = a.geo.lg_l;
+  const int bpc = kChunk >> lg_l;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -217,7 +255,7 @@ __global__ void __launch_bounds__(192, 1)
           for (int sub = 0; sub < bpc; ++sub) {
             const int bs = c * bpc + sub;
             const int blk = bs < n ? sel[bs] : -1;
-            const int row = blk >= 0 ? c0 + blk * l : -(1 << 24);
+            const int row = blk >= 0 ? c0 + (blk << lg_l) : -(1 << 24);
 #pragma unroll
             for (int h = 0; h < D / 64; ++h)
               tma_load_3d(dst + h * 16384 + sub * l * 128, is_v ? &maps.v_blk : &maps.k_blk,
@@ -300,18 +338,13 @@ __global__ void __launch_bounds__(192, 1)
         mma_commit(st_empty + (sc % L::kStages));
         ++sc;
       };
-      auto acquire_s = [&]() -> int {
+      auto qk = [&](const SwTile& t, int jb) {
+        const int ty = job_type(t, jb);
         const int buf = sbc & 1, u = sbc >> 1;
         if (u > 0 && !mbar_wait(s_empty + buf, (u - 1) & 1, abort_flag, status, kWaitCycles)) {
           ok = false;
-          return -1;
+          return;
         }
-        return buf;
-      };
-      auto qk = [&](const SwTile& t, int jb) {
-        const int ty = job_type(t, jb);
-        const int buf = acquire_s();
-        if (!ok) return;
         const uint32_t dcol = tmem + buf * 128;
         if (ty != kJobTok) {
           const uint32_t st = wait_stage();
@@ -344,13 +377,16 @@ __global__ void __launch_bounds__(192, 1)
       auto pv = [&](const SwTile& t, int jb) {
         const int ty = job_type(t, jb);
         if (ty == kJobWinA) return;
-        if (!mbar_wait(p_full, pc & 1, abort_flag, status, kWaitCycles)) {
+        const int pb = pc & 1;
+        if (!mbar_wait(p_full + pb, (pc >> 1) & 1, abort_flag, status, kWaitCycles)) {
           ok = false;
           return;
         }
+        const uint32_t P = Ps + pb * L::kPBytes;
         if (ty == kJobWinB) {
           const int c = jb - t.nwc;
-          if (c == 0 && owc > 0 && !mbar_wait(owin_empty, (owc - 1) & 1, abort_flag, status, kWaitCycles)) {
+          if (c == 0 && owc > 0 &&
+              !mbar_wait(owin_empty, (owc - 1) & 1, abort_flag, status, kWaitCycles)) {
             ok = false;
             return;
           }
@@ -359,12 +395,12 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int ks = 0; ks < kChunk / 16; ++ks) {
             const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
-            mma_bf16_ss(tmem + kColOwin, smem_desc(Ps + aoff, 16, 1024, kLayoutSw128),
+            mma_bf16_ss(tmem + kColOwin, smem_desc(P + aoff, 16, 1024, kLayoutSw128),
                         smem_desc(st + ks * 2048, 16384, 1024, kLayoutSw128), id_win_pv,
                         (c > 0 || ks > 0) ? 1u : 0u);
           }
           release_stage();
-          mma_commit(p_empty);
+          mma_commit(p_empty + pb);
           ++pc;
           if (c == t.nwc - 1) {
             mma_commit(owin_full);
@@ -372,7 +408,7 @@ __global__ void __launch_bounds__(192, 1)
           }
         } else {
           const int slot = tc & 1, u = tc >> 1;
-          if (u > 0 && !mbar_wait(oslc_empty + slot, (u - 1) & 1, abort_flag, status, kWaitCycles)) {
+          if (u > 0 && !mbar_wait(tok_done + slot, (u - 1) & 1, abort_flag, status, kWaitCycles)) {
             ok = false;
             return;
           }
@@ -383,11 +419,11 @@ __global__ void __launch_bounds__(192, 1)
             for (int ks = 0; ks < kChunk / 16; ++ks)
               mma_bf16_ss(tmem + kColOslc + slot * 16,
                           smem_desc(st + ks * 2048, 16384, 1024, kLayoutSw128),
-                          smem_desc(Ps + c * 4096 + ks * 256, 128, 2048, kLayoutNone), id_slc_pv,
+                          smem_desc(P + c * 4096 + ks * 256, 128, 2048, kLayoutNone), id_slc_pv,
                           (c > 0 || ks > 0) ? 1u : 0u);
             release_stage();
           }
-          mma_commit(p_empty);
+          mma_commit(p_empty + pb);
           ++pc;
           mma_commit(oslc_full + slot);
           ++tc;
@@ -429,75 +465,41 @@ __global__ void __launch_bounds__(192, 1)
       volatile int never = 0;
       mbar_wait(fin, 0, &never, nullptr, kWaitCycles / 4);
     }
-  } else {
-    // ------------------------------------------------------------ softmax / epilogues
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ softmax
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float sl2 = a.geo.scale_log2;
     const int w = a.geo.w;
-    float* scratch = a.scratch + (size_t)blockIdx.x * a.geo.tpt * G * D;
-    int sbc = 0, pc = 0, owc = 0, tce = 0;
-    float inv_prev[16], inv_cur[16];
-#pragma unroll
-    for (int h = 0; h < 16; ++h) inv_prev[h] = inv_cur[h] = 0.f;
+    int sbc = 0, pc = 0, tcs = 0, tiles_done = 0;
     auto wait_s = [&]() -> int {
       const int buf = sbc & 1;
       mbar_wait(s_full + buf, (sbc >> 1) & 1, abort_flag, status, kWaitCycles);
       tc_fence_after();
       return buf;
     };
-    auto release_s = [&](int buf, bool with_p) {
+    auto release_s = [&](int buf, bool with_p, int pb) {
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(s_empty + buf);
-        if (with_p) mbar_arrive(p_full);
+        if (with_p) mbar_arrive(p_full + pb);
       }
       ++sbc;
     };
-    auto wait_p_free = [&]() {
-      if (pc > 0) mbar_wait(p_empty, (pc - 1) & 1, abort_flag, status, kWaitCycles);
+    // claims the next P buffer: waits until the MMA finished reading its last use
+    auto claim_p = [&]() -> int {
+      const int pb = pc & 1, u = pc >> 1;
+      if (u > 0) mbar_wait(p_empty + pb, (u - 1) & 1, abort_flag, status, kWaitCycles);
       ++pc;
+      return pb;
     };
-    // final output of token i of tile t from O_slc^T (lane = channel)
-    auto token_epilogue = [&](const SwTile& t, int i, const float (&inv)[16]) {
-      const int slot = tce & 1;
-      mbar_wait(oslc_full + slot, (tce >> 1) & 1, abort_flag, status, kWaitCycles);
-      tc_fence_after();
-      float o[16];
-      tmem_ld16(lane_addr + kColOslc + slot * 16, o);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(oslc_empty + slot);
-      ++tce;
-      if (r < D && !*abort_flag) {
-        const int co = (i * G) & 7;
-        const size_t tg = (size_t)t.row0 + i;
-#pragma unroll
-        for (int col = 0; col < 16; ++col) {
-          const int h = col - co;
-          if (h < 0 || h >= G) continue;
-          const int gh = t.g * G + h;
-          const float* gt = a.gates + (tg * Hq + gh) * 3;
-          const float val = __ldg(gt + 0) * a.o_cmp[(tg * Hq + gh) * D + r] +
-                            __ldg(gt + 1) * o[col] * inv[col] +
-                            scratch[(i * G + h) * D + r];
-          const size_t oi = (tg * Hq + gh) * D + r;
-          if (a.geo.out_f32) {
-            static_cast<float*>(a.out)[oi] = val;
-          } else {
-            const __nv_bfloat16 bv = __float2bfloat16_rn(val);
-            static_cast<uint16_t*>(a.out)[oi] = *reinterpret_cast<const uint16_t*>(&bv);
-          }
-        }
-      }
-    };
+    const int key_in_blk = r & (l - 1), slot_in_chunk = r >> lg_l;
     for (int k = blockIdx.x;; k += gridDim.x) {
       const SwTile t = sw_tile(a, k);
       if (!t.valid) break;
-      const int i_row = r >> a.geo.lg_G, h_row = r & (G - 1);
+      const int i_row = r >> a.geo.lg_G;
       const bool row_ok = i_row < t.ntok;
       // window keys of this row, as offsets into the tile's window span
       const int o_lo = max(i_row, -t.ws), o_hi = i_row + w - 1;
@@ -514,7 +516,7 @@ __global__ void __launch_bounds__(192, 1)
           for (int j = 0; j < 16; ++j) x[grp * 16 + j] = v[j];
         }
         tmem_ld_wait();
-        release_s(buf, false);
+        release_s(buf, false, 0);
         const int lo = o_lo - c * kChunk, hi = o_hi - c * kChunk;
         float cm = -INFINITY;
 #pragma unroll
@@ -531,95 +533,87 @@ __global__ void __launch_bounds__(192, 1)
           m = mn;
         }
       }
-      const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
-      // ---- window pass B: P = exp(s - max) (largest element exactly 1), O_win += P V
+      // 1 / row sum for the window epilogue (after it released the previous tile's)
+      if (tiles_done > 0) mbar_wait(owin_empty, (tiles_done - 1) & 1, abort_flag, status, kWaitCycles);
+      wstat[r] = lsum > 0.f ? 1.f / lsum : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(wstat_full);
+      // ---- window pass B: P = exp(s - max), O_win += P V (in the MMA warp)
       for (int c = 0; c < t.nwc; ++c) {
         const int buf = wait_s();
-        wait_p_free();
+        const int pb = claim_p();
         const int lo = o_lo - c * kChunk, hi = o_hi - c * kChunk;
-        const uint32_t prow = sbase + L::kP + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t prow = sbase + L::kP + pb * L::kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-        for (int grp = 0; grp < kChunk / 16; ++grp) {
-          float v[16];
-          tmem_ld16(lane_addr + buf * 128 + grp * 16, v);
-          tmem_ld_wait();
-          uint32_t pk[8];
+        for (int half = 0; half < 2; ++half) {
+          float v[64];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int j0 = grp * 16 + 2 * j;
-            const float p0 = (row_ok && j0 >= lo && j0 <= hi) ? ex2(v[2 * j] * sl2 - m) : 0.f;
-            const float p1 = (row_ok && j0 + 1 >= lo && j0 + 1 <= hi) ? ex2(v[2 * j + 1] * sl2 - m) : 0.f;
-            pk[j] = pack_bf16x2(p0, p1);
+          for (int g4 = 0; g4 < 4; ++g4) {
+            float u16[16];
+            tmem_ld16(lane_addr + buf * 128 + half * 64 + g4 * 16, u16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[g4 * 16 + j] = u16[j];
           }
+          tmem_ld_wait();
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int kc8 = grp * 2 + cc;  // 8-key chunk index
-            const uint32_t addr = prow + (kc8 >> 3) * 16384 + (((kc8 & 7) ^ (r & 7)) << 4);
-            st_shared_v4(addr, pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+          for (int g8 = 0; g8 < 8; ++g8) {  // 8 keys per 16-byte chunk
+            uint32_t pk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int j0 = half * 64 + g8 * 8 + 2 * j;
+              const float p0 = (row_ok && j0 >= lo && j0 <= hi) ? ex2(v[g8 * 8 + 2 * j] * sl2 - m) : 0.f;
+              const float p1 = (row_ok && j0 + 1 >= lo && j0 + 1 <= hi) ? ex2(v[g8 * 8 + 2 * j + 1] * sl2 - m) : 0.f;
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+            const uint32_t addr = prow + half * 16384 + ((g8 ^ (r & 7)) << 4);
+            st_shared_v4(addr, pk[0], pk[1], pk[2], pk[3]);
           }
         }
         fence_async_smem();
-        release_s(buf, true);
+        release_s(buf, true, pb);
       }
-      // ---- window epilogue: g_win * O_win rows into the scratch slab
-      mbar_wait(owin_full, owc & 1, abort_flag, status, kWaitCycles);
-      tc_fence_after();
-      softmax_bar();  // token epilogues of the previous tile are done with the slab
-      {
-        const size_t tg = (size_t)t.row0 + i_row;
-        const float gw = row_ok ? __ldg(a.gates + (tg * Hq + t.g * G + h_row) * 3 + 2) * inv_l : 0.f;
-#pragma unroll
-        for (int grp = 0; grp < D / 16; ++grp) {
-          float v[16];
-          tmem_ld16(lane_addr + kColOwin + grp * 16, v);
-          tmem_ld_wait();
-          if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(scratch + (size_t)r * D + grp * 16);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_float4(gw * v[4 * j], gw * v[4 * j + 1], gw * v[4 * j + 2], gw * v[4 * j + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(owin_empty);
-      ++owc;
-      __threadfence_block();
-      softmax_bar();
+      ++tiles_done;
       // ---- selected branch, one job per token; this thread owns key lane r
       const int* selbase = a.sel + ((size_t)t.row0 * Hkv + t.g) * n;
-      const int lg_l = a.geo.lg_l, key_in_blk = r & (l - 1), slot_in_chunk = r >> lg_l;
       for (int i = 0; i < t.ntok; ++i) {
         const int tt = t.t0 + i;
         const int* sel = selbase + (size_t)i * Hkv * n;
-        // first key of this thread's block in every chunk (-1: no block / beyond t)
-        int kfirst[8];
+        bool kok[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const int bs = c * bpc + slot_in_chunk;
           const int blk = (c < t.nsc && bs < n) ? __ldg(sel + bs) : -1;
-          kfirst[c] = (blk >= 0 && (blk << lg_l) + key_in_blk <= tt) ? 1 : 0;
+          kok[c] = blk >= 0 && (blk << lg_l) + key_in_blk <= tt;
         }
         const int buf = wait_s();
         float mx[16];
 #pragma unroll
         for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
-        // sweep 1: per-head maximum over this thread's keys
+        // sweep 1: per-column maximum over this thread's keys
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          if (c >= t.nsc) break;
-          float v[16];
-          tmem_ld16(lane_addr + buf * 128 + c * 16, v);
+        for (int c0 = 0; c0 < 8; c0 += 4) {
+          if (c0 >= t.nsc) break;
+          float v[64];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            float u16[16];
+            tmem_ld16(lane_addr + buf * 128 + (c0 + cc) * 16, u16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[cc * 16 + j] = u16[j];
+          }
           tmem_ld_wait();
-          if (kfirst[c]) {
 #pragma unroll
-            for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[h] * sl2);
+          for (int cc = 0; cc < 4; ++cc) {
+            if (c0 + cc < t.nsc && kok[c0 + cc]) {
+#pragma unroll
+              for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[cc * 16 + h] * sl2);
+            }
           }
         }
         reduce16(mx, red, q4, lane, true);
-        // sweep 2: probabilities, per-head sums, P^T chunks
-        wait_p_free();
+        // sweep 2: probabilities, column sums, P^T chunks
+        const int pb = claim_p();
+        const uint32_t pbase = sbase + L::kP + pb * L::kPBytes + (r >> 3) * 128 + (r & 7) * 16;
         float sm16[16];
 #pragma unroll
         for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
@@ -628,36 +622,134 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int h = 0; h < 16; ++h) colmask |= (h >= co && h < co + G) ? (1u << h) : 0u;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          if (c >= t.nsc) break;
-          float v[16];
-          tmem_ld16(lane_addr + buf * 128 + c * 16, v);
-          tmem_ld_wait();
-          float p[16];
+        for (int c0 = 0; c0 < 8; c0 += 4) {
+          if (c0 >= t.nsc) break;
+          float v[64];
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            p[h] = (kfirst[c] && ((colmask >> h) & 1u)) ? ex2(v[h] * sl2 - mx[h]) : 0.f;
-            sm16[h] += p[h];
+          for (int cc = 0; cc < 4; ++cc) {
+            float u16[16];
+            tmem_ld16(lane_addr + buf * 128 + (c0 + cc) * 16, u16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[cc * 16 + j] = u16[j];
           }
-          uint32_t pk[8];
+          tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
-          const uint32_t base = sbase + L::kP + c * 4096 + (r >> 3) * 128 + (r & 7) * 16;
-          st_shared_v4(base, pk[0], pk[1], pk[2], pk[3]);
-          st_shared_v4(base + 2048, pk[4], pk[5], pk[6], pk[7]);
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = c0 + cc;
+            if (c >= t.nsc) break;
+            float p[16];
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+              p[h] = (kok[c] && ((colmask >> h) & 1u)) ? ex2(v[cc * 16 + h] * sl2 - mx[h]) : 0.f;
+              sm16[h] += p[h];
+            }
+            uint32_t pk[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
+            st_shared_v4(pbase + c * 4096, pk[0], pk[1], pk[2], pk[3]);
+            st_shared_v4(pbase + c * 4096 + 2048, pk[4], pk[5], pk[6], pk[7]);
+          }
         }
         fence_async_smem();
-        release_s(buf, true);
+        release_s(buf, true, pb);
         reduce16(sm16, red + 64, q4, lane, false);
-        // inv_cur[col]: 1 / sum of column col (columns of other tokens get 0)
+        // 1 / column sum for the epilogue warps (after they released this slot)
+        const int slot = tcs & 1, u = tcs >> 1;
+        if (u > 0) mbar_wait(tok_done + slot, (u - 1) & 1, abort_flag, status, kWaitCycles);
+        if (r < 16) {
+          float sv = 0.f;
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          inv_prev[h] = inv_cur[h];
-          inv_cur[h] = (((colmask >> h) & 1u) && sm16[h] > 0.f) ? 1.f / sm16[h] : 0.f;
+          for (int h = 0; h < 16; ++h) sv = (h == r) ? sm16[h] : sv;
+          inv_s[slot * 16 + r] = (((colmask >> r) & 1u) && sv > 0.f) ? 1.f / sv : 0.f;
         }
-        if (i > 0) token_epilogue(t, i - 1, inv_prev);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tok_ready + slot);
+        ++tcs;
       }
-      if (t.ntok > 0) token_epilogue(t, t.ntok - 1, inv_cur);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    float* scratch = a.scratch + (size_t)blockIdx.x * a.geo.tpt * G * D;
+    int tiles_done = 0, tce = 0;
+    for (int k = blockIdx.x;; k += gridDim.x) {
+      const SwTile t = sw_tile(a, k);
+      if (!t.valid) break;
+      // ---- window: g_win * O_win / sum rows into the scratch slab (lane = row)
+      const int i_row = r >> a.geo.lg_G, h_row = r & (G - 1);
+      const bool row_ok = i_row < t.ntok;
+      const size_t tg_row = (size_t)t.row0 + i_row;
+      const float gw = row_ok ? __ldg(a.gates + (tg_row * Hq + t.g * G + h_row) * 3 + 2) : 0.f;
+      epilogue_bar();  // the previous tile's token outputs are done with the slab
+      mbar_wait(wstat_full, tiles_done & 1, abort_flag, status, kWaitCycles);
+      mbar_wait(owin_full, tiles_done & 1, abort_flag, status, kWaitCycles);
+      tc_fence_after();
+      const float scale = gw * wstat[r];
+#pragma unroll
+      for (int g4 = 0; g4 < D / 64; ++g4) {
+        float v[64];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float u16[16];
+          tmem_ld16(lane_addr + kColOwin + g4 * 64 + cc * 16, u16);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[cc * 16 + j] = u16[j];
+        }
+        tmem_ld_wait();
+        if (row_ok) {
+          float4* dst = reinterpret_cast<float4*>(scratch + (size_t)r * D + g4 * 64);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            dst[j] = make_float4(scale * v[4 * j], scale * v[4 * j + 1], scale * v[4 * j + 2],
+                                 scale * v[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(owin_empty);
+      ++tiles_done;
+      __threadfence_block();
+      epilogue_bar();  // slab rows visible to every epilogue thread
+      // ---- tokens: lane = channel
+      for (int i = 0; i < t.ntok; ++i) {
+        const int slot = tce & 1, ph = (tce >> 1) & 1;
+        mbar_wait(tok_ready + slot, ph, abort_flag, status, kWaitCycles);
+        mbar_wait(oslc_full + slot, ph, abort_flag, status, kWaitCycles);
+        tc_fence_after();
+        float o[16];
+        tmem_ld16(lane_addr + kColOslc + slot * 16, o);
+        tmem_ld_wait();
+        float inv[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) inv[h] = inv_s[slot * 16 + h];
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tok_done + slot);
+        ++tce;
+        if (r < D && !*abort_flag) {
+          const int co = (i * G) & 7;
+          const size_t tg = (size_t)t.row0 + i;
+#pragma unroll
+          for (int col = 0; col < 16; ++col) {
+            const int h = col - co;
+            if (h < 0 || h >= G) continue;
+            const int gh = t.g * G + h;
+            const float* gt = a.gates + (tg * Hq + gh) * 3;
+            const float val = __ldg(gt + 0) * a.o_cmp[(tg * Hq + gh) * D + r] +
+                              __ldg(gt + 1) * o[col] * inv[col] +
+                              scratch[(i * G + h) * D + r];
+            const size_t oi = (tg * Hq + gh) * D + r;
+            if (a.geo.out_f32) {
+              static_cast<float*>(a.out)[oi] = val;
+            } else {
+              const __nv_bfloat16 bv = __float2bfloat16_rn(val);
+              static_cast<uint16_t*>(a.out)[oi] = *reinterpret_cast<const uint16_t*>(&bv);
+            }
+          }
+        }
+      }
     }
   }
   tc_fence_before();
@@ -682,7 +774,7 @@ cudaError_t launch_slc_win_t(const PrefillArgs& a, const PrefillMaps& m, int num
     configured[dev] = true;
   }
   const int grid = num_sms < kMaxPersistentCtas ? num_sms : kMaxPersistentCtas;
-  nsa_slc_win_kernel<D><<<grid, 192, L::kSmem, s>>>(a, m);
+  nsa_slc_win_kernel<D><<<grid, kThreads, L::kSmem, s>>>(a, m);
   return cudaGetLastError();
 }
 
