@@ -300,9 +300,94 @@ def run_ours(args, rank, world):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
+    if not args.no_decode:
+        del d, host
+        torch.cuda.empty_cache()
+        result["decode"] = run_decode_leg(args, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(cfg, inputs)
     return result
+
+
+# ---------------------------------------------------------------- decode leg
+def decode_bytes(cfg, lens, sel):
+    """Unique HBM bytes one decode step must read/write: per (sequence, group)
+    the compressed keys and values of the complete blocks, the selected blocks'
+    keys and values and the window's (their union counted once), plus q,
+    gates and out."""
+    D, Hq, Hkv, l, w = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads, cfg.cmp_block, cfg.window
+    total = 0
+    for b, L in enumerate(lens):
+        t = L - 1
+        win = set(range(max(0, t - w + 1), t + 1))
+        for g in range(Hkv):
+            keys = set(win)
+            for blk in sel[b, g]:
+                if blk >= 0:
+                    keys.update(range(blk * l, min(blk * l + l, t + 1)))
+            total += (L // l) * D * 2 * 2 + len(keys) * D * 2 * 2
+        total += Hq * D * 2 + Hq * 3 * 4 + Hq * D * 2
+    return total
+
+
+def run_decode_leg(args, dev):
+    import torch
+    from sparse_attention_long_06_b200 import nsa
+    cfg = wl.CONFIGS["decode_64k"]
+    inp = wl.decode_inputs(cfg)
+    B, cap = cfg.decode_batch, int(inp["capacity"])
+    d = {}
+    for k in ("q", "k", "v", "kc", "vc", "gates", "w_k", "w_v", "seqlens"):
+        a = np.ascontiguousarray(inp[k])
+        d[k] = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+    del inp["k"], inp["v"]
+    plan = nsa.Plan.for_config(cfg, max_batch=B, max_seqlen=cap, out_dtype=nsa.OUT_BF16)
+    out = torch.empty((B, cfg.num_q_heads, cfg.head_dim), dtype=torch.int16, device=dev)
+    sel = torch.empty((B, cfg.num_kv_heads, cfg.top_n), dtype=torch.int32, device=dev)
+    ws = plan.alloc_workspace(nsa.MODE_DECODE, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        plan.decode(d["q"], d["k"], d["v"], d["kc"], d["vc"], d["seqlens"], d["gates"], d["w_k"],
+                    d["w_v"], out, ws, sel_idx=sel)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if nsa.read_device_status(ws) != nsa.NSA_OK:
+        raise RuntimeError("decode device status after warm-up")
+    steps = max(args.steps, 20)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    med = statistics.median(ms)
+    nsa.profile_enable(True)
+    flush.zero_()
+    step()
+    stage = nsa.profile_stage_ms()
+    nsa.profile_enable(False)
+    nbytes = decode_bytes(cfg, [int(x) for x in d["seqlens"].cpu()], sel.cpu().numpy())
+    hbm, _, _, src = _peaks()
+    gbs = nbytes / (med / 1e3) / 1e9
+    kgbs = nbytes / (stage[1] / 1e3) / 1e9
+    return {"metric": "NSA decode tokens/s", "value": round(B / (med / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step_median": round(med, 5), "steps": steps,
+            "config": {"workload": cfg.name, "batch": B, "context": int(cfg.decode_len),
+                       "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
+                       "l": cfg.cmp_block, "top_n": cfg.top_n, "window": cfg.window,
+                       "l2": "flushed before every timed step"},
+            "stage_ms": {"nsa_decode_compress_kernel": round(stage[0], 5),
+                         "nsa_decode_kernel": round(stage[1], 5)},
+            "roofline": {"bound": "hbm", "kernel": "nsa_decode_kernel", "achieved": round(kgbs, 1),
+                         "peak": hbm, "unit": "GB/s", "frac": round(kgbs / hbm, 4),
+                         "algorithmic_bytes": int(nbytes), "step_gbs": round(gbs, 1),
+                         "peak_source": f"{src} copy bandwidth"}}
 
 
 # ---------------------------------------------------------------- reference arm
@@ -339,6 +424,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill_64k", choices=["prefill_64k", "prefill_8k", "varlen"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -165,8 +165,11 @@ int nsa_prefill_noalloc(nsa_plan_t plan, const void* q, const void* k, const voi
  *               token; when the newest token completes a block (len % l == 0)
  *               that block is compressed here from the cache and written back
  *   seqlens     [batch] int32 device, tokens in the cache including the newest,
- *               1 <= len <= cache_capacity
- *   cache_capacity  multiple of l, <= plan max_seqlen
+ *               1 <= len <= cache_capacity and len < 1025 * l (all of a query's
+ *               compressed scores are kept on chip); cache rows at or past
+ *               len are never read
+ *   cache_capacity  multiple of l, <= plan max_seqlen and <= 1025 * l; the
+ *               window must be at most 1024 tokens
  *   gates       [batch, Hq, 3] fp32
  *   w_k, w_v    [Hkv, D, l*D] fp32
  *   out         [batch, Hq, D] bf16 or fp32

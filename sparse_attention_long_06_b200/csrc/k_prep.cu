@@ -6,11 +6,13 @@
 // section on what dynamic sparsity sparsifies (each block is flattened and
 // mapped by one learned linear layer to a single compressed token).
 // Selection follows the config page, section 3 (select_top_k), and the
-// manufacturing page, same section (the highest-scoring blocks are kept).
+// manufacturing page, same section (the highest-scoring blocks are kept);
+// the selection itself is in topn_util.cuh.
 #include <cuda_bf16.h>
 
 #include "nsa_internal.cuh"
 #include "sm100.cuh"
+#include "topn_util.cuh"
 
 namespace nsa {
 
@@ -155,103 +157,21 @@ cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s) {
 }
 
 // ------------------------------------------------------------------ top-n
-// One warp per (token, KV group).  Candidates are the blocks j with j*l <= t;
-// the complete ones (j < (t+1)/l) carry their score, the incomplete block
-// holding t competes with score 0.  The n largest under (score descending,
-// index ascending) are found by an 8-bit radix select on the score bits
-// (scores are non-negative, so their bit patterns order like the values),
-// followed by taking the lowest-index ties at the threshold.  The result is
-// written in ascending block order, padded with -1.
-__device__ __forceinline__ uint32_t score_bits(const float* S, int j, int ncmp) {
-  return j < ncmp ? __float_as_uint(S[j]) : 0u;
-}
-
+// One warp per (token, KV group); the selection itself is warp_topn.
 __global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  unsigned* hist = hist_all[warp];
+  const int warp = threadIdx.x / 32;
   const int H = a.geo.Hkv, l = a.geo.l, n = a.geo.n;
   const long long row = (long long)blockIdx.x * 8 + warp;
   if (row >= (long long)a.total_tokens * H) return;
   const int tg = (int)(row / H), g = (int)(row % H);
   const int b = seq_of_token(a.cu, a.batch, tg);
   const int t = tg - __ldg(a.cu + b);
-  const int ncmp = (t + 1) / l;
-  const int ncand = t / l + 1;
   const float* S = a.scores + ((size_t)tg * H + g) * a.geo.cmp_cap;
   int* out = a.sel + ((size_t)tg * H + g) * n;
-  const unsigned lt_mask = (1u << lane) - 1u;
-
-  if (ncand <= n) {
-    for (int j = lane; j < n; j += 32) out[j] = j < ncand ? j : -1;
-    return;
-  }
-  uint32_t prefix = 0, pmask = 0;
-  int k = n;  // rank still to be found inside the current prefix class
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = lane; i < 256; i += 32) hist[i] = 0;
-    __syncwarp();
-    for (int j = lane; j < ncand; j += 32) {
-      const uint32_t x = score_bits(S, j, ncmp);
-      if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
-    }
-    __syncwarp();
-    unsigned c[8];
-    unsigned mine = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      c[e] = hist[lane * 8 + e];
-      mine += c[e];
-    }
-    // suffix sum over lanes (higher lanes hold higher digits)
-    unsigned suf = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned other = __shfl_down_sync(0xffffffffu, suf, o);
-      if (lane + o < 32) suf += other;
-    }
-    const unsigned above = suf - mine;  // keys with a digit above my 8 bins
-    const bool owner = (above < (unsigned)k) && ((unsigned)k <= suf);
-    const unsigned ob = __ballot_sync(0xffffffffu, owner);
-    const int src = __ffs(ob) - 1;
-    int digit = 0;
-    unsigned count_above = 0;
-    if (lane == src) {
-      unsigned acc = above;
-      for (int e = 7; e >= 0; --e) {
-        if (acc + c[e] >= (unsigned)k) {
-          digit = lane * 8 + e;
-          break;
-        }
-        acc += c[e];
-      }
-      count_above = acc;
-    }
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    count_above = __shfl_sync(0xffffffffu, count_above, src);
-    prefix |= (uint32_t)digit << shift;
-    pmask |= 255u << shift;
-    k -= (int)count_above;
-    __syncwarp();
-  }
-  // prefix is the n-th largest score; take every larger score and the k
-  // lowest-index ties.
-  int written = 0, ties_seen = 0;
-  for (int base = 0; base < ncand; base += 32) {
-    const int j = base + lane;
-    const bool valid = j < ncand;
-    const uint32_t x = valid ? score_bits(S, j, ncmp) : 0u;
-    const bool gt = valid && x > prefix;
-    const bool eq = valid && x == prefix;
-    const unsigned em = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && ties_seen + __popc(em & lt_mask) < k);
-    const unsigned tm = __ballot_sync(0xffffffffu, take);
-    if (take) out[written + __popc(tm & lt_mask)] = j;
-    written += __popc(tm);
-    ties_seen += __popc(em);
-  }
-  for (int j = written + lane; j < n; j += 32) out[j] = -1;
+  warp_topn([&](int j) { return S[j]; }, (t + 1) / l, t / l + 1, n, hist_all[warp],
+            [&](int i, int j) { out[i] = j; });
 }
 
 cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s) {

@@ -35,6 +35,7 @@
 
 #include "nsa_internal.cuh"
 #include "sm100.cuh"
+#include "softmax_util.cuh"
 
 namespace nsa {
 using namespace sm100;
@@ -101,49 +102,9 @@ __device__ __forceinline__ int job_type(const SwTile& t, int jb) {
 __device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
-// Max (is_max) or sum of 16 per-thread values over the 128 softmax threads.
-// A reduce-scatter butterfly leaves lane pair (2j, 2j+1) of each warp with
-// column col(lane) of its warp; the four warp partials meet in shared memory
-// laid out [column][warp], and every thread reads back all 16 columns.
 __device__ __forceinline__ void reduce16(float (&v)[16], float* red, int q4, int lane,
                                          bool is_max) {
-  float a[8];
-  {
-    const bool up = lane & 16;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float send = up ? v[j] : v[j + 8];
-      const float keep = up ? v[j + 8] : v[j];
-      const float r = __shfl_xor_sync(0xffffffffu, send, 16);
-      a[j] = is_max ? fmaxf(keep, r) : keep + r;
-    }
-  }
-#pragma unroll
-  for (int o = 8, half = 4; o >= 2; o >>= 1, half >>= 1) {
-    const bool up = lane & o;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (j < half) {
-        const float send = up ? a[j] : a[j + half];
-        const float keep = up ? a[j + half] : a[j];
-        const float r = __shfl_xor_sync(0xffffffffu, send, o);
-        a[j] = is_max ? fmaxf(keep, r) : keep + r;
-      }
-    }
-  }
-  {
-    const float r = __shfl_xor_sync(0xffffffffu, a[0], 1);
-    a[0] = is_max ? fmaxf(a[0], r) : a[0] + r;
-  }
-  const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
-                  ((lane >> 1) & 1);
-  if ((lane & 1) == 0) red[col * 4 + q4] = a[0];
-  softmax_bar();
-#pragma unroll
-  for (int h = 0; h < 16; ++h) {
-    const float4 p = *reinterpret_cast<const float4*>(red + h * 4);
-    v[h] = is_max ? fmaxf(fmaxf(p.x, p.y), fmaxf(p.z, p.w)) : (p.x + p.y) + (p.z + p.w);
-  }
+  reduce16_across_128<1>(v, red, q4, lane, is_max);
 }
 
 template <int D>
@@ -575,15 +536,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++tiles_done;
       // ---- selected branch, one job per token; this thread owns key lane r
       const int* selbase = a.sel + ((size_t)t.row0 * Hkv + t.g) * n;
+      // block index of this thread's key in every chunk, loaded one token ahead
+      int blk_next[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int bs = c * bpc + slot_in_chunk;
+        blk_next[c] = (t.ntok > 0 && c < t.nsc && bs < n) ? __ldg(selbase + bs) : -1;
+      }
       for (int i = 0; i < t.ntok; ++i) {
         const int tt = t.t0 + i;
-        const int* sel = selbase + (size_t)i * Hkv * n;
         bool kok[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int bs = c * bpc + slot_in_chunk;
-          const int blk = (c < t.nsc && bs < n) ? __ldg(sel + bs) : -1;
-          kok[c] = blk >= 0 && (blk << lg_l) + key_in_blk <= tt;
+        for (int c = 0; c < 8; ++c) kok[c] = blk_next[c] >= 0 && (blk_next[c] << lg_l) + key_in_blk <= tt;
+        if (i + 1 < t.ntok) {
+          const int* seln = selbase + (size_t)(i + 1) * Hkv * n;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int bs = c * bpc + slot_in_chunk;
+            blk_next[c] = (c < t.nsc && bs < n) ? __ldg(seln + bs) : -1;
+          }
         }
         const int buf = wait_s();
         float mx[16];

@@ -106,6 +106,23 @@ bool encode3d(CUtensorMap* m, const void* base, int D, int heads, long long rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D bf16 tensor (D, heads, rows, batch), 128-byte swizzled box (64, 1, box_rows, 1).
+bool encode4d(CUtensorMap* m, const void* base, int D, int heads, long long rows, int batch,
+              int box_rows) {
+  memset(m, 0, sizeof(*m));
+  if (rows <= 0 || batch <= 0) return true;
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2 * heads,
+                           (cuuint64_t)D * 2 * heads * rows};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int num_sms_current() {
@@ -199,6 +216,7 @@ void nsa_plan_destroy(nsa_plan_t plan) { delete plan; }
 size_t nsa_workspace_size(nsa_plan_t plan, int mode) {
   if (!plan) return 0;
   if (mode == NSA_MODE_PREFILL) return prefill_layout(plan).total;
+  if (mode == NSA_MODE_DECODE) return kHeaderBytes;
   return 0;
 }
 
@@ -315,11 +333,69 @@ int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* 
                void* k_cmp_cache, void* v_cmp_cache, const int* seqlens, int batch,
                int cache_capacity, const float* gates, const float* w_k, const float* w_v,
                void* out, int* sel_idx, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)plan; (void)q; (void)k_cache; (void)v_cache; (void)k_cmp_cache; (void)v_cmp_cache;
-  (void)seqlens; (void)batch; (void)cache_capacity; (void)gates; (void)w_k; (void)w_v;
-  (void)out; (void)sel_idx; (void)workspace; (void)workspace_bytes; (void)stream;
   g_last_launches = 0;
-  return NSA_ERR_UNSUPPORTED;
+  if (!plan) return NSA_ERR_INVALID_ARG;
+  const nsa_params& p = plan->p;
+  const Geometry& geo = plan->geo;
+  if (batch <= 0 || batch > p.max_batch || cache_capacity <= 0 ||
+      cache_capacity > p.max_seqlen || cache_capacity % geo.l != 0)
+    return NSA_ERR_INVALID_ARG;
+  // all of one query's compressed scores, window and selected keys stay in
+  // TMEM: at most 1024 compressed blocks, 8 window chunks of 128 keys
+  if (cache_capacity / geo.l > kDecodeMaxCmp + 1 || geo.w > 8 * kChunk) return NSA_ERR_UNSUPPORTED;
+  if (!workspace) return NSA_ERR_WORKSPACE;
+  if (workspace_bytes < kHeaderBytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return NSA_ERR_WORKSPACE;
+  if (!q || !k_cache || !v_cache || !k_cmp_cache || !v_cmp_cache || !seqlens || !gates || !w_k ||
+      !w_v || !out)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_cmp_cache) ||
+      !aligned16(v_cmp_cache) || !aligned16(w_k) || !aligned16(w_v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(gates) & 3u) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sel_idx) & 3u))
+    return NSA_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a{};
+  a.geo = geo;
+  a.batch = batch;
+  a.cap = cache_capacity;
+  a.ccap = cache_capacity / geo.l;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k_cache = static_cast<const uint16_t*>(k_cache);
+  a.v_cache = static_cast<const uint16_t*>(v_cache);
+  a.k_cmp = static_cast<uint16_t*>(k_cmp_cache);
+  a.v_cmp = static_cast<uint16_t*>(v_cmp_cache);
+  a.seqlens = seqlens;
+  a.gates = gates;
+  a.w_k = w_k;
+  a.w_v = w_v;
+  a.out = out;
+  a.sel = sel_idx;
+  a.status = static_cast<int*>(workspace);
+  DecodeMaps m;
+  bool ok = encode3d(&m.q, q, geo.D, geo.Hq, batch, geo.Hq < 16 ? geo.Hq : 16, 1) &&
+            encode4d(&m.kc, k_cmp_cache, geo.D, geo.Hkv, a.ccap, batch, kChunk) &&
+            encode4d(&m.vc, v_cmp_cache, geo.D, geo.Hkv, a.ccap, batch, kChunk) &&
+            encode4d(&m.k_blk, k_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.l) &&
+            encode4d(&m.v_blk, v_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.l) &&
+            encode4d(&m.k_win, k_cache, geo.D, geo.Hkv, cache_capacity, batch, kChunk) &&
+            encode4d(&m.v_win, v_cache, geo.D, geo.Hkv, cache_capacity, batch, kChunk);
+  if (!ok) return NSA_ERR_CUDA;
+  if (cudaMemsetAsync(a.status, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
+  prof_reset();
+  prof_mark(s);
+  cudaError_t e = launch_decode_compress(a, s);
+  if (e == cudaSuccess) {
+    prof_mark(s);
+    e = launch_decode(a, m, s);
+  }
+  prof_mark(s);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "nsa_decode: launch failed: %s\n", cudaGetErrorString(e));
+    return NSA_ERR_CUDA;
+  }
+  g_last_launches = 2;
+  return NSA_OK;
 }
 
 int nsa_read_device_status(const void* workspace, void* stream) {

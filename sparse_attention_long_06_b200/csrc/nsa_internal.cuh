@@ -81,6 +81,39 @@ struct PrefillMaps {
   CUtensorMap v_win;
 };
 
+struct DecodeArgs {
+  Geometry geo;
+  int batch;
+  int cap;   // cache capacity in tokens (multiple of l)
+  int ccap;  // compressed-cache capacity = cap / l
+  const uint16_t* q;        // [B, Hq, D]
+  const uint16_t* k_cache;  // [B, cap, Hkv, D]
+  const uint16_t* v_cache;
+  uint16_t* k_cmp;          // [B, ccap, Hkv, D]
+  uint16_t* v_cmp;
+  const int* seqlens;       // [B]
+  const float* gates;       // [B, Hq, 3]
+  const float* w_k;
+  const float* w_v;
+  void* out;                // [B, Hq, D]
+  int* sel;                 // [B, Hkv, n] or null
+  int* status;
+};
+
+struct DecodeMaps {
+  CUtensorMap q;      // (D, Hq, B) box (64, 16, 1)
+  CUtensorMap kc;     // (D, Hkv, ccap, B) box (64, 1, 128, 1)
+  CUtensorMap vc;
+  CUtensorMap k_blk;  // (D, Hkv, cap, B) box (64, 1, l, 1)
+  CUtensorMap v_blk;
+  CUtensorMap k_win;  // (D, Hkv, cap, B) box (64, 1, 128, 1)
+  CUtensorMap v_win;
+};
+
+// Largest number of compressed blocks one decode query may see (all of its
+// compressed scores stay in TMEM: 8 chunks of 128).
+constexpr int kDecodeMaxCmp = 1024;
+
 // Sequence of token `tok` (binary search over cu[0..B]).
 __device__ __forceinline__ int seq_of_token(const int* cu, int B, int tok) {
   int lo = 0, hi = B - 1;
@@ -109,5 +142,7 @@ cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_slc_win(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
                            cudaStream_t s);
 cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s);
+cudaError_t launch_decode_compress(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);
 
 }  // namespace nsa

@@ -1,0 +1,95 @@
+// Warp-level top-n block selection (step 4), shared by the prefill and
+// decode kernels.
+//
+// Candidates are blocks j < ncand; the complete ones (j < ncmp) carry their
+// score, the incomplete block holding the query competes with score 0.  The
+// n largest under (score descending, index ascending) are found by an 8-bit
+// radix select on the score bits (scores are non-negative, so their bit
+// patterns order like the values), followed by taking the lowest-index ties
+// at the threshold.  The result is written in ascending block order, padded
+// with -1.
+#pragma once
+#include <cstdint>
+
+namespace nsa {
+
+// `score(j)` returns the fp32 score of complete block j; `hist` is 256
+// words of warp-private shared memory; `out(i, j)` stores result i.
+template <typename ScoreFn, typename OutFn>
+__device__ __forceinline__ void warp_topn(ScoreFn score, int ncmp, int ncand, int n,
+                                          unsigned* hist, OutFn out) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  auto bits = [&](int j) -> uint32_t { return j < ncmp ? __float_as_uint(score(j)) : 0u; };
+  if (ncand <= n) {
+    for (int j = lane; j < n; j += 32) out(j, j < ncand ? j : -1);
+    return;
+  }
+  uint32_t prefix = 0, pmask = 0;
+  int k = n;  // rank still to be found inside the current prefix class
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) hist[i] = 0;
+    __syncwarp();
+    for (int j = lane; j < ncand; j += 32) {
+      const uint32_t x = bits(j);
+      if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    unsigned c[8];
+    unsigned mine = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = hist[lane * 8 + e];
+      mine += c[e];
+    }
+    // suffix sum over lanes (higher lanes hold higher digits)
+    unsigned suf = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned other = __shfl_down_sync(0xffffffffu, suf, o);
+      if (lane + o < 32) suf += other;
+    }
+    const unsigned above = suf - mine;  // keys with a digit above this lane's bins
+    const bool owner = (above < (unsigned)k) && ((unsigned)k <= suf);
+    const unsigned ob = __ballot_sync(0xffffffffu, owner);
+    const int src = __ffs(ob) - 1;
+    int digit = 0;
+    unsigned count_above = 0;
+    if (lane == src) {
+      unsigned acc = above;
+      for (int e = 7; e >= 0; --e) {
+        if (acc + c[e] >= (unsigned)k) {
+          digit = lane * 8 + e;
+          break;
+        }
+        acc += c[e];
+      }
+      count_above = acc;
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    count_above = __shfl_sync(0xffffffffu, count_above, src);
+    prefix |= (uint32_t)digit << shift;
+    pmask |= 255u << shift;
+    k -= (int)count_above;
+    __syncwarp();
+  }
+  // prefix holds the n-th largest score; take every larger score and the k
+  // lowest-index ties
+  int written = 0, ties_seen = 0;
+  for (int base = 0; base < ncand; base += 32) {
+    const int j = base + lane;
+    const bool valid = j < ncand;
+    const uint32_t x = valid ? bits(j) : 0u;
+    const bool gt = valid && x > prefix;
+    const bool eq = valid && x == prefix;
+    const unsigned em = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && ties_seen + __popc(em & lt_mask) < k);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out(written + __popc(tm & lt_mask), j);
+    written += __popc(tm);
+    ties_seen += __popc(em);
+  }
+  for (int j = written + lane; j < n; j += 32) out(j, -1);
+}
+
+}  // namespace nsa
