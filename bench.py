@@ -18,6 +18,7 @@ workload on the host cores (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -36,7 +37,11 @@ from sparse_attention_long_06_b200 import workloads as wl  # noqa: E402
 
 METRIC = "NSA prefill tokens/s"
 KERNEL_NAMES = ["nsa_meta_kernel", "nsa_compress_kernel", "nsa_cmp_attn_kernel",
-                "nsa_topn_kernel", "nsa_slc_win_kernel"]
+                "nsa_topn_kernel", "nsa_win_kernel", "nsa_slc_kernel"]
+# tensor-core kernels: (stage index, source file, algorithmic FLOP key)
+TENSOR_KERNELS = {"nsa_cmp_attn_kernel": (2, "k_cmp.cu", "cmp"),
+                  "nsa_win_kernel": (4, "k_win.cu", "win"),
+                  "nsa_slc_kernel": (5, "k_slc.cu", "slc")}
 
 
 def _peaks():
@@ -151,11 +156,12 @@ def oracle_sample(cfg, inputs, nrows=512):
 
 
 # ---------------------------------------------------------------- traffic record
-def traffic_record():
-    """DRAM bytes per launch of the fused selected+window kernel from the
-    committed ncu summary, or None when the kernel source changed since."""
-    path = os.path.join(ROOT, "profiles", "traffic_slc_win.json")
-    src = os.path.join(ROOT, "sparse_attention_long_06_b200", "csrc", "k_slcwin.cu")
+def traffic_record(kernel, src_file):
+    """DRAM bytes per 64k launch of `kernel` from the committed ncu summary
+    profiles/traffic_<kernel>.json, or None when the kernel's source changed
+    since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{kernel}.json")
+    src = os.path.join(ROOT, "sparse_attention_long_06_b200", "csrc", src_file)
     try:
         rec = json.load(open(path))
         digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
@@ -249,13 +255,15 @@ def run_ours(args, rank, world):
     sel_h = sel.cpu().numpy()
     flops = algorithmic_flops(cfg, T, sel_h)
     hbm, tc_burst, tc_sust, peak_src = _peaks()
-    k4_ms = stage_ms[4]
-    k4_flops = flops["slc"] + flops["win"]
-    achieved = k4_flops / (k4_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "nsa_slc_win_kernel", "achieved": round(achieved, 2),
-                "peak": tc_sust, "unit": "TFLOP/s", "frac": round(achieved / tc_sust, 4),
-                "traffic": traffic_record(),
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a repeated step)"}
+    rooflines = {}
+    for name, (idx, src_file, key) in TENSOR_KERNELS.items():
+        ach = flops[key] / (stage_ms[idx] / 1e3) / 1e12
+        rooflines[name] = {"bound": "tensor", "kernel": name, "achieved": round(ach, 2),
+                           "peak": tc_sust, "unit": "TFLOP/s", "frac": round(ach / tc_sust, 4),
+                           "traffic": traffic_record(name, src_file),
+                           "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a repeated step)"}
+    dominant = max(TENSOR_KERNELS, key=lambda k: stage_ms[TENSOR_KERNELS[k][0]])
+    roofline = rooflines[dominant]
 
     # end to end through the public API with host buffers
     e2e_steps = max(2, min(5, args.steps))
@@ -295,6 +303,7 @@ def run_ours(args, rank, world):
         "algorithmic_flop_per_step": flops,
         "stage_ms": dict(zip(KERNEL_NAMES, [round(x, 4) for x in stage_ms])),
         "roofline": roofline,
+        "rooflines": rooflines,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": launches_per_step * args.steps,
@@ -334,6 +343,8 @@ def run_decode_leg(args, dev):
     import torch
     from sparse_attention_long_06_b200 import nsa
     cfg = wl.CONFIGS["decode_64k"]
+    if args.decode_batch:
+        cfg = dataclasses.replace(cfg, decode_batch=args.decode_batch)
     inp = wl.decode_inputs(cfg)
     B, cap = cfg.decode_batch, int(inp["capacity"])
     d = {}
@@ -425,6 +436,10 @@ def main():
     ap.add_argument("--workload", default="prefill_64k", choices=["prefill_64k", "prefill_8k", "varlen"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode leg and print its object (profiling)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="sequences in the decode leg (default: the workload's 32)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -446,7 +461,10 @@ def main():
         build.build()
     if world > 1:
         torch.distributed.barrier()
-    res = run_ours(args, rank, world)
+    if args.decode_only:
+        res = run_decode_leg(args, torch.device("cuda", torch.cuda.current_device()))
+    else:
+        res = run_ours(args, rank, world)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:

@@ -105,7 +105,8 @@ typedef enum {
   NSA_WS_LSE = 2,     /* fp32 [T_total, Hq] compressed-branch log-sum-exp (natural log) */
   NSA_WS_SCORES = 3,  /* fp32 [T_total, Hkv, max_seqlen / l] block scores; entry j
                          of row t is defined for j < number of complete blocks */
-  NSA_WS_SEL = 4      /* int32 [T_total, Hkv, top_n] selection (when sel_idx is NULL) */
+  NSA_WS_SEL = 4,     /* int32 [T_total, Hkv, top_n] selection (when sel_idx is NULL) */
+  NSA_WS_WIN = 5      /* fp32 [T_total, Hq, D] window-branch output times its gate */
 } nsa_ws_region;
 int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, size_t* bytes);
 

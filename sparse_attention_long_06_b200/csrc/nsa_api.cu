@@ -45,7 +45,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool is_pow2_le16(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
 
 struct PrefillLayout {
-  size_t meta, o_cmp, lse, scores, sel, scratch, total;
+  size_t meta, o_cmp, lse, scores, sel, o_win, total;
 };
 
 PrefillLayout prefill_layout(const nsa_plan_s* pl) {
@@ -65,7 +65,7 @@ PrefillLayout prefill_layout(const nsa_plan_s* pl) {
   L.lse = take(T * g.Hq * sizeof(float));
   L.scores = take(T * g.Hkv * (size_t)g.cmp_cap * sizeof(float));
   L.sel = take(T * g.Hkv * (size_t)g.n * sizeof(int));
-  L.scratch = take((size_t)kMaxPersistentCtas * g.tpt * g.G * g.D * sizeof(float));
+  L.o_win = take(T * g.Hq * g.D * sizeof(float));
   L.total = off;
   return L;
 }
@@ -231,6 +231,7 @@ int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, 
     case NSA_WS_LSE: *offset = L.lse; *bytes = T * g.Hq * sizeof(float); break;
     case NSA_WS_SCORES: *offset = L.scores; *bytes = T * g.Hkv * (size_t)g.cmp_cap * sizeof(float); break;
     case NSA_WS_SEL: *offset = L.sel; *bytes = T * g.Hkv * (size_t)g.n * sizeof(int); break;
+    case NSA_WS_WIN: *offset = L.o_win; *bytes = T * g.Hq * g.D * sizeof(float); break;
     default: return NSA_ERR_INVALID_ARG;
   }
   return NSA_OK;
@@ -292,7 +293,7 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   a.lse = reinterpret_cast<float*>(ws + L.lse);
   a.scores = reinterpret_cast<float*>(ws + L.scores);
   a.sel = sel_idx ? sel_idx : reinterpret_cast<int*>(ws + L.sel);
-  a.scratch = reinterpret_cast<float*>(ws + L.scratch);
+  a.o_win = reinterpret_cast<float*>(ws + L.o_win);
 
   // status word: cleared at the start of every call
   if (cudaMemsetAsync(a.status, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
@@ -302,6 +303,7 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   }
   PrefillMaps m;
   bool ok = encode3d(&m.q, q, geo.D, geo.Hq, total_tokens, geo.G, geo.tpt) &&
+            encode3d(&m.q_tok, q, geo.D, geo.Hq, total_tokens, geo.Hq < 16 ? geo.Hq : 16, 1) &&
             encode3d(&m.kc, k_cmp, geo.D, geo.Hkv, cmp_rows, 1, kChunk) &&
             encode3d(&m.vc, v_cmp, geo.D, geo.Hkv, cmp_rows, 1, kChunk) &&
             encode3d(&m.k_blk, k, geo.D, geo.Hkv, total_tokens, 1, geo.l) &&
@@ -319,7 +321,8 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_compress(a, s); }
   if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_cmp_attn(a, m, sms, s); }
   if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_topn(a, s); }
-  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_slc_win(a, m, sms, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_win(a, m, sms, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_slc(a, m, sms, s); }
   prof_mark(s);
   if (e != cudaSuccess) {
     fprintf(stderr, "nsa_prefill: launch failed: %s\n", cudaGetErrorString(e));

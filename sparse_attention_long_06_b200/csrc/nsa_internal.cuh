@@ -68,11 +68,12 @@ struct PrefillArgs {
   float* o_cmp;   // [T, Hq, D]
   float* lse;     // [T, Hq]
   float* scores;  // [T, Hkv, cmp_cap]
-  float* scratch; // [kMaxPersistentCtas, tpt * G * D]
+  float* o_win;   // [T, Hq, D] g_win * O_win
 };
 
 struct PrefillMaps {
   CUtensorMap q;      // (D, Hq, T) box (64, G, tpt)
+  CUtensorMap q_tok;  // (D, Hq, T) box (64, min(16, Hq), 1)
   CUtensorMap kc;     // (D, Hkv, cmp_rows) box (64, 1, 128)
   CUtensorMap vc;
   CUtensorMap k_blk;  // (D, Hkv, T) box (64, 1, l)
@@ -139,8 +140,8 @@ cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
                             cudaStream_t s);
 cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s);
-cudaError_t launch_slc_win(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
-                           cudaStream_t s);
+cudaError_t launch_win(const PrefillArgs& a, const PrefillMaps& m, int num_sms, cudaStream_t s);
+cudaError_t launch_slc(const PrefillArgs& a, const PrefillMaps& m, int num_sms, cudaStream_t s);
 cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s);
 cudaError_t launch_decode_compress(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);

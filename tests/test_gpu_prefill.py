@@ -61,7 +61,7 @@ def test_tiny_config_all_rows():
     inputs = wl.prefill_inputs(cfg)
     res = gu.run_prefill(cfg, inputs, both_dtypes=True)
     assert res["status"] == nsa.NSA_OK
-    assert res["launches"] == 5
+    assert res["launches"] == 6
     rep = gu.check_prefill(cfg, inputs, res, [np.arange(1024, dtype=np.int32)])
     _assert_report(rep, res)
 
