@@ -211,45 +211,44 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         ++qc;
       }
       // K: slot = (chunk c, channel half hh), bpc blocks of l keys each;
-      // V: slot = (chunk c, 64-key half hv), 64 / l blocks x D channels
+      // V: slot = (chunk c, 64-key half hv), 64 / l blocks x D channels.
+      // Slots go in pairs: lane 0 claims both, then one lane per copy issues
+      // (a thread streams one copy per few hundred cycles, so the copies of a
+      // pair are spread over up to eight lanes).
       const int per_chunk = is_k ? D / 64 : 2;
-      for (int c = 0; c < nsc && ok; ++c) {
-        for (int part = 0; part < per_chunk && ok; ++part) {
-          const int s = slot_uses % nslots, u = slot_uses / nslots;
-          const int nblk = is_k ? bpc : (64 >> lg_l);
-          const int bs0 = is_k ? c * bpc : c * bpc + part * nblk;
-          int rows[4];
-#pragma unroll
-          for (int sub = 0; sub < 4; ++sub) {
-            const int blk = __shfl_sync(0xffffffffu, idx, (bs0 + sub) & 31);
-            rows[sub] = (sub < nblk && bs0 + sub < n && blk >= 0) ? job.cu0 + (blk << lg_l)
-                                                                  : -(1 << 24);
-          }
-          if (lane == 0) {
+      const int nblk = is_k ? bpc : (64 >> lg_l);       // blocks per slot
+      const int cps = is_k ? nblk : nblk * (D / 64);    // copies per slot
+      const int slots_per_job = nsc * per_chunk;
+      for (int q0 = 0; q0 < slots_per_job && ok; q0 += 2) {
+        const int ns = slots_per_job - q0 < 2 ? slots_per_job - q0 : 2;
+        if (lane == 0) {
+          for (int i = 0; i < ns && ok; ++i) {
+            const int s = (slot_uses + i) % nslots, u = (slot_uses + i) / nslots;
             if (u > 0 && !mbar_wait(empty + s, (u - 1) & 1, abort_flag, status, kWaitCycles))
               ok = false;
-            if (ok) {
-              uint8_t* dst = sm + (is_k ? L::kK + s * L::kKBytes : L::kV + s * L::kVBytes);
+            else
               mbar_arrive_expect_tx(full + s, is_k ? L::kKBytes : L::kVBytes);
-#pragma unroll
-              for (int sub = 0; sub < 4; ++sub) {
-                if (sub < nblk) {
-                  if (is_k) {
-                    tma_load_3d(dst + sub * l * 128, &maps.k_blk, full + s, part * 64, job.g,
-                                rows[sub]);
-                  } else {
-#pragma unroll
-                    for (int dh = 0; dh < D / 64; ++dh)
-                      tma_load_3d(dst + dh * 8192 + sub * l * 128, &maps.v_blk, full + s,
-                                  dh * 64, job.g, rows[sub]);
-                  }
-                }
-              }
-            }
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          ++slot_uses;
         }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        // copy `lane`: slot q0 + lane / cps, copy e = lane % cps of that slot
+        const int qi = lane / cps, e = lane - qi * cps, q = q0 + qi;
+        const int c = q / per_chunk, part = q - c * per_chunk;
+        const int sub = is_k ? e : e / (D / 64);
+        const int dh = is_k ? part : e - sub * (D / 64);
+        const int bs = c * bpc + (is_k ? 0 : part * nblk) + sub;
+        const int blk = __shfl_sync(0xffffffffu, idx, bs & 31);
+        if (ok && qi < ns) {
+          const int s = (slot_uses + qi) % nslots;
+          const int row = (bs < n && blk >= 0) ? job.cu0 + (blk << lg_l) : -(1 << 24);
+          if (is_k)
+            tma_load_3d(sm + L::kK + s * L::kKBytes + sub * l * 128, &maps.k_blk, k_full + s,
+                        dh * 64, job.g, row);
+          else
+            tma_load_3d(sm + L::kV + s * L::kVBytes + dh * 8192 + sub * l * 128, &maps.v_blk,
+                        v_full + s, dh * 64, job.g, row);
+        }
+        if (ok) slot_uses += ns;  // slots with copies in flight (drained below)
       }
     }
     // drain: every issued copy has landed before the CTA retires (also after
