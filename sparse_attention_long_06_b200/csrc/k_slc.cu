@@ -178,8 +178,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
     // job ahead); lane 0 waits on the ring and issues the copies.
     const bool is_k = warp == 0;
     if (lane == 0) {
-      tma_prefetch_desc(is_k ? &maps.k_blk : &maps.v_blk);
-      if (is_k) tma_prefetch_desc(&maps.q_tok);
+      tma_prefetch_desc(is_k ? &maps.k_blk : (a.split_v ? &maps.v_split : &maps.v_blk));
+      if (is_k) tma_prefetch_desc(a.split_q ? &maps.q_split : &maps.q_tok);
     }
     int slot_uses = 0;  // ring slots filled so far
     int qc = 0;
@@ -201,10 +201,15 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
             ok = false;
           if (ok) {
             mbar_arrive_expect_tx(q_full + qs, q_heads * D * 2);
+            if (a.split_q) {
+              tma_load_4d(sm + L::kQ + qs * L::kQBytes, &maps.q_split, q_full + qs, 0, job.g * G,
+                          0, job.row);
+            } else {
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_3d(sm + L::kQ + qs * L::kQBytes + h * 2048, &maps.q_tok, q_full + qs,
-                          h * 64, job.g * G, job.row);
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_3d(sm + L::kQ + qs * L::kQBytes + h * 2048, &maps.q_tok, q_full + qs,
+                            h * 64, job.g * G, job.row);
+            }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -217,7 +222,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       // pair are spread over up to eight lanes).
       const int per_chunk = is_k ? D / 64 : 2;
       const int nblk = is_k ? bpc : (64 >> lg_l);       // blocks per slot
-      const int cps = is_k ? nblk : nblk * (D / 64);    // copies per slot
+      const bool v_one = !is_k && a.split_v;            // one copy brings a whole V block
+      const int cps = is_k ? nblk : (v_one ? 1 : nblk * (D / 64));  // copies per slot
       const int slots_per_job = nsc * per_chunk;
       for (int q0 = 0; q0 < slots_per_job && ok; q0 += 2) {
         const int ns = slots_per_job - q0 < 2 ? slots_per_job - q0 : 2;
@@ -234,8 +240,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         // copy `lane`: slot q0 + lane / cps, copy e = lane % cps of that slot
         const int qi = lane / cps, e = lane - qi * cps, q = q0 + qi;
         const int c = q / per_chunk, part = q - c * per_chunk;
-        const int sub = is_k ? e : e / (D / 64);
-        const int dh = is_k ? part : e - sub * (D / 64);
+        const int sub = is_k ? e : (v_one ? 0 : e / (D / 64));
+        const int dh = is_k ? part : (v_one ? 0 : e - sub * (D / 64));
         const int bs = c * bpc + (is_k ? 0 : part * nblk) + sub;
         const int blk = __shfl_sync(0xffffffffu, idx, bs & 31);
         if (ok && qi < ns) {
@@ -244,6 +250,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
           if (is_k)
             tma_load_3d(sm + L::kK + s * L::kKBytes + sub * l * 128, &maps.k_blk, k_full + s,
                         dh * 64, job.g, row);
+          else if (v_one)
+            tma_load_4d(sm + L::kV + s * L::kVBytes, &maps.v_split, v_full + s, 0, row, 0, job.g);
           else
             tma_load_3d(sm + L::kV + s * L::kVBytes + dh * 8192 + sub * l * 128, &maps.v_blk,
                         v_full + s, dh * 64, job.g, row);

@@ -123,6 +123,30 @@ bool encode4d(CUtensorMap* m, const void* base, int D, int heads, long long rows
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D view of a bf16 [rows, heads, D] tensor whose box brings both 64-channel
+// halves of `box_rows` consecutive rows of one head (or `box_heads` heads of
+// one row) in one copy, laid out [half][row or head][64 channels] in shared
+// memory: dims (64 channels, inner, D / 64 halves, outer).  `inner_is_rows`
+// picks (rows, heads) or (heads, rows) for the inner/outer dims.  Returns
+// false when the driver rejects the map (the kernels then use 3-D boxes).
+bool encode_split4d(CUtensorMap* m, const void* base, int D, int heads, long long rows,
+                    bool inner_is_rows, int box_inner) {
+  memset(m, 0, sizeof(*m));
+  if (rows <= 0) return false;
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t row_stride = (cuuint64_t)D * 2 * heads, head_stride = (cuuint64_t)D * 2;
+  cuuint64_t dims[4] = {64, inner_is_rows ? (cuuint64_t)rows : (cuuint64_t)heads,
+                        (cuuint64_t)(D / 64), inner_is_rows ? (cuuint64_t)heads : (cuuint64_t)rows};
+  cuuint64_t strides[3] = {inner_is_rows ? row_stride : head_stride, 128,
+                           inner_is_rows ? head_stride : row_stride};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_inner, (cuuint32_t)(D / 64), 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int num_sms_current() {
@@ -311,6 +335,16 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
             encode3d(&m.k_win, k, geo.D, geo.Hkv, total_tokens, 1, kChunk) &&
             encode3d(&m.v_win, v, geo.D, geo.Hkv, total_tokens, 1, kChunk);
   if (!ok) return NSA_ERR_CUDA;
+  // one-copy query rows (16 heads) and one-copy V blocks (64 keys), when the
+  // driver accepts the channel-split maps
+  a.split_q = geo.Hq >= 16 && encode_split4d(&m.q_split, q, geo.D, geo.Hq, total_tokens, false, 16);
+  a.split_v = geo.l == 64 && encode_split4d(&m.v_split, v, geo.D, geo.Hkv, total_tokens, true, 64);
+  static std::once_flag split_note;
+  if ((geo.Hq >= 16 && !a.split_q) || (geo.l == 64 && !a.split_v))
+    std::call_once(split_note, [] {
+      fprintf(stderr, "nsa_prefill: channel-split tensor maps rejected by the driver; "
+                      "using one copy per 64-channel half\n");
+    });
   const int sms = num_sms_current();
   if (sms <= 0) return NSA_ERR_CUDA;
 

@@ -69,11 +69,15 @@ struct PrefillArgs {
   float* lse;     // [T, Hq]
   float* scores;  // [T, Hkv, cmp_cap]
   float* o_win;   // [T, Hq, D] g_win * O_win
+  int split_q;    // PrefillMaps.q_split is valid (Hq >= 16)
+  int split_v;    // PrefillMaps.v_split is valid (l = 64)
 };
 
 struct PrefillMaps {
   CUtensorMap q;      // (D, Hq, T) box (64, G, tpt)
   CUtensorMap q_tok;  // (D, Hq, T) box (64, min(16, Hq), 1)
+  CUtensorMap q_split;  // (64, Hq, D/64, T) box (64, 16, D/64, 1): [half][head][64]
+  CUtensorMap v_split;  // (64, T, D/64, Hkv) box (64, l, D/64, 1): [half][key][64] (l = 64)
   CUtensorMap kc;     // (D, Hkv, cmp_rows) box (64, 1, 128)
   CUtensorMap vc;
   CUtensorMap k_blk;  // (D, Hkv, T) box (64, 1, l)
