@@ -12,10 +12,10 @@
 // 0 first).  The tile's window keys [t0 - w + 1, t0 + 128 / G - 1] are shared
 // by all of its rows and are streamed in chunks of 128 keys:
 //   pass 1: S = Q K^T (rows on TMEM lanes), masked to each row's window:
-//           running max and sum per row;
+//           row maximum;
 //   pass 2: S again, P = exp(s - max) (largest element exactly 1, K-major A
-//           operand in shared memory), O += P V in TMEM; the epilogue scales
-//           row r by g_win / sum.
+//           operand in shared memory) and its row sum in fp32, O += P V in
+//           TMEM; the epilogue scales row r by g_win / sum.
 // Warp roles: 0 = TMA producer, 1 = tcgen05.mma issuer, 2..5 and 6..9 = two
 // softmax warpgroups that take alternate key chunks of both passes (each with
 // its own TMEM score buffer and P buffer) and split the epilogue's columns
@@ -96,9 +96,9 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 22);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
   float* m_s = reinterpret_cast<float*>(sm + L::kStat);  // merged row max (scaled, log2)
-  float* l_s = m_s + 128;                                 // merged row sum
+  float* l_s = m_s + 128;                                 // row sum, warpgroup 0's part
   float* m1_s = m_s + 256;
-  float* l1_s = m_s + 384;
+  float* l1_s = m_s + 384;                                // row sum, warpgroup 1's part
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (a.meta->bad) return;
@@ -288,8 +288,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       // window keys of this row as offsets from the tile's first chunk key
       const int o_lo = max(t_row - wlen + 1, 0) - it.ws, o_hi = t_row - it.ws;
       const size_t orow = ((size_t)(it.row0 + i_row) * Hq + it.g * G + h_row);
-      // ---- pass 1: running max / sum per row over this warpgroup's chunks
-      float m = -INFINITY, lsum = 0.f;
+      // ---- pass 1: row maximum over this warpgroup's chunks (scaled, log2 units)
+      float m = -INFINITY;
       for (int c = w; c < it.nc; c += 2) {
         mbar_wait(s_full + w, s_use & 1, abort_flag, status, kWaitCycles);
         tc_fence_after();
@@ -310,40 +310,22 @@ __global__ void __launch_bounds__(kWinThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(s_empty + w);
           }
-          float cm = -INFINITY;
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const int o = half * 64 + j;
-            x[j] = (row_ok && o >= lo && o <= hi) ? x[j] * sl2 : -INFINITY;
-            cm = fmaxf(cm, x[j]);
-          }
-          const float mn = fmaxf(m, cm);
-          if (mn != -INFINITY) {
-            float s = 0.f;
-#pragma unroll
-            for (int j = 0; j < 64; ++j) s += ex2(x[j] - mn);
-            lsum = lsum * ex2(m - mn) + s;
-            m = mn;
+            if (row_ok && o >= lo && o <= hi) m = fmaxf(m, x[j]);
           }
         }
         ++s_use;
       }
-      // merge the two warpgroups' row statistics
-      if (w == 1) {
-        m1_s[r] = m;
-        l1_s[r] = lsum;
-      }
-      both_bar();  // every thread is also done with the previous tile's m_s / l_s
-      if (w == 0) {
-        const float m1 = m1_s[r], l1 = l1_s[r];
-        const float mm = fmaxf(m, m1);
-        float ls = 0.f;
-        if (mm != -INFINITY) ls = lsum * ex2(m - mm) + l1 * ex2(m1 - mm);
-        m_s[r] = mm;
-        l_s[r] = ls;
-      }
+      m *= sl2;
+      // merge the two warpgroups' row maxima
+      if (w == 1) m1_s[r] = m;
+      both_bar();  // every thread is also done with the previous tile's m_s / l_s / l1_s
+      if (w == 0) m_s[r] = fmaxf(m, m1_s[r]);
       both_bar();
       const float mrow = m_s[r];
+      float lsum = 0.f;  // this warpgroup's part of the row sum
       // ---- pass 2: P = exp2(s - max) into this warpgroup's P buffer (row r)
       for (int c = w; c < it.nc; c += 2) {
         mbar_wait(s_full + w, s_use & 1, abort_flag, status, kWaitCycles);
@@ -372,6 +354,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
               const float p1 = (row_ok && o0 + 1 >= lo && o0 + 1 <= hi)
                                    ? ex2(v[g8 * 8 + 2 * j + 1] * sl2 - mrow)
                                    : 0.f;
+              lsum += p0 + p1;
               pk[j] = pack_bf16x2(p0, p1);
             }
             st_shared_v4(prow + half * 16384 + ((g8 ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
@@ -388,9 +371,11 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         ++p_use;
       }
       // ---- epilogue: this warpgroup's half of the row, g_win * O / sum
+      (w == 0 ? l_s : l1_s)[r] = lsum;
+      both_bar();
+      const float ls = l_s[r] + l1_s[r];
       mbar_wait(o_full, oc & 1, abort_flag, status, kWaitCycles);
       tc_fence_after();
-      const float ls = l_s[r];
       const float gw = row_ok ? __ldg(a.gates + orow * 3 + 2) : 0.f;
       const float scale = ls > 0.f ? gw / ls : 0.f;
 #pragma unroll
