@@ -161,6 +161,7 @@ cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s) {
 __global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
+  __shared__ unsigned long long cand_all[8][kTopnCand];
   const int warp = threadIdx.x / 32;
   const int H = a.geo.Hkv, l = a.geo.l, n = a.geo.n;
   const long long row = (long long)blockIdx.x * 8 + warp;
@@ -170,8 +171,11 @@ __global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   const int t = tg - __ldg(a.cu + b);
   const float* S = a.scores + ((size_t)tg * H + g) * a.geo.cmp_cap;
   int* out = a.sel + ((size_t)tg * H + g) * n;
-  warp_topn([&](int j) { return S[j]; }, (t + 1) / l, t / l + 1, n, hist_all[warp],
-            [&](int i, int j) { out[i] = j; });
+  const int ncmp = (t + 1) / l, ncand = t / l + 1;
+  auto score = [&](int j) { return S[j]; };
+  auto put = [&](int i, int j) { out[i] = j; };
+  if (ncand <= 1024 && n <= 32 && warp_topn_regs(score, ncmp, ncand, n, cand_all[warp], put)) return;
+  warp_topn(score, ncmp, ncand, n, hist_all[warp], put);
 }
 
 cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s) {

@@ -42,11 +42,11 @@ namespace {
 
 template <int D>
 struct SlcLayout {
-  static constexpr int kQSlots = 4;
+  static constexpr int kQSlots = 2;
   static constexpr int kQBytes = 16 * D * 2;  // 16 query rows
-  static constexpr int kKSlots = 5;
+  static constexpr int kKSlots = 4;
   static constexpr int kKBytes = kChunk * 64 * 2;  // 128 keys x 64 channels
-  static constexpr int kVSlots = D == 128 ? 4 : 8;
+  static constexpr int kVSlots = D == 128 ? 5 : 8;
   static constexpr int kVBytes = 64 * D * 2;  // 64 keys x D channels
   static constexpr int kPBytes = 8 * 4096;    // P^T: up to 8 chunks x 128 keys x 16 heads
   static constexpr int kQ = 0;
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       nj = slc_job(a, blockIdx.x + (long long)(j + 1) * gridDim.x);
       nidx = job_sel(a, nj, lane);
       if (is_k) {
-        const int qs = qc & 3, u = qc >> 2;
+        const int qs = qc % L::kQSlots, u = qc / L::kQSlots;
         if (lane == 0) {
           if (u > 0 && !mbar_wait(q_empty + qs, (u - 1) & 1, abort_flag, status, kWaitCycles))
             ok = false;
@@ -267,9 +267,9 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         const int last = slot_uses - 1 - ((slot_uses - 1 - s) % nslots);
         mbar_wait(full + s, (last / nslots) & 1, &never, nullptr, kWaitCycles / 4);
       }
-      for (int qs = 0; qs < 4 && qs < qc; ++qs) {
-        const int last = qc - 1 - ((qc - 1 - qs) % 4);
-        mbar_wait(q_full + qs, (last >> 2) & 1, &never, nullptr, kWaitCycles / 4);
+      for (int qs = 0; qs < L::kQSlots && qs < qc; ++qs) {
+        const int last = qc - 1 - ((qc - 1 - qs) % L::kQSlots);
+        mbar_wait(q_full + qs, (last / L::kQSlots) & 1, &never, nullptr, kWaitCycles / 4);
       }
     }
   } else if (warp == 1) {
@@ -279,8 +279,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       int kc = 0;
       bool ok = true;
       for (int j = 0; j < njobs && ok; ++j) {
-        const int qs = j & 3, buf = j & 1, u = j >> 1;
-        if (!mbar_wait(q_full + qs, (j >> 2) & 1, abort_flag, status, kWaitCycles) ||
+        const int qs = j % L::kQSlots, buf = j & 1, u = j >> 1;
+        if (!mbar_wait(q_full + qs, (j / L::kQSlots) & 1, abort_flag, status, kWaitCycles) ||
             (u > 0 && !mbar_wait(s_empty + buf, (u - 1) & 1, abort_flag, status, kWaitCycles))) {
           ok = false;
           break;

@@ -92,4 +92,81 @@ __device__ __forceinline__ void warp_topn(ScoreFn score, int ncmp, int ncand, in
   for (int j = written + lane; j < n; j += 32) out(j, -1);
 }
 
+// Register path of the same selection for rows with at most 1024 candidates
+// (32 per lane).  Every candidate j gets the 64-bit key (score bits << 32) |
+// (0xFFFFFFFF - j), so larger keys rank first and equal scores rank by lower
+// index; keys are distinct.  The n-th largest of the 32 per-lane maxima is a
+// lower bound T0 of the n-th largest key (n lanes hold a key >= it); the keys
+// >= T0 (normally a few dozen) are ranked exactly in shared memory (`cand`,
+// kCand words per warp) to find the n-th largest key K, and every key >= K is
+// emitted in ascending block order.  Returns false, having written nothing,
+// when more than kCand keys reach T0; the caller then uses warp_topn.
+constexpr int kTopnCand = 64;
+
+template <typename ScoreFn, typename OutFn>
+__device__ __forceinline__ bool warp_topn_regs(ScoreFn score, int ncmp, int ncand, int n,
+                                               unsigned long long* cand, OutFn out) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  if (ncand <= n) {
+    for (int j = lane; j < n; j += 32) out(j, j < ncand ? j : -1);
+    return true;
+  }
+  unsigned long long key[32];
+  unsigned long long lmax = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int j = lane + 32 * i;
+    const uint32_t b = j < ncmp ? __float_as_uint(score(j)) : 0u;
+    key[i] = j < ncand ? (((unsigned long long)b << 32) | (0xFFFFFFFFu - (uint32_t)j)) : 0ull;
+    lmax = key[i] > lmax ? key[i] : lmax;
+  }
+  // T0 = n-th largest lane maximum (at least n + 1 lanes hold candidates)
+  int rank = 0;
+#pragma unroll
+  for (int o = 0; o < 32; ++o) {
+    const unsigned long long other = __shfl_sync(0xffffffffu, lmax, o);
+    rank += other > lmax;
+  }
+  const unsigned tb = __ballot_sync(0xffffffffu, rank == n - 1 && lmax != 0ull);
+  const unsigned long long t0 = __shfl_sync(0xffffffffu, lmax, __ffs(tb) - 1);
+  // gather the keys >= T0
+  int count = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const bool p = key[i] >= t0 && key[i] != 0ull;
+    const unsigned m = __ballot_sync(0xffffffffu, p);
+    const int pos = count + __popc(m & lt_mask);
+    if (p && pos < kTopnCand) cand[pos] = key[i];
+    count += __popc(m);
+  }
+  if (count > kTopnCand) return false;
+  __syncwarp();
+  // K = n-th largest gathered key
+  unsigned long long kth = 0ull;
+  bool have = false;
+  for (int c = lane; c < count; c += 32) {
+    const unsigned long long mine = cand[c];
+    int r = 0;
+    for (int d = 0; d < count; ++d) r += cand[d] > mine;
+    if (r == n - 1) {
+      kth = mine;
+      have = true;
+    }
+  }
+  const unsigned hb = __ballot_sync(0xffffffffu, have);
+  kth = __shfl_sync(0xffffffffu, kth, __ffs(hb) - 1);
+  __syncwarp();
+  // every key >= K, in ascending block order
+  int written = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const bool take = key[i] >= kth && key[i] != 0ull;
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (take) out(written + __popc(m & lt_mask), lane + 32 * i);
+    written += __popc(m);
+  }
+  return true;
+}
+
 }  // namespace nsa
