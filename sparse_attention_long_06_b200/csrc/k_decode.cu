@@ -10,12 +10,13 @@
 // nsa_decode_kernel: one CTA per (sequence, KV group), the group's G heads
 // sharing every load.  All products are swap-AB tcgen05 MMAs with 128 keys on
 // the TMEM lanes and the heads on 16 columns (S^T = K Q^T, O^T += V^T P^T):
-//   window    the w tokens ending at t (chunks end at t, so no cache row past
-//             the sequence is read), two-sweep softmax, O_win;
 //   compressed all complete blocks (chunks end at the last one), two-sweep
 //             softmax, O_cmp, and a third sweep for the block scores
 //             S_j = sum over heads of the normalised probabilities;
-//   top-n     one warp selects n blocks from the scores in shared memory;
+//   top-n     one warp selects n blocks from the scores in shared memory
+//             (the window's keys and values stream in meanwhile);
+//   window    the w tokens ending at t (chunks end at t, so no cache row past
+//             the sequence is read), two-sweep softmax, O_win;
 //   selected  the chosen blocks (the incomplete block is loaded as the l rows
 //             ending at t), two-sweep softmax, O_slc;
 //   epilogue  out = g_cmp O_cmp + g_slc O_slc + g_win O_win, lane = channel.
@@ -237,10 +238,12 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive_expect_tx(q_full, qrows * D * 2);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) tma_load_3d(sm + L::kQ + h * 2048, &maps.q, q_full, h * 64, g * G, b);
-      for (int c = 0; c < it.nwc && ok; ++c) load_rows(&maps.k_win, win_row0 + c * kChunk);
+      // compressed keys first: the block scores (and the top-n that the
+      // selected loads wait for) are computed while the rest streams in
       for (int c = 0; c < it.ncc && ok; ++c) load_rows(&maps.kc, cmp_row0 + c * kChunk);
-      for (int c = 0; c < it.nwc && ok; ++c) load_rows(&maps.v_win, win_row0 + c * kChunk);
+      for (int c = 0; c < it.nwc && ok; ++c) load_rows(&maps.k_win, win_row0 + c * kChunk);
       for (int c = 0; c < it.ncc && ok; ++c) load_rows(&maps.vc, cmp_row0 + c * kChunk);
+      for (int c = 0; c < it.nwc && ok; ++c) load_rows(&maps.v_win, win_row0 + c * kChunk);
       if (ok && mbar_wait(idx_ready, 0, abort_flag, status, kWaitCycles)) {
         load_sel(false);
         if (ok) load_sel(true);
@@ -300,22 +303,22 @@ __global__ void __launch_bounds__(192, 1)
           release_stage();
         }
       };
+      if (ok && it.ncc > 0) {
+        qk(it.ncc, kColSC);
+        mma_commit(sC_full);
+      }
       if (ok) {
         qk(it.nwc, kColSW);
         mma_commit(sW_full);
       }
-      if (ok && it.ncc > 0) {
-        qk(it.ncc, kColSC);
-        mma_commit(sC_full);
+      if (ok && it.ncc > 0 && mbar_wait(pC_full, 0, abort_flag, status, kWaitCycles)) {
+        tc_fence_after();
+        pv(it.ncc, Ps + L::kPBytes, kColOC);
       }
       if (ok && mbar_wait(pW_full, 0, abort_flag, status, kWaitCycles)) {
         tc_fence_after();
         pv(it.nwc, Ps, kColOW);
         mma_commit(pW_empty);
-      }
-      if (ok && it.ncc > 0 && mbar_wait(pC_full, 0, abort_flag, status, kWaitCycles)) {
-        tc_fence_after();
-        pv(it.ncc, Ps + L::kPBytes, kColOC);
       }
       if (ok) {
         qk(it.nsc, kColSS);
@@ -404,19 +407,6 @@ __global__ void __launch_bounds__(192, 1)
     };
     const uint32_t P0 = sbase + L::kP, P1 = P0 + L::kPBytes;
     float inv_w[16], inv_c[16], inv_s[16];
-    // ---- window
-    {
-      bool kok[8];
-      const int lo = max(0, t - a.geo.w + 1);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) kok[c] = c < it.nwc && win_row0 + c * kChunk + r >= lo;
-      mbar_wait(sW_full, 0, abort_flag, status, kWaitCycles);
-      tc_fence_after();
-      softmax(kColSW, it.nwc, kok, P0, inv_w);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pW_full);
-    }
     // ---- compressed branch and block scores
 #pragma unroll
     for (int h = 0; h < 16; ++h) inv_c[h] = 0.f;
@@ -511,6 +501,19 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) mbar_arrive(idx_ready);
     }
     named_bar_128<1>();
+    // ---- window
+    {
+      bool kok[8];
+      const int lo = max(0, t - a.geo.w + 1);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) kok[c] = c < it.nwc && win_row0 + c * kChunk + r >= lo;
+      mbar_wait(sW_full, 0, abort_flag, status, kWaitCycles);
+      tc_fence_after();
+      softmax(kColSW, it.nwc, kok, P0, inv_w);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pW_full);
+    }
     // ---- selected branch
     {
       bool kok[8];
