@@ -91,8 +91,9 @@ struct Pass2Rows {
 // p (the G heads of a token are G consecutive columns of this thread), and
 // p * rowsum (= exp2(s - row max), largest element exactly 1) into P^T as
 // bf16 in the 128-byte-swizzled MN-major layout.
-template <int G>
+template <int G, bool kFull>
 __device__ __forceinline__ void pass2_rows(const Pass2Rows& a) {
+  const bool live = !*a.abort_flag;
 #pragma unroll
   for (int grp = 0; grp < kTileRows / 16; ++grp) {
     float v[16];
@@ -109,7 +110,8 @@ __device__ __forceinline__ void pass2_rows(const Pass2Rows& a) {
       for (int jj = 0; jj < 4; ++jj) {
         const int j = j4 * 4 + jj;
         const int row = grp * 16 + j;
-        p[j] = (row >= a.row_lo && row < a.row_hi) ? ex2(v[j] * a.sl2 - lsv[jj]) : 0.f;
+        p[j] = (kFull || (row >= a.row_lo && row < a.row_hi)) ? ex2(fmaf(v[j], a.sl2, -lsv[jj]))
+                                                               : 0.f;
         pm[j] = p[j] * suv[jj];
       }
     }
@@ -119,7 +121,7 @@ __device__ __forceinline__ void pass2_rows(const Pass2Rows& a) {
 #pragma unroll
       for (int j = 0; j < G; ++j) ts += p[kt * G + j];
       const int row = grp * 16 + kt * G;
-      if (row >= a.row_lo && row < a.row_hi && !*a.abort_flag)
+      if ((kFull || (row >= a.row_lo && row < a.row_hi)) && live)
         a.srow[(size_t)(row / G) * a.tok_stride] = ts;
     }
     uint32_t pk[8];
@@ -388,18 +390,29 @@ __global__ void __launch_bounds__(kCmpThreads, 1)
             if (lane == 0) mbar_arrive(s_empty + w);
           }
           float cm = -INFINITY;
+          if (jmax >= (half + 1) * 64) {  // every column of this half is visible
 #pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            x[j] = (half * 64 + j) < jmax ? x[j] * sl2 : -INFINITY;
-            cm = fmaxf(cm, x[j]);
-          }
-          const float mn = fmaxf(m, cm);
-          if (mn != -INFINITY) {
+            for (int j = 0; j < 64; ++j) cm = fmaxf(cm, x[j]);
+            const float mn = fmaxf(m, cm * sl2);
             float s = 0.f;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) s += ex2(x[j] - mn);
+            for (int j = 0; j < 64; ++j) s += ex2(fmaf(x[j], sl2, -mn));
             lsum = lsum * ex2(m - mn) + s;
             m = mn;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              x[j] = (half * 64 + j) < jmax ? x[j] * sl2 : -INFINITY;
+              cm = fmaxf(cm, x[j]);
+            }
+            const float mn = fmaxf(m, cm);
+            if (mn != -INFINITY) {
+              float s = 0.f;
+#pragma unroll
+              for (int j = 0; j < 64; ++j) s += ex2(x[j] - mn);
+              lsum = lsum * ex2(m - mn) + s;
+              m = mn;
+            }
           }
         }
         ++s_use;
@@ -434,12 +447,21 @@ __global__ void __launch_bounds__(kCmpThreads, 1)
         float* srow = a.scores + ((size_t)it.row0 * Hkv + it.g) * cap + key;
         const Pass2Rows rows{lane_addr + w * 128, lse_s, sum_s, sl2, row_lo, row_hi, prow, r,
                              srow, (size_t)Hkv * cap, abort_flag};
-        switch (lgG) {
-          case 0: pass2_rows<1>(rows); break;
-          case 1: pass2_rows<2>(rows); break;
-          case 2: pass2_rows<4>(rows); break;
-          case 3: pass2_rows<8>(rows); break;
-          default: pass2_rows<16>(rows); break;
+        // rows (token, head) of the tile all see every key of this warp: no
+        // per-row test.  Warp-uniform, because pass2_rows issues warp-wide
+        // (.sync.aligned) TMEM loads.
+        const bool full = __all_sync(0xffffffffu, row_lo == 0 && row_hi == kTileRows);
+        switch (lgG * 2 + (full ? 1 : 0)) {
+          case 0: pass2_rows<1, false>(rows); break;
+          case 1: pass2_rows<1, true>(rows); break;
+          case 2: pass2_rows<2, false>(rows); break;
+          case 3: pass2_rows<2, true>(rows); break;
+          case 4: pass2_rows<4, false>(rows); break;
+          case 5: pass2_rows<4, true>(rows); break;
+          case 6: pass2_rows<8, false>(rows); break;
+          case 7: pass2_rows<8, true>(rows); break;
+          case 8: pass2_rows<16, false>(rows); break;
+          default: pass2_rows<16, true>(rows); break;
         }
         fence_async_smem();
         tc_fence_before();
