@@ -53,6 +53,23 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(x, world, device):
+    """The largest of every rank's `x` (device time of the slowest replica);
+    every rank must call it at the same point."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, ms):
+    """Whole-job throughput: the units all ranks processed over the max time."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 # ---------------------------------------------------------------- algorithmic work
 def algorithmic_flops(cfg, T, sel):
     """Exact FLOPs of the method on one sequence (the work it does, not the
@@ -231,16 +248,12 @@ def run_ours(args, rank, world):
     if world > 1:
         torch.distributed.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     status = nsa.read_device_status(ws)
     if status != nsa.NSA_OK:
         raise RuntimeError(f"device status {nsa.strerror(status)} in the timed region")
     ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step / 1e3)
+    value = job_rate(T, world, ms_per_step)
 
     # per-launch times (same stream, events recorded by the library)
     nsa.profile_enable(True)
@@ -282,12 +295,8 @@ def run_ours(args, rank, world):
         torch.cuda.synchronize()
         if i > 0:
             e2e_ms.append(a.elapsed_time(b))
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = world * T / (e2e_total / len(e2e_ms) / 1e3)
+    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
+    e2e_value = job_rate(T, world, e2e_total / len(e2e_ms))
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -312,7 +321,7 @@ def run_ours(args, rank, world):
     if not args.no_decode:
         del d, host
         torch.cuda.empty_cache()
-        result["decode"] = run_decode_leg(args, dev)
+        result["decode"] = run_decode_leg(args, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(cfg, inputs)
     return result
@@ -339,7 +348,7 @@ def decode_bytes(cfg, lens, sel):
     return total
 
 
-def run_decode_leg(args, dev):
+def run_decode_leg(args, dev, world=1):
     import torch
     from sparse_attention_long_06_b200 import nsa
     cfg = wl.CONFIGS["decode_64k"]
@@ -377,7 +386,7 @@ def run_decode_leg(args, dev):
         ev[i][1].record()
     torch.cuda.synchronize()
     ms = [a.elapsed_time(b) for a, b in ev]
-    med = statistics.median(ms)
+    med = max_over_ranks(statistics.median(ms), world, dev)
     nsa.profile_enable(True)
     flush.zero_()
     step()
@@ -387,7 +396,7 @@ def run_decode_leg(args, dev):
     hbm, _, _, src = _peaks()
     gbs = nbytes / (med / 1e3) / 1e9
     kgbs = nbytes / (stage[1] / 1e3) / 1e9
-    return {"metric": "NSA decode tokens/s", "value": round(B / (med / 1e3), 1), "unit": "tokens/s",
+    return {"metric": "NSA decode tokens/s", "value": round(job_rate(B, world, med), 1), "unit": "tokens/s",
             "ms_per_step_median": round(med, 5), "steps": steps,
             "config": {"workload": cfg.name, "batch": B, "context": int(cfg.decode_len),
                        "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
@@ -462,7 +471,7 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     if args.decode_only:
-        res = run_decode_leg(args, torch.device("cuda", torch.cuda.current_device()))
+        res = run_decode_leg(args, torch.device("cuda", torch.cuda.current_device()), world)
     else:
         res = run_ours(args, rank, world)
     if world > 1:

@@ -76,6 +76,13 @@ def test_plan_sizes(L):
     assert off % 256 == 0 and nb == T * Hq * D * 4
     off2, nb2 = p.workspace_region(nsa.WS_SCORES)
     assert off2 >= off + nb and nb2 == T * Hkv * 1024 * 4 and off2 + nb2 <= ws
+    # every region is 256-byte aligned, inside the workspace, and disjoint
+    regions = sorted(p.workspace_region(r) for r in (nsa.WS_O_CMP, nsa.WS_LSE, nsa.WS_SCORES,
+                                                     nsa.WS_SEL, nsa.WS_WIN))
+    for (o1, n1), (o2, _) in zip(regions, regions[1:]):
+        assert o1 % 256 == 0 and o1 + n1 <= o2
+    assert regions[-1][0] + regions[-1][1] <= ws
+    assert p.workspace_region(nsa.WS_WIN)[1] == T * Hq * D * 4
     assert p.cmp_rows(65536) == 1024 and p.cmp_rows(100) == 1
     assert nsa.Plan(**_params(head_dim=64, num_q_heads=4, num_kv_heads=1, cmp_block=32,
                               cmp_stride=32, sel_block=32, top_n=4, window=128)).workspace_size() > 0
