@@ -137,7 +137,10 @@ class Plan:
 
     def close(self):
         if getattr(self, "handle", None) is not None and self.handle.value:
-            lib().nsa_plan_destroy(self.handle)
+            try:
+                lib().nsa_plan_destroy(self.handle)
+            except (TypeError, AttributeError):  # interpreter shutdown: module state is gone
+                pass
             self.handle = None
 
     __del__ = close

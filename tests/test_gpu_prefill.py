@@ -74,6 +74,7 @@ def test_tiny_config_all_rows():
     (64, 8, 4, 64, 3, 64, [900]),                          # G = 2
     (128, 8, 8, 32, 32, 1000, [2000]),                     # G = 1, n = 32 (l = 32), w >= T/2
     (128, 32, 2, 64, 16, 4096, [1024]),                    # dense reduction: n >= blocks, w >= T
+    (64, 4, 1, 32, 4, 128, [200, 0, 130, 0]),              # empty sequences inside and at the end
 ])
 def test_edge_geometries(case):
     D, Hq, Hkv, l, n, w, lens = case
@@ -114,6 +115,26 @@ def test_prefill_64k_sampled_rows():
     rows = [gu.sample_rows(65536, 96, 11, 8, 64)]
     rep = gu.check_prefill(cfg, inputs, res, rows)
     _assert_report(rep, res)
+
+
+def test_empty_prefill_is_a_no_op():
+    import torch
+    cfg = _custom("empty", 64, 4, 1, 32, 4, 128, [100])
+    plan = nsa.Plan.for_config(cfg, 2, 128, 128)
+    inputs = wl.prefill_inputs(cfg)
+
+    def e(*shape, dt=torch.int16):
+        return torch.empty(shape, dtype=dt, device="cuda")
+
+    w_k = torch.from_numpy(inputs["w_k"]).cuda()
+    w_v = torch.from_numpy(inputs["w_v"]).cuda()
+    ws = plan.alloc_workspace()
+    cu = torch.zeros(3, dtype=torch.int32, device="cuda")  # two sequences of length 0
+    plan.prefill(e(0, 4, 64), e(0, 1, 64), e(0, 1, 64), e(0, 4, 3, dt=torch.float32), w_k, w_v,
+                 cu, e(0, 4, 64, dt=torch.float32), None, None, ws)
+    torch.cuda.synchronize()
+    assert nsa.last_launch_count() == 0
+    assert nsa.read_device_status(ws) == nsa.NSA_OK
 
 
 def test_repeated_calls_are_deterministic():
