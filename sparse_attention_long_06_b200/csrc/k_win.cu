@@ -20,6 +20,8 @@
 // softmax warpgroups that take alternate key chunks of both passes (each with
 // its own TMEM score buffer and P buffer) and split the epilogue's columns
 // (thread i of warp w owns TMEM lane 32 * (w % 4) + i).
+#include <type_traits>
+
 #include "nsa_internal.cuh"
 #include "sm100.cuh"
 
@@ -48,8 +50,16 @@ struct WinLayout {
 constexpr int kWinThreads = 320;
 
 struct WinItem {
-  int valid, b, g, t0, T, row0, ntok, ws, nc, cu0;
+  int valid, b, g, t0, T, row0, ntok, ws, nc, cu0, span;
 };
+
+// Keys of chunk c that lie in the tile's window span, rounded up to a
+// multiple of 16 (the N of its QK^T and 16 x the K-steps of its PV): the
+// last chunk of a span of w + 128/G - 1 keys is mostly empty.
+__device__ __forceinline__ int chunk_width(const WinItem& it, int c) {
+  const int rem = it.span - c * kChunk;
+  return ((rem < kChunk ? rem : kChunk) + 15) & ~15;
+}
 
 __device__ __forceinline__ WinItem win_item(const PrefillArgs& a, int k) {
   WinItem it{};
@@ -70,7 +80,8 @@ __device__ __forceinline__ WinItem win_item(const PrefillArgs& a, int k) {
   const int first = max(it.ws, 0);
   it.ws = first == 0 ? 0 : it.ws;
   const int last = it.t0 + it.ntok - 1;
-  it.nc = (last - it.ws + kChunk) / kChunk;
+  it.span = last - it.ws + 1;
+  it.nc = (it.span + kChunk - 1) / kChunk;
   return it;
 }
 
@@ -191,13 +202,13 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t id_pv = idesc_bf16(128, D, false, true);
       int qc = 0, sc = 0, oc = 0;
       int s_use[2] = {0, 0}, p_use[2] = {0, 0};
       bool ok = true;
       // chunk c goes to TMEM score buffer c & 1 (owned by warpgroup c & 1)
-      auto qk = [&](int qb, int c) {
+      auto qk = [&](int qb, int c, int cw) {
+        const uint32_t id_qk = idesc_bf16(128, cw, false, false);
         const int s = sc % L::kStages;
         if (!mbar_wait(st_full + s, (sc / L::kStages) & 1, abort_flag, status, kWaitCycles)) {
           ok = false;
@@ -222,7 +233,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         ++sc;
         ++s_use[buf];
       };
-      auto pv = [&](int c) {
+      auto pv = [&](int c, int cw) {
         const int s = sc % L::kStages, pb = c & 1;
         if (!mbar_wait(st_full + s, (sc / L::kStages) & 1, abort_flag, status, kWaitCycles) ||
             !mbar_wait(p_full + pb, p_use[pb] & 1, abort_flag, status, kWaitCycles)) {
@@ -236,8 +247,7 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         tc_fence_after();
         const uint32_t stage = sbase + L::kRing + s * L::kChunkBytes;
         const uint32_t P = sbase + L::kP + pb * L::kPBytes;
-#pragma unroll
-        for (int ks = 0; ks < kChunk / 16; ++ks)
+        for (int ks = 0; ks < cw / 16; ++ks)
           mma_bf16_ss(tmem + 256, smem_desc(P + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSw128),
                       smem_desc(stage + ks * 2048, 16384, 1024, kLayoutSw128), id_pv,
                       (c > 0 || ks > 0) ? 1u : 0u);
@@ -251,11 +261,11 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         if (!it.valid) break;
         const int qb = qc & 1;
         if (!mbar_wait(q_full + qb, (qc >> 1) & 1, abort_flag, status, kWaitCycles)) break;
-        for (int c = 0; c < it.nc && ok; ++c) qk(qb, c);
-        if (ok) qk(qb, 0);
+        for (int c = 0; c < it.nc && ok; ++c) qk(qb, c, chunk_width(it, c));
+        if (ok) qk(qb, 0, chunk_width(it, 0));
         for (int c = 0; c < it.nc && ok; ++c) {
-          if (c + 1 < it.nc) qk(qb, c + 1);
-          if (ok) pv(c);
+          if (c + 1 < it.nc) qk(qb, c + 1, chunk_width(it, c + 1));
+          if (ok) pv(c, chunk_width(it, c));
         }
         if (!ok) break;
         mma_commit(o_full);
@@ -294,28 +304,43 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         mbar_wait(s_full + w, s_use & 1, abort_flag, status, kWaitCycles);
         tc_fence_after();
         const int lo = o_lo - c * kChunk, hi = o_hi - c * kChunk;
+        // 16-column groups holding keys, and 64-column halves holding them
+        // (tile-uniform: the TMEM loads below are warp-wide)
+        const int ngc = chunk_width(it, c) >> 4;
+        auto chunk_max = [&](auto full_tag) {
+          constexpr bool kFull = decltype(full_tag)::value;
+          const int ng = kFull ? 8 : ngc, nh = kFull ? 2 : (ngc + 3) >> 2;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float x[64];
+          for (int half = 0; half < 2; ++half) {
+            if (!kFull && half >= nh) break;
+            float x[64];
 #pragma unroll
-          for (int g4 = 0; g4 < 4; ++g4) {
-            float v[16];
-            tmem_ld16(lane_addr + w * 128 + half * 64 + g4 * 16, v);
+            for (int g4 = 0; g4 < 4; ++g4) {
+              float v[16];
+              if (kFull || half * 4 + g4 < ng) {
+                tmem_ld16(lane_addr + w * 128 + half * 64 + g4 * 16, v);
+              } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) x[g4 * 16 + j] = v[j];
+                for (int j = 0; j < 16; ++j) v[j] = 0.f;  // past the span: masked below
+              }
+#pragma unroll
+              for (int j = 0; j < 16; ++j) x[g4 * 16 + j] = v[j];
+            }
+            tmem_ld_wait();
+            if (half == nh - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(s_empty + w);
+            }
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+              const int o = half * 64 + j;
+              if (row_ok && o >= lo && o <= hi) m = fmaxf(m, x[j]);
+            }
           }
-          tmem_ld_wait();
-          if (half == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_empty + w);
-          }
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const int o = half * 64 + j;
-            if (row_ok && o >= lo && o <= hi) m = fmaxf(m, x[j]);
-          }
-        }
+        };
+        if (ngc == 8) chunk_max(std::true_type{});
+        else chunk_max(std::false_type{});
         ++s_use;
       }
       m *= sl2;
@@ -333,33 +358,47 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         if (p_use > 0) mbar_wait(p_empty + w, (p_use - 1) & 1, abort_flag, status, kWaitCycles);
         const int lo = o_lo - c * kChunk, hi = o_hi - c * kChunk;
         const uint32_t prow = sbase + L::kP + w * L::kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+        const int ngc = chunk_width(it, c) >> 4;
+        auto chunk_p = [&](auto full_tag) {
+          constexpr bool kFull = decltype(full_tag)::value;
+          const int ng = kFull ? 8 : ngc, nh = kFull ? 2 : (ngc + 3) >> 2;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float v[64];
+          for (int half = 0; half < 2; ++half) {
+            if (!kFull && half >= nh) break;
+            float v[64];
 #pragma unroll
-          for (int g4 = 0; g4 < 4; ++g4) {
-            float u16[16];
-            tmem_ld16(lane_addr + w * 128 + half * 64 + g4 * 16, u16);
+            for (int g4 = 0; g4 < 4; ++g4) {
+              float u16[16];
+              if (kFull || half * 4 + g4 < ng) {
+                tmem_ld16(lane_addr + w * 128 + half * 64 + g4 * 16, u16);
+              } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[g4 * 16 + j] = u16[j];
-          }
-          tmem_ld_wait();
+                for (int j = 0; j < 16; ++j) u16[j] = 0.f;
+              }
 #pragma unroll
-          for (int g8 = 0; g8 < 8; ++g8) {  // 8 keys per 16-byte chunk of the row
-            uint32_t pk[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int o0 = half * 64 + g8 * 8 + 2 * j;
-              const float p0 = (row_ok && o0 >= lo && o0 <= hi) ? ex2(v[g8 * 8 + 2 * j] * sl2 - mrow) : 0.f;
-              const float p1 = (row_ok && o0 + 1 >= lo && o0 + 1 <= hi)
-                                   ? ex2(v[g8 * 8 + 2 * j + 1] * sl2 - mrow)
-                                   : 0.f;
-              lsum += p0 + p1;
-              pk[j] = pack_bf16x2(p0, p1);
+              for (int j = 0; j < 16; ++j) v[g4 * 16 + j] = u16[j];
             }
-            st_shared_v4(prow + half * 16384 + ((g8 ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int g8 = 0; g8 < 8; ++g8) {  // 8 keys per 16-byte chunk of the row
+              if (!kFull && half * 8 + g8 >= 2 * ng) break;  // columns the PV does not read
+              uint32_t pk[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int o0 = half * 64 + g8 * 8 + 2 * j;
+                const float p0 = (row_ok && o0 >= lo && o0 <= hi) ? ex2(v[g8 * 8 + 2 * j] * sl2 - mrow) : 0.f;
+                const float p1 = (row_ok && o0 + 1 >= lo && o0 + 1 <= hi)
+                                     ? ex2(v[g8 * 8 + 2 * j + 1] * sl2 - mrow)
+                                     : 0.f;
+                lsum += p0 + p1;
+                pk[j] = pack_bf16x2(p0, p1);
+              }
+              st_shared_v4(prow + half * 16384 + ((g8 ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
+            }
           }
-        }
+        };
+        if (ngc == 8) chunk_p(std::true_type{});
+        else chunk_p(std::false_type{});
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
