@@ -13,7 +13,7 @@ namespace nsa {
 constexpr int kTileRows = 128;
 // Keys per MMA chunk (M of the swap-AB products, N of the dense ones).
 constexpr int kChunk = 128;
-// Fixed upper bound on persistent CTAs (scratch regions are sized for it).
+// Upper bound on persistent CTAs (grids are min(SM count, this)).
 constexpr int kMaxPersistentCtas = 256;
 // Header of every workspace: status word and counters.
 constexpr size_t kHeaderBytes = 256;
