@@ -189,6 +189,47 @@ def traffic_record(kernel, src_file):
         return None
 
 
+# ---------------------------------------------------------------- end to end
+def e2e_pipelined(plan, host, d, out, kc, vc, sel, ws, out_host, steps):
+    """Mean ms per step of `steps` prefill calls through the public API, each
+    uploading its inputs from pinned host memory and downloading its output,
+    with upload / kernels / download on three streams and two device buffer
+    sets so that consecutive steps overlap."""
+    import torch
+    dsets = [d, {k: torch.empty_like(v) for k, v in d.items()}]
+    outs = [out, torch.empty_like(out)]
+    hosts_out = [out_host, torch.empty_like(out_host).pin_memory()]
+    s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(steps)]
+    c_done = [torch.cuda.Event() for _ in range(steps)]
+    out_done = [torch.cuda.Event() for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(s_in)
+    for i in range(steps):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(c_done[i - 2])  # kernels of step i-2 are done with set b
+            for k in dsets[b]:
+                dsets[b][k].copy_(host[k], non_blocking=True)
+            in_done[i].record(s_in)
+        s_c.wait_event(in_done[i])
+        if i >= 2:
+            s_c.wait_event(out_done[i - 2])  # download of step i-2 is done with outs[b]
+        ds = dsets[b]
+        plan.prefill(ds["q"], ds["k"], ds["v"], ds["gates"], ds["w_k"], ds["w_v"], ds["cu_seqlens"],
+                     outs[b], kc, vc, ws, sel_idx=sel, stream=s_c)
+        c_done[i].record(s_c)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(c_done[i])
+            hosts_out[b].copy_(outs[b], non_blocking=True)
+            out_done[i].record(s_out)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world):
     import torch
@@ -278,25 +319,16 @@ def run_ours(args, rank, world):
     dominant = max(TENSOR_KERNELS, key=lambda k: stage_ms[TENSOR_KERNELS[k][0]])
     roofline = rooflines[dominant]
 
-    # end to end through the public API with host buffers
-    e2e_steps = max(2, min(5, args.steps))
+    # end to end through the public API with host buffers: every step uploads
+    # its inputs from pinned host memory and downloads its output; steps are
+    # pipelined as a server would run them (upload of step i+1 and download of
+    # step i-1 overlap the kernels of step i, on two device buffer sets)
+    e2e_steps = max(4, min(8, args.steps))
     h2d = sum(host[k].numel() * host[k].element_size() for k in host)
     d2h = out_host.numel() * out_host.element_size()
-    e2e_ms = []
-    for i in range(e2e_steps + 1):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        a.record()
-        for k in d:
-            d[k].copy_(host[k], non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
-        b.record()
-        torch.cuda.synchronize()
-        if i > 0:
-            e2e_ms.append(a.elapsed_time(b))
-    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
-    e2e_value = job_rate(T, world, e2e_total / len(e2e_ms))
+    e2e_step_ms = e2e_pipelined(plan, host, d, out, kc, vc, sel, ws, out_host, e2e_steps)
+    e2e_ms_max = max_over_ranks(e2e_step_ms, world, dev)
+    e2e_value = job_rate(T, world, e2e_ms_max)
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -314,7 +346,9 @@ def run_ours(args, rank, world):
         "roofline": roofline,
         "rooflines": rooflines,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
+                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms_max, 3),
+                "steps": e2e_steps, "schedule": "pipelined: upload, kernels, download on 3 streams, "
+                                                "2 device buffer sets"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }
