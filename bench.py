@@ -53,6 +53,17 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# ---------------------------------------------------------------- config
+def prefill_config(cfg, T, world):
+    """The workload description both arms print."""
+    return {"workload": cfg.name, "batch": len(wl.seqlens_of(cfg)), "seq_len": T,
+            "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
+            "cmp_block": cfg.cmp_block, "sel_block": cfg.sel_block, "top_n": cfg.top_n,
+            "window": cfg.window, "out": "bf16",
+            "l2": "flushed (256 MB write) before every timed step",
+            "parallelism": f"replicas x{world} (independent sequences)"}
+
+
 # ---------------------------------------------------------------- ranks
 def max_over_ranks(x, world, device):
     """The largest of every rank's `x` (device time of the slowest replica);
@@ -335,11 +346,7 @@ def run_ours(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, U(0,1) gates, N(0,1/(l*D)) compressor)",
-        "config": {"workload": cfg.name, "batch": 1, "seq_len": T, "q_heads": Hq, "kv_heads": Hkv,
-                   "head_dim": D, "cmp_block": cfg.cmp_block, "sel_block": cfg.sel_block,
-                   "top_n": cfg.top_n, "window": cfg.window, "out": "bf16",
-                   "l2": "flushed (256 MB write) before every timed step",
-                   "parallelism": f"replicas x{world} (independent sequences)"},
+        "config": prefill_config(cfg, T, world),
         "sparse_tflops": round(flops["total"] / (ms_per_step / 1e3) / 1e12, 2),
         "algorithmic_flop_per_step": flops,
         "stage_ms": dict(zip(KERNEL_NAMES, [round(x, 4) for x in stage_ms])),
@@ -464,7 +471,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * wall / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "seq_len": int(inputs["cu_seqlens"][-1])},
+            "config": prefill_config(cfg, int(inputs["cu_seqlens"][-1]), args.gpus),
             "cpu_baseline": cb,
             "e2e": {"value": round(v, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
