@@ -38,7 +38,7 @@ def _rank(rank, world, port, out):
 
 def test_max_over_ranks_two_gloo_ranks():
     world = 2
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_rank, args=(world, _free_port(), out), nprocs=world, join=True)
         got = dict(out)
