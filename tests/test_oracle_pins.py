@@ -307,3 +307,41 @@ def test_workload_generator_is_seeded_and_bf16():
     # bf16 rounding of the generator is round-to-nearest-even
     x = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -3.0], np.float32)
     assert list(wl.bf16_bits(x)) == [0x3F80, 0x3F82, 0xC040]
+
+
+def test_worked_example_by_hand():
+    """Four tokens, worked out by hand from the definition (zero queries make
+    every softmax uniform; mean-pooling weights make the compressed values
+    block means; all numbers are exact dyadic fractions).
+
+    D = 2, one head, l = d = l' = 2, n = 1, w = 1; v = (1,0), (0,1), (2,2), (4,0);
+    gates (g_cmp, g_slc, g_win) = (1/2, 1/4, 1/4) for every token.
+      compressed: Vc0 = (1/2, 1/2), Vc1 = (3, 1); token t sees blocks i with
+        2i + 1 <= t, so O_cmp = 0, Vc0, Vc0, (Vc0 + Vc1)/2 = (7/4, 3/4);
+      scores: t = 1, 2: S0 = 1 (block 1 is incomplete at t = 2, score 0);
+        t = 3: S0 = S1 = 1/2, an exact tie that the lower index wins;
+      selected: block 0 for every t, keys u <= t in it: O_slc = v0, then
+        (v0 + v1)/2 = (1/2, 1/2) for t = 1, 2, 3;
+      window of one: O_win = v_t;
+      out = O_cmp/2 + O_slc/4 + O_win/4 =
+        (1/2, 0), (3/8, 5/8), (7/8, 7/8), (2, 1/2)."""
+    D, l = 2, 2
+    p = OracleParams(D, 1, 1, l, l, l, 1, 1)
+    q = wl.bf16_bits(np.zeros((4, 1, D), dtype=np.float32))
+    k = wl.bf16_bits(np.array([[[1, 2]], [[3, -1]], [[0, 5]], [[-2, 2]]], dtype=np.float32))
+    v = wl.bf16_bits(np.array([[[1, 0]], [[0, 1]], [[2, 2]], [[4, 0]]], dtype=np.float32))
+    gates = np.tile(np.array([0.5, 0.25, 0.25], dtype=np.float32), (4, 1, 1))
+    w = np.zeros((1, D, l * D), dtype=np.float32)
+    for c in range(D):
+        for pos in range(l):
+            w[0, c, pos * D + c] = 1.0 / l
+    _, kc = oracle.compress(p, k, w)
+    _, vc = oracle.compress(p, v, w)
+    assert np.array_equal(bf16_to_f64(vc)[:, 0], [[0.5, 0.5], [3.0, 1.0]])
+    r = oracle.nsa_rows(p, q, k, v, kc, vc, gates, np.arange(4, dtype=np.int32), cmax=2)
+    assert np.array_equal(r["o_cmp"][:, 0], [[0, 0], [0.5, 0.5], [0.5, 0.5], [1.75, 0.75]])
+    assert np.array_equal(r["scores"][1:, 0, :], [[1, 0], [1, 0], [0.5, 0.5]])
+    assert np.array_equal(r["sel"][:, 0, 0], [0, 0, 0, 0])
+    assert np.array_equal(r["o_slc"][:, 0], [[1, 0], [0.5, 0.5], [0.5, 0.5], [0.5, 0.5]])
+    assert np.array_equal(r["o_win"][:, 0], [[1, 0], [0, 1], [2, 2], [4, 0]])
+    assert np.array_equal(r["out"][:, 0], [[0.5, 0], [0.375, 0.625], [0.875, 0.875], [2.0, 0.5]])
