@@ -116,6 +116,45 @@ def test_prefill_rejects_bad_arguments_before_launch(L):
     assert L.nsa_plan_create(None, ctypes.byref(ctypes.c_void_p())) == nsa.NSA_ERR_INVALID_ARG
 
 
+def test_decode_rejects_bad_arguments_before_launch(L):
+    p = nsa.Plan(**_params(max_batch=4, max_seqlen=65536 + 64))
+    fake = 1 << 20  # an aligned address that is never dereferenced
+    args = dict(q=fake, k=fake, v=fake, kc=fake, vc=fake, lens=fake, batch=2, cap=4096,
+                gates=fake, w_k=fake, w_v=fake, out=fake, sel=None, ws=fake, wsb=256)
+
+    def call(**over):
+        a = dict(args)
+        a.update(over)
+        return L.nsa_decode(p.handle, a["q"], a["k"], a["v"], a["kc"], a["vc"], a["lens"],
+                            a["batch"], a["cap"], a["gates"], a["w_k"], a["w_v"], a["out"],
+                            a["sel"], a["ws"], a["wsb"], None)
+
+    assert call(batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(batch=5) == nsa.NSA_ERR_INVALID_ARG
+    assert call(cap=4000) == nsa.NSA_ERR_INVALID_ARG            # not a multiple of l
+    assert call(cap=65536 + 128) == nsa.NSA_ERR_INVALID_ARG     # above the plan's max_seqlen
+    assert call(ws=None) == nsa.NSA_ERR_WORKSPACE
+    assert call(wsb=255) == nsa.NSA_ERR_WORKSPACE
+    assert call(q=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(k=fake + 2) == nsa.NSA_ERR_MISALIGNED
+    assert call(lens=fake + 2) == nsa.NSA_ERR_MISALIGNED
+    wide = nsa.Plan(**_params(max_seqlen=70 * 1024 + 64, window=2048))
+    assert L.nsa_decode(wide.handle, fake, fake, fake, fake, fake, fake, 1, 4096, fake, fake,
+                        fake, fake, None, fake, 256, None) == nsa.NSA_ERR_UNSUPPORTED  # w > 1024
+    assert L.nsa_last_launch_count() == 0
+
+
+def test_noalloc_rejects_plans_beyond_its_static_array(L):
+    big = nsa.Plan(**_params())  # 64k tokens: several GB of workspace
+    assert big.workspace_size() > 32 << 20
+    fake = 1 << 20
+    rc = L.nsa_prefill_noalloc(big.handle, fake, fake, fake, fake, fake, fake, fake, 1, 65536,
+                               fake, fake, fake, None, None)
+    assert rc == nsa.NSA_ERR_WORKSPACE
+    assert L.nsa_prefill_noalloc(None, fake, fake, fake, fake, fake, fake, fake, 1, 1, fake,
+                                 fake, fake, None, None) == nsa.NSA_ERR_INVALID_ARG
+
+
 def test_strerror_covers_every_code(L):
     for code in range(8):
         assert nsa.strerror(code) not in ("unknown status", "")
