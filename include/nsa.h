@@ -27,7 +27,9 @@
  *      with the gate values given per token and head (post-sigmoid).
  * An empty branch contributes 0.  This version supports l == d == l'
  * (compress block == stride == select block) in {32, 64}, head_dim in
- * {64, 128}, G in {1, 2, 4, 8, 16}, 1 <= top_n <= 64, window >= 1.
+ * {64, 128}, G in {1, 2, 4, 8, 16}, 1 <= top_n <= 1024 / l (16 blocks of 64
+ * or 32 of 32 tokens: a token's selected keys fit in 8 chunks of 128),
+ * window >= 1; other valid geometries return NSA_ERR_UNSUPPORTED.
  *
  * Memory: every pointer except the plan is caller-owned device memory (bf16
  * is passed as raw 16-bit storage).  The library never allocates device
