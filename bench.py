@@ -82,6 +82,18 @@ def job_rate(units_per_rank, world, ms):
 
 
 # ---------------------------------------------------------------- algorithmic work
+def algorithmic_flops_packed(cfg, lens, sel):
+    """algorithmic_flops summed over the sequences of a packed batch."""
+    tot = {"cmp": 0, "slc": 0, "win": 0, "compress": 0, "total": 0}
+    s = 0
+    for T in lens:
+        f = algorithmic_flops(cfg, T, sel[s:s + T])
+        for k in tot:
+            tot[k] += f[k]
+        s += T
+    return tot
+
+
 def algorithmic_flops(cfg, T, sel):
     """Exact FLOPs of the method on one sequence (the work it does, not the
     dense work it avoids): per (t, head) 4 D (|cmp(t)| + |slc(t)| + |win(t)|),
@@ -363,9 +375,98 @@ def run_ours(args, rank, world):
         del d, host
         torch.cuda.empty_cache()
         result["decode"] = run_decode_leg(args, dev, world)
+    if not args.no_legs:
+        torch.cuda.empty_cache()
+        result["legs"] = {name: run_prefill_leg(name, dev, world)
+                          for name in ("prefill_8k", "varlen") if name != args.workload}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(cfg, inputs)
+        result["cpu_baseline_1core"] = oracle_single_core()
     return result
+
+
+# ---------------------------------------------------------------- other prefill workloads
+def run_prefill_leg(name, dev, world, steps=10, warmup=3):
+    """Device-timed prefill of another configuration (8k, varlen): tokens/s,
+    sparse TFLOP/s and the tensor roofline of every tensor-core kernel."""
+    import torch
+    from sparse_attention_long_06_b200 import nsa
+    cfg = wl.CONFIGS[name]
+    inputs = wl.prefill_inputs(cfg)
+    lens = list(inputs["seqlens"])
+    T = int(inputs["cu_seqlens"][-1])
+    D, Hq, Hkv = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads
+    d = {}
+    for k in ("q", "k", "v", "gates", "w_k", "w_v", "cu_seqlens"):
+        a = np.ascontiguousarray(inputs[k])
+        d[k] = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+    plan = nsa.Plan.for_config(cfg, max_batch=len(lens), max_seqlen=max(lens), max_total_tokens=T,
+                               out_dtype=nsa.OUT_BF16)
+    out = torch.empty((T, Hq, D), dtype=torch.int16, device=dev)
+    kc = torch.empty((max(plan.cmp_rows(T), 1), Hkv, D), dtype=torch.int16, device=dev)
+    vc = torch.empty_like(kc)
+    sel = torch.empty((T, Hkv, cfg.top_n), dtype=torch.int32, device=dev)
+    ws = plan.alloc_workspace(device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        plan.prefill(d["q"], d["k"], d["v"], d["gates"], d["w_k"], d["w_v"], d["cu_seqlens"],
+                     out, kc, vc, ws, sel_idx=sel)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if nsa.read_device_status(ws) != nsa.NSA_OK:
+        raise RuntimeError(f"{name}: device status after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ev), world, dev)
+    nsa.profile_enable(True)
+    stage = []
+    for _ in range(3):
+        flush.zero_()
+        step()
+        stage.append(nsa.profile_stage_ms())
+    nsa.profile_enable(False)
+    stage_ms = [statistics.median(x[i] for x in stage) for i in range(len(stage[0]))]
+    flops = algorithmic_flops_packed(cfg, lens, sel.cpu().numpy())
+    _, _, tc_sust, src = _peaks()
+    roof = {}
+    for kname, (idx, _, key) in TENSOR_KERNELS.items():
+        ach = flops[key] / (stage_ms[idx] / 1e3) / 1e12
+        roof[kname] = {"achieved": round(ach, 2), "frac": round(ach / tc_sust, 4)}
+    tflops = flops["total"] / (ms / 1e3) / 1e12
+    return {"metric": "NSA prefill tokens/s", "value": round(job_rate(T, world, ms), 1),
+            "unit": "tokens/s", "ms_per_step_median": round(ms, 4), "steps": steps,
+            "sparse_tflops": round(tflops, 2), "frac_of_peak": round(tflops / tc_sust, 4),
+            "peak": tc_sust, "peak_source": f"{src} bf16 sustained",
+            "config": prefill_config(cfg, T, world) | {"seqlens": lens},
+            "algorithmic_flop_per_step": flops,
+            "stage_ms": dict(zip(KERNEL_NAMES, [round(x, 4) for x in stage_ms])),
+            "rooflines": roof}
+
+
+def oracle_single_core(names=("tiny", "prefill_8k"), nrows=64):
+    """The oracle's tokens/s on one host core for small configurations, in a
+    child process with OMP_NUM_THREADS=1 (bounded: `nrows` sampled rows)."""
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    out = {}
+    for name in names:
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--oracle-sample", name,
+                            "--oracle-rows", str(nrows)], env=env, capture_output=True, text=True,
+                           timeout=600)
+        if r.returncode != 0:
+            out[name] = {"error": r.stderr.strip().splitlines()[-1:]}
+            continue
+        out[name] = json.loads(r.stdout.strip().splitlines()[-1])
+    return out
 
 
 # ---------------------------------------------------------------- decode leg
@@ -490,7 +591,16 @@ def main():
                     help="run only the decode leg and print its object (profiling)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="sequences in the decode leg (default: the workload's 32)")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the 8k / varlen prefill lines")
+    ap.add_argument("--oracle-sample", default="",
+                    help=argparse.SUPPRESS)  # child process of oracle_single_core
+    ap.add_argument("--oracle-rows", type=int, default=64, help=argparse.SUPPRESS)
     args = ap.parse_args()
+    if args.oracle_sample:
+        cfg = wl.CONFIGS[args.oracle_sample]
+        print(json.dumps(oracle_sample(cfg, wl.prefill_inputs(cfg), nrows=args.oracle_rows)))
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -93,6 +93,8 @@ typedef struct nsa_plan_s* nsa_plan_t;
  * A plan is immutable; it may be shared by calls on several streams as long
  * as each concurrent call has its own workspace. */
 int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out);
+/* The same call under its short name. */
+int nsa_plan(const nsa_params* params, nsa_plan_t* plan_out);
 void nsa_plan_destroy(nsa_plan_t plan);
 
 /* Bytes of device workspace a call of `mode` needs under the plan's bounds
@@ -152,11 +154,23 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,
  * make that first call before any stream capture.  All calls share the array
  * and it keeps the last call's contents (the status word is cleared by every
  * call); calls that overlap on the GPU race on it and must not be issued.
+ * The cached address belongs to the device's current context: after a
+ * cudaDeviceReset (or any reset of the primary context) this entry point
+ * must not be used again in the same process.  Device-side faults of a call
+ * land in the array's status word: read them with
+ * nsa_noalloc_read_device_status.
  */
 int nsa_prefill_noalloc(nsa_plan_t plan, const void* q, const void* k, const void* v,
                         const float* gates, const float* w_k, const float* w_v,
                         const int* cu_seqlens, int batch, int total_tokens, void* out,
                         void* k_cmp, void* v_cmp, int* sel_idx, void* stream);
+
+/* nsa_read_device_status for the static array of nsa_prefill_noalloc:
+ * synchronises `stream`, returns the status word of the last no-allocation
+ * call on the current device (NSA_OK or NSA_ERR_DEVICE_*) and clears it.
+ * Allocates nothing.  Returns NSA_ERR_CUDA if the stream failed or the
+ * array's address cannot be found. */
+int nsa_noalloc_read_device_status(void* stream);
 
 /*
  * One decode step for a batch of sequences (steps 1-7 for the newest token of

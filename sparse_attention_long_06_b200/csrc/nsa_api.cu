@@ -235,6 +235,10 @@ int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out) {
   return NSA_OK;
 }
 
+int nsa_plan(const nsa_params* params, nsa_plan_t* plan_out) {
+  return nsa_plan_create(params, plan_out);
+}
+
 void nsa_plan_destroy(nsa_plan_t plan) { delete plan; }
 
 size_t nsa_workspace_size(nsa_plan_t plan, int mode) {

@@ -21,6 +21,10 @@
 // launch sequence clears the one field that must start at zero (the status
 // word) itself.  Calls that overlap on the GPU (on different streams, or
 // from different host threads) race on the array and must not be issued.
+// The cached address is tied to the device's primary context: after a
+// device reset it is stale and the entry point must not be used again.
+// Device-side faults land in the array's status word (offset 0), which
+// nsa_noalloc_read_device_status reads and clears.
 #include <cstdio>
 #include <mutex>
 
@@ -76,4 +80,11 @@ extern "C" int nsa_prefill_noalloc(nsa_plan_t plan, const void* q, const void* k
   if (rc != NSA_OK) return rc;
   return nsa_prefill(plan, q, k, v, gates, w_k, w_v, cu_seqlens, batch, total_tokens, out, k_cmp,
                      v_cmp, sel_idx, ws, kStaticWorkspaceBytes, stream);
+}
+
+extern "C" int nsa_noalloc_read_device_status(void* stream) {
+  void* ws = nullptr;
+  const int rc = static_workspace(&ws);
+  if (rc != NSA_OK) return NSA_ERR_CUDA;
+  return nsa_read_device_status(ws, stream);
 }

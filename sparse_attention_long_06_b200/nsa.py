@@ -29,7 +29,8 @@ WS_STATUS, WS_O_CMP, WS_LSE, WS_SCORES, WS_SEL, WS_WIN = 0, 1, 2, 3, 4, 5
 EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_workspace_region",
             "nsa_cmp_rows", "nsa_prefill", "nsa_decode", "nsa_read_device_status",
             "nsa_selftest_timeout", "nsa_strerror", "nsa_last_launch_count",
-            "nsa_profile_enable", "nsa_profile_stage_ms", "nsa_prefill_noalloc"]
+            "nsa_profile_enable", "nsa_profile_stage_ms", "nsa_prefill_noalloc",
+            "nsa_plan", "nsa_noalloc_read_device_status"]
 
 
 class NsaError(RuntimeError):
@@ -64,6 +65,8 @@ def lib():
             vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
             L.nsa_plan_create.argtypes = [ctypes.POINTER(Params), ctypes.POINTER(vp)]
             L.nsa_plan_create.restype = i
+            L.nsa_plan.argtypes = [ctypes.POINTER(Params), ctypes.POINTER(vp)]
+            L.nsa_plan.restype = i
             L.nsa_plan_destroy.argtypes = [vp]
             L.nsa_plan_destroy.restype = None
             L.nsa_workspace_size.argtypes = [vp, i]
@@ -80,6 +83,8 @@ def lib():
             L.nsa_decode.restype = i
             L.nsa_read_device_status.argtypes = [vp, vp]
             L.nsa_read_device_status.restype = i
+            L.nsa_noalloc_read_device_status.argtypes = [vp]
+            L.nsa_noalloc_read_device_status.restype = i
             L.nsa_selftest_timeout.argtypes = [vp, sz, ctypes.c_longlong, vp]
             L.nsa_selftest_timeout.restype = i
             L.nsa_strerror.argtypes = [i]
@@ -126,7 +131,7 @@ class Plan:
                              sel_block, top_n, window, float(softmax_scale), max_batch,
                              max_seqlen, max_total_tokens, out_dtype)
         h = ctypes.c_void_p()
-        _check(lib().nsa_plan_create(ctypes.byref(self.params), ctypes.byref(h)), "nsa_plan_create")
+        _check(lib().nsa_plan(ctypes.byref(self.params), ctypes.byref(h)), "nsa_plan")
         self.handle = h
 
     @classmethod
@@ -200,6 +205,12 @@ class Plan:
 
 def read_device_status(workspace, stream=None) -> int:
     return int(lib().nsa_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+def noalloc_read_device_status(stream=None) -> int:
+    """Status word of the last nsa_prefill_noalloc call on the current device
+    (synchronises the stream, then clears the word)."""
+    return int(lib().nsa_noalloc_read_device_status(_stream(stream)))
 
 
 def selftest_timeout(workspace, cycles: int, stream=None):

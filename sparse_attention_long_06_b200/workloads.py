@@ -105,16 +105,21 @@ def compressor_weights(cfg: NsaConfig):
     return wk, wv
 
 
-def _plant(cfg: NsaConfig, b: int, T: int, q32: np.ndarray, k32: np.ndarray) -> None:
-    """Planted shared direction for the peaked-score varlen workload (in place)."""
+def _plant(cfg: NsaConfig, b: int, T: int, q32: np.ndarray, k32: np.ndarray,
+           blocks=None) -> None:
+    """Planted shared direction for the peaked-score varlen workload (in place):
+    queries biased toward a per-sequence unit direction u, and the keys of
+    `blocks` (default: a seeded 5 % of the key blocks) rotated to cosine 0.8
+    with u, norm preserved."""
     D = cfg.head_dim
     rng = _rng(cfg.seed, "plant", b)
     u = rng.standard_normal(D).astype(np.float64)
     u /= np.linalg.norm(u)
     q32[...] = ((q32.astype(np.float64) + math.sqrt(D) * u) / math.sqrt(2.0)).astype(np.float32)
     nblk = T // cfg.sel_block
-    nplant = max(1, int(round(0.05 * nblk)))
-    blocks = rng.choice(nblk, size=nplant, replace=False)
+    if blocks is None:
+        nplant = max(1, int(round(0.05 * nblk)))
+        blocks = rng.choice(nblk, size=nplant, replace=False)
     for j in blocks:
         kb = k32[j * cfg.sel_block:(j + 1) * cfg.sel_block].astype(np.float64)  # [l', Hkv, D]
         along = kb @ u                                                            # [l', Hkv]
@@ -147,6 +152,59 @@ def prefill_inputs(cfg: NsaConfig, seqlens: list[int] | None = None) -> dict:
     wk, wv = compressor_weights(cfg)
     out = {key: np.concatenate([p[key] for p in parts], axis=0) for key in ("q", "k", "v", "gates")}
     out.update(w_k=wk, w_v=wv, cu_seqlens=cu, seqlens=lens)
+    return out
+
+
+def lane_planted_prefill_inputs(cfg: NsaConfig, residues=(0, 1, 2), modulus: int = 32) -> dict:
+    """prefill_inputs with the planted direction of the varlen recipe on the
+    key blocks j with j % modulus in `residues` (every such block of every
+    sequence): the strongest blocks of a query all share a few residues, the
+    tie-heavy case for warp-level selections that deal blocks to lanes by
+    j % 32."""
+    lens = seqlens_of(cfg)
+    parts = []
+    for b, T in enumerate(lens):
+        D, Hq, Hkv = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads
+        q32 = _rng(cfg.seed, "q", b).standard_normal((T, Hq, D), dtype=np.float32)
+        k32 = _rng(cfg.seed, "k", b).standard_normal((T, Hkv, D), dtype=np.float32)
+        v32 = _rng(cfg.seed, "v", b).standard_normal((T, Hkv, D), dtype=np.float32)
+        nblk = T // cfg.sel_block
+        _plant(cfg, b, T, q32, k32, blocks=[j for j in range(nblk) if j % modulus in residues])
+        gates = _rng(cfg.seed, "gates", b).random((T, Hq, 3), dtype=np.float32)
+        parts.append({"q": bf16_bits(q32), "k": bf16_bits(k32), "v": bf16_bits(v32), "gates": gates})
+    cu = np.zeros(len(lens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lens)
+    wk, wv = compressor_weights(cfg)
+    out = {key: np.concatenate([p[key] for p in parts], axis=0) for key in ("q", "k", "v", "gates")}
+    out.update(w_k=wk, w_v=wv, cu_seqlens=cu, seqlens=lens)
+    return out
+
+
+def mean_pool_weights(cfg: NsaConfig):
+    """W_K = W_V = [I/l, ..., I/l] per KV head ([Hkv, D, l*D] fp32): the
+    compressor that averages a block's keys, so that a block of keys aligned
+    with a direction gives a compressed key aligned with it too."""
+    D, l, H = cfg.head_dim, cfg.cmp_block, cfg.num_kv_heads
+    w = np.zeros((H, D, l * D), dtype=np.float32)
+    for p in range(l):
+        w[:, np.arange(D), p * D + np.arange(D)] = np.float32(1.0 / l)
+    return w, w.copy()
+
+
+def make_keys_periodic(cfg: NsaConfig, inputs: dict, period_blocks: int) -> dict:
+    """Copies of prefill inputs whose keys repeat every `period_blocks` key
+    blocks inside each sequence (K[t] = K[t mod (period_blocks * l)]), so that
+    equal blocks give bit-identical compressed keys and exactly equal block
+    scores: the exact-tie case of the selection."""
+    out = dict(inputs)
+    k = inputs["k"].copy()
+    cu = inputs["cu_seqlens"]
+    span = period_blocks * cfg.cmp_block
+    for b in range(len(cu) - 1):
+        s, e = int(cu[b]), int(cu[b + 1])
+        idx = s + (np.arange(e - s) % span)
+        k[s:e] = inputs["k"][idx]
+    out["k"] = k
     return out
 
 

@@ -2,6 +2,9 @@
 seeded inputs and compare it with the fp64 oracle."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 
 import oracle
@@ -191,3 +194,38 @@ def check_prefill(cfg, inputs, res, rows_per_seq, check_e2e=True):
                                          float(np.abs(res["out"][tg][agree] - r2["out"][agree]).max()))
     rep["rel_l2"] = (rep["rel_l2_num"] / rep["rel_l2_den"]) ** 0.5 if rep["rel_l2_den"] else 0.0
     return rep
+
+
+def log_report(name: str, rep: dict) -> None:
+    """Prints a parity report and, when NSA_PARITY_LOG names a file, appends
+    it there as one JSON line (so that the observed counts of a GPU run are
+    kept beside its pass/fail status)."""
+    rec = {"test": name}
+    rec.update({k: (float(v) if isinstance(v, (float, np.floating)) else v)
+                for k, v in rep.items() if isinstance(v, (int, float, np.integer, np.floating))})
+    print(json.dumps(rec))
+    path = os.environ.get("NSA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
+def topn_path(score_row: np.ndarray, ncmp: int, ncand: int, n: int, cand_cap: int = 64) -> str:
+    """Which branch of the prefill top-n kernel a row takes, from its fp32
+    scores: "all" (at most n candidates), "regs" (the register selection) or
+    "radix" (the radix-select fallback: more than 1024 candidates, or more
+    than `cand_cap` keys at or above the n-th largest per-lane maximum of the
+    64-bit (score bits, inverted index) keys dealt to lanes by j % 32)."""
+    if ncand <= n:
+        return "all"
+    if ncand > 1024 or n > 32:
+        return "radix"
+    j = np.arange(1024, dtype=np.uint64)
+    b = np.zeros(1024, dtype=np.uint64)
+    b[:ncmp] = np.ascontiguousarray(score_row[:ncmp], dtype=np.float32).view(np.uint32)
+    key = (b << np.uint64(32)) | (np.uint64(0xFFFFFFFF) - j)
+    key[ncand:] = 0
+    lmax = key.reshape(32, 32).max(axis=0)      # lane = j % 32
+    t0 = np.sort(lmax)[::-1][n - 1]
+    count = int(np.count_nonzero((key >= t0) & (key != 0)))
+    return "radix" if count > cand_cap else "regs"

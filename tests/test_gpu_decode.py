@@ -102,6 +102,28 @@ def test_decode_64k_config_sampled_sequences():
                           wl.bf16_bits(res16["out"].astype(np.float32)))
 
 
+@pytest.mark.parametrize("period", [1, 3])
+def test_decode_exact_score_ties_go_to_the_lower_block(period):
+    """Compressed caches that repeat every `period` blocks give exactly equal
+    block scores: the decode selection must equal the oracle's on every
+    sequence, with no gap exemption (ties broken toward the lower index)."""
+    cfg = wl.NsaConfig("dec_ties", 33, 128, 64, 4, 64, 64, 64, 16, 512, decode_batch=4)
+    lens = [700, 4000, 5000, 9000]  # none completes a block: the cache is used as given
+    inp = wl.decode_inputs(cfg, lengths=lens, capacity=9024)
+    for name in ("kc", "vc"):
+        c = inp[name]
+        c[:] = c[:, np.arange(c.shape[1]) % period]
+    res = run_decode(cfg, inp)
+    assert res["status"] == nsa.NSA_OK
+    p = OracleParams.of(cfg)
+    for b, L in enumerate(lens):
+        r = oracle.decode_reference(p, inp, b, kc=res["kc"][b], vc=res["vc"][b])
+        assert np.array_equal(r["sel"], res["sel"][b]), b
+        if period == 1:
+            assert np.array_equal(res["sel"][b], np.tile(np.arange(16), (4, 1)))
+    check(cfg, inp, res, range(len(lens)))
+
+
 def test_decode_rejects_lengths_beyond_capacity():
     cfg = wl.NsaConfig("dec", 32, 64, 4, 1, 32, 32, 32, 4, 128, decode_batch=2)
     inp = wl.decode_inputs(cfg, lengths=[100, 200], capacity=256)

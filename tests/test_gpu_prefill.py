@@ -37,8 +37,8 @@ def _lib():
     nsa.lib()
 
 
-def _assert_report(rep, res=None, e2e=True):
-    print(rep)
+def _assert_report(rep, res=None, e2e=True, name="prefill"):
+    gu.log_report(name, rep)
     assert rep["kc_bound_fail"] == 0
     assert rep["kc_total"] == 0 or rep["kc_diff"] / rep["kc_total"] < 0.01
     assert rep["idx_bad_stageB"] == 0
@@ -63,7 +63,7 @@ def test_tiny_config_all_rows():
     assert res["status"] == nsa.NSA_OK
     assert res["launches"] == 6
     rep = gu.check_prefill(cfg, inputs, res, [np.arange(1024, dtype=np.int32)])
-    _assert_report(rep, res)
+    _assert_report(rep, res, name="tiny")
 
 
 @pytest.mark.parametrize("case", [
@@ -84,7 +84,7 @@ def test_edge_geometries(case):
     assert res["status"] == nsa.NSA_OK
     rows = [np.arange(T, dtype=np.int32) for T in lens]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep)
+    _assert_report(rep, name=f"edge{case}")
 
 
 def test_prefill_8k_sampled_rows():
@@ -94,7 +94,7 @@ def test_prefill_8k_sampled_rows():
     assert res["status"] == nsa.NSA_OK
     rows = [gu.sample_rows(8192, 384, 7, 8, 64)]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep, res)
+    _assert_report(rep, res, name="prefill_8k")
 
 
 def test_varlen_planted_sampled_rows():
@@ -104,17 +104,79 @@ def test_varlen_planted_sampled_rows():
     assert res["status"] == nsa.NSA_OK
     rows = [gu.sample_rows(T, 40, 100 + b, 8, 64) for b, T in enumerate(inputs["seqlens"])]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep, res)
+    _assert_report(rep, res, name="varlen")
 
 
 def test_prefill_64k_sampled_rows():
+    """Every 16th row of the 64k sequence plus the rows at block and tile
+    edges and the last rows: 4096+ rows checked against the oracle."""
     cfg = wl.CONFIGS["prefill_64k"]
     inputs = wl.prefill_inputs(cfg)
     res = gu.run_prefill(cfg, inputs, both_dtypes=True)
     assert res["status"] == nsa.NSA_OK
-    rows = [gu.sample_rows(65536, 96, 11, 8, 64)]
+    T = 65536
+    edges = [t for b in (1, 2, 511, 512, 1023) for t in (b * 64 - 1, b * 64)]
+    edges += [7, 8, 9, 15, 16, T - 9, T - 8, T - 2, T - 1]
+    rows = np.unique(np.concatenate([np.arange(5, T, 16), edges])).astype(np.int32)
+    assert len(rows) >= 4096
+    rep = gu.check_prefill(cfg, inputs, res, [rows])
+    _assert_report(rep, res, name="prefill_64k")
+
+
+@pytest.mark.parametrize("case", [
+    # D, Hq, Hkv, l, n, w, lengths, period in blocks
+    (128, 64, 4, 64, 16, 512, [4096], 3),
+    (64, 4, 1, 32, 4, 128, [3000, 500], 1),
+])
+def test_exact_score_ties_go_to_the_lower_block(case):
+    """Keys repeating every `period` blocks give bit-identical compressed keys,
+    hence exactly equal block scores on both sides: the index sets must agree
+    with the oracle on every row (no gap exemption), i.e. every exact tie is
+    broken toward the lower block index, on the GPU as in the definition."""
+    D, Hq, Hkv, l, n, w, lens, period = case
+    cfg = _custom("ties", D, Hq, Hkv, l, n, w, lens, seed=23)
+    inputs = wl.make_keys_periodic(cfg, wl.prefill_inputs(cfg), period)
+    res = gu.run_prefill(cfg, inputs, out_dtype=nsa.OUT_F32)
+    assert res["status"] == nsa.NSA_OK
+    rows = [np.arange(T, dtype=np.int32) for T in lens]
     rep = gu.check_prefill(cfg, inputs, res, rows)
-    _assert_report(rep, res)
+    _assert_report(rep, name=f"ties{case}")
+    assert rep["idx_exempt"] == 0
+    if period == 1:
+        # every complete block ties: the lowest n complete blocks win
+        s = 0
+        for T in lens:
+            for t in range(T):
+                ncmp = (t + 1) // l
+                if ncmp >= n:
+                    assert np.array_equal(res["sel"][s + t], np.tile(np.arange(n), (Hkv, 1)))
+            s += T
+
+
+def test_topn_fallback_rows_are_exact():
+    """Rows the register top-n hands to the radix fallback: more than 1024
+    candidates (T = 40000, l = 32), and rows whose strongest blocks all sit on
+    three lanes (planted blocks j % 32 in {0, 1, 2}), so that more than 64
+    keys reach the per-lane bound; the mean-pooling compressor keeps the
+    planted blocks' compressed keys aligned with the queries.  Stage A (the
+    oracle's selection on the GPU's scores) must hold bit for bit on both
+    kinds."""
+    cfg = _custom("fallback", 64, 4, 1, 32, 4, 128, [40000], seed=29)
+    inputs = wl.lane_planted_prefill_inputs(cfg)
+    inputs["w_k"], inputs["w_v"] = wl.mean_pool_weights(cfg)
+    res = gu.run_prefill(cfg, inputs, out_dtype=nsa.OUT_F32)
+    assert res["status"] == nsa.NSA_OK
+    T = 40000
+    rows = np.unique(np.concatenate([np.arange(3, T, 97), [32767, 32768, 32799, T - 1]]))
+    rows = rows.astype(np.int32)
+    paths = [gu.topn_path(res["scores"][t, 0], (t + 1) // 32, t // 32 + 1, 4) for t in rows]
+    n_big = sum(1 for t in rows if t // 32 + 1 > 1024)
+    n_tie = sum(1 for t, p in zip(rows, paths) if p == "radix" and t // 32 + 1 <= 1024)
+    assert n_big >= 50 and n_tie >= 50, (n_big, n_tie)
+    rep = gu.check_prefill(cfg, inputs, res, [rows])
+    rep.update(rows_radix_many_candidates=n_big, rows_radix_tied_lanes=n_tie,
+               rows_register=sum(1 for p in paths if p == "regs"))
+    _assert_report(rep, name="topn_fallback")
 
 
 def test_empty_prefill_is_a_no_op():

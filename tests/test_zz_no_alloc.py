@@ -47,13 +47,40 @@ def test_noalloc_matches_workspace_entry_point_twice():
         out, kc, vc, sel = buffers()
         plan.prefill_noalloc(d["q"], d["k"], d["v"], d["gates"], d["w_k"], d["w_v"],
                              d["cu_seqlens"], out, kc, vc, sel_idx=sel)
-        torch.cuda.synchronize()
+        assert nsa.noalloc_read_device_status() == nsa.NSA_OK
         got = out.cpu().numpy().astype(np.float64)
         assert np.isfinite(got).all()
         assert np.max(np.abs(got - ref)) <= 1e-2
         assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 5e-3
         assert np.array_equal(sel.cpu().numpy(), ref_sel.cpu().numpy())
         assert np.array_equal(kc.cpu().numpy(), ref_kc.cpu().numpy())
+        assert np.array_equal(vc.cpu().numpy(), ref_vc.cpu().numpy())
+
+
+def test_noalloc_reports_device_side_input_errors():
+    """A sequence longer than the plan's max_seqlen is caught on the device;
+    the caller reads the fault from the static array's status word."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from sparse_attention_long_06_b200 import build
+    build.build()
+    cfg = wl.NsaConfig("bad", 21, 64, 4, 1, 32, 32, 32, 4, 128, seqlens=(100, 100))
+    inp = wl.prefill_inputs(cfg)
+    plan = nsa.Plan.for_config(cfg, max_batch=2, max_seqlen=128, max_total_tokens=200,
+                               out_dtype=nsa.OUT_F32)
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    d = {k: dev(inp[k]) for k in ("q", "k", "v", "gates", "w_k", "w_v")}
+    cu = torch.tensor([0, 150, 200], dtype=torch.int32, device="cuda")  # first length > 128
+    out = torch.zeros((200, 4, 64), device="cuda")
+    kc = torch.zeros((plan.cmp_rows(200), 1, 64), dtype=torch.int16, device="cuda")
+    vc = torch.zeros_like(kc)
+    plan.prefill_noalloc(d["q"], d["k"], d["v"], d["gates"], d["w_k"], d["w_v"], cu, out, kc, vc)
+    assert nsa.noalloc_read_device_status() == nsa.NSA_ERR_DEVICE_BAD_INPUT
+    assert nsa.noalloc_read_device_status() == nsa.NSA_OK  # cleared by the read
 
 
 def test_noalloc_rejects_plans_beyond_the_static_array():
