@@ -28,10 +28,13 @@
  *    separate maps for keys and values; the compressed tensor is stored in
  *    bf16 (round to nearest even), and steps 2-3 use that stored tensor;
  *  - a compressed block is visible to query t once its last token is <= t;
- *  - block score = sum over the query heads of the KV group of the compressed
- *    softmax probabilities (l == d == l'), the incomplete block holding t is a
- *    candidate with score 0; ties go to the lower block index; if there are at
- *    most n candidates, all are taken;
+ *  - block score of selection block j (tokens j*l' .. j*l' + l' - 1) = sum
+ *    over the query heads of the KV group of the compressed softmax
+ *    probabilities of every visible compressed block (tokens i*d .. i*d + l - 1)
+ *    that overlaps it; with l == d == l' that is the probability of block j
+ *    itself, and the incomplete block holding t (which no visible compressed
+ *    block overlaps) is a candidate with score 0; ties go to the lower block
+ *    index; if there are at most n candidates, all are taken;
  *  - window = the w tokens ending at t (t included);
  *  - scale 1/sqrt(D) by default for all three branches;
  *  - an empty branch contributes 0;
@@ -201,10 +204,11 @@ double oracle_select(const double* S, int ncand, int n, int* sel) {
  * Outputs (any may be NULL):
  *   o_cmp, o_slc, o_win, out  [Hq, D]
  *   lse    [Hq]               log-sum-exp of the compressed branch
- *   scores [Hkv, cmax]        block scores (entries >= C(t) left 0)
+ *   scores [Hkv, cmax]        selection-block scores (entries >= t / l' + 1 left 0)
  *   sel    [Hkv, n]           selected block indices (ascending, -1 pad)
  *   gap    [Hkv]              n-th minus (n+1)-th ranked score
- * Returns 0, or -1 on an unsupported geometry.
+ * Returns 0, or -1 on an invalid geometry (d > l, or a group size that does
+ * not divide the heads).
  */
 int oracle_nsa_query(const nsa_oracle_params* P, int t, const uint16_t* q, const uint16_t* k,
                      const uint16_t* v, const uint16_t* kc, const uint16_t* vc,
@@ -212,7 +216,7 @@ int oracle_nsa_query(const nsa_oracle_params* P, int t, const uint16_t* q, const
                      double* out, double* lse, double* scores, int cmax, int* sel,
                      double* gap) {
   const int D = P->D, Hq = P->Hq, Hkv = P->Hkv, G = Hq / Hkv;
-  if (P->l != P->d || P->lsel != P->l || Hq % Hkv != 0) return -1;
+  if (Hq % Hkv != 0 || P->d < 1 || P->l < P->d || P->lsel < 1) return -1;
   /* visible compressed blocks: i*d + l - 1 <= t */
   const int ncmp = (t + 1 >= P->l) ? (t + 1 - P->l) / P->d + 1 : 0;
   /* selection candidates: blocks j with j*l' <= t */
@@ -240,10 +244,16 @@ int oracle_nsa_query(const nsa_oracle_params* P, int t, const uint16_t* q, const
       for (int c = 0; c < D; ++c) qh[c] = oracle_bf16_to_f64(q[(size_t)h * D + c]);
       double L = attend(P, qh, kc, vc, g, cmp_rows, ncmp, oc + (size_t)hh * D, prob, scratch);
       if (lse) lse[h] = L;
-      for (int i = 0; i < ncmp; ++i) S[i] += prob[i]; /* l == d == l' */
+      /* compressed block i covers tokens [i*d, i*d + l - 1]: its probability
+         goes to every selection block [j*l', j*l' + l' - 1] it overlaps (all
+         of them are candidates: i*d + l - 1 <= t) */
+      for (int i = 0; i < ncmp; ++i) {
+        const int j0 = (i * P->d) / P->lsel, j1 = (i * P->d + P->l - 1) / P->lsel;
+        for (int j = j0; j <= j1; ++j) S[j] += prob[i];
+      }
     }
     if (scores) {
-      for (int j = 0; j < cmax; ++j) scores[(size_t)g * cmax + j] = (j < ncmp) ? S[j] : 0.0;
+      for (int j = 0; j < cmax; ++j) scores[(size_t)g * cmax + j] = (j < ncand) ? S[j] : 0.0;
     }
     /* step 4 */
     double gp = oracle_select(S, ncand, P->n, chosen);

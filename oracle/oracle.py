@@ -221,7 +221,9 @@ def decode_reference(p: OracleParams, inputs: dict, b: int, kc=None, vc=None) ->
     kc = np.array(inputs["kc"][b] if kc is None else kc, copy=True)
     vc = np.array(inputs["vc"][b] if vc is None else vc, copy=True)
     C = num_cmp_blocks(p, L)
-    if C > 0 and L % p.cmp_stride == 0 and L >= p.cmp_block:
+    # the newest token completes compressed block C - 1 when its last token
+    # (C - 1) * d + l - 1 is the newest one
+    if C > 0 and (C - 1) * p.cmp_stride + p.cmp_block == L:
         blk = C - 1
         s = blk * p.cmp_stride
         _, kb = compress(p, k[s:s + p.cmp_block], inputs["w_k"])

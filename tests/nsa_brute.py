@@ -26,21 +26,31 @@ def masked_softmax(z, mask):
     return np.divide(e, s, out=np.zeros_like(e), where=s > 0)
 
 
-def nsa_dense(q, k, v, kc, vc, gates, D, Hq, Hkv, l, n, w, scale=None):
+def nsa_dense(q, k, v, kc, vc, gates, D, Hq, Hkv, l, n, w, scale=None, d=None, lsel=None):
     """q [T,Hq,D], k/v [T,Hkv,D], kc/vc [C,Hkv,D] (float64), gates [T,Hq,3].
-    Block geometry: l == d == l'.  Returns dict of [T,Hq,D] arrays plus
-    scores [T,Hkv,C] and sel (list of per-(t,g) index arrays)."""
+    Block geometry: compression block l, stride d (default l), selection
+    block lsel (default l).  Returns dict of [T,Hq,D] arrays plus scores
+    [T,Hkv,J] (selection-block scores, J = T // lsel + 1) and sel (per-(t,g)
+    index arrays)."""
+    d = l if d is None else d
+    lsel = l if lsel is None else lsel
     T = q.shape[0]
     C = kc.shape[0]
     G = Hq // Hkv
+    J = T // lsel + 1
     s = 1.0 / np.sqrt(D) if scale is None else scale
     tt = np.arange(T)[:, None]
     uu = np.arange(T)[None, :]
     ii = np.arange(C)[None, :]
-    cmp_mask = (ii * l + l - 1) <= tt                       # [T, C]
+    cmp_mask = (ii * d + l - 1) <= tt                       # [T, C]
     win_mask = (uu <= tt) & (uu > tt - w)                   # [T, T]
+    # overlap[i, j]: compressed block i (tokens [i d, i d + l)) meets
+    # selection block j (tokens [j lsel, (j + 1) lsel))
+    ci = np.arange(C)[:, None]
+    jj = np.arange(J)[None, :]
+    overlap = ((ci * d) < (jj + 1) * lsel) & ((ci * d + l) > jj * lsel)
     out = {key: np.zeros((T, Hq, D)) for key in ("o_cmp", "o_slc", "o_win", "out")}
-    scores = np.zeros((T, Hkv, C))
+    scores = np.zeros((T, Hkv, J))
     sel = {}
     for g in range(Hkv):
         P = []
@@ -50,17 +60,17 @@ def nsa_dense(q, k, v, kc, vc, gates, D, Hq, Hkv, l, n, w, scale=None):
             p = masked_softmax(z, cmp_mask)
             P.append(p)
             out["o_cmp"][:, h, :] = p @ vc[:, g, :]
-        S = np.sum(P, axis=0)                                 # [T, C]
+        S = np.sum(P, axis=0) @ overlap.astype(np.float64)   # [T, J]
         scores[:, g, :] = S
         slc_mask = np.zeros((T, T), dtype=bool)
         for t in range(T):
-            ncand = t // l + 1
-            cand = np.array([S[t, j] if j < C and (j * l + l - 1) <= t else 0.0 for j in range(ncand)])
+            ncand = t // lsel + 1
+            cand = S[t, :ncand]
             order = np.lexsort((np.arange(ncand), -cand))     # score desc, index asc
             chosen = np.sort(order[:n])
             sel[(t, g)] = chosen
             for j in chosen:
-                slc_mask[t, j * l:(j + 1) * l] = True
+                slc_mask[t, j * lsel:(j + 1) * lsel] = True
         slc_mask &= (uu <= tt)
         for hh in range(G):
             h = g * G + hh

@@ -42,7 +42,9 @@ def _run(p, q, k, v, gates, wk, wv, rows=None, kc=None, vc=None):
         kc = np.zeros((1, p.num_kv_heads, p.head_dim), np.uint16)
         vc = np.zeros((1, p.num_kv_heads, p.head_dim), np.uint16)
     rows = np.arange(T) if rows is None else rows
-    return oracle.nsa_rows(p, q, k, v, kc, vc, gates, rows, cmax=max(1, T // p.cmp_block)), kc, vc
+    # score columns: every selection block a query of this sequence may rank
+    cmax = max(1, T // p.sel_block + 1)
+    return oracle.nsa_rows(p, q, k, v, kc, vc, gates, rows, cmax=cmax), kc, vc
 
 
 def _dense_causal(q, k, v, D, G):
@@ -267,30 +269,115 @@ def test_oracle_matches_dense_mask_statement(T, Hq, Hkv, D, l, n, w):
     for key in ("o_cmp", "o_slc", "o_win", "out"):
         assert np.max(np.abs(r[key] - ref[key])) < 1e-12, key
     if C:
-        assert np.max(np.abs(r["scores"][:, :, :C] - ref["scores"])) < 1e-12
+        assert np.max(np.abs(r["scores"][:, :, :C] - ref["scores"][:, :, :C])) < 1e-12
     for t in range(T):
         for g in range(Hkv):
             got = [j for j in r["sel"][t, g] if j >= 0]
             assert got == list(ref["sel"][(t, g)]), (t, g)
 
 
-def test_decode_query_equals_last_prefill_row():
-    T, Hq, Hkv, D, l = 128, 4, 2, 8, 8
-    p = OracleParams(D, Hq, Hkv, l, l, l, 3, 16)
+@pytest.mark.parametrize("T,Hq,Hkv,D,l,d,lsel,n,w", [
+    (100, 4, 2, 8, 8, 4, 8, 3, 13),   # overlapping compression (d < l)
+    (100, 4, 1, 8, 8, 4, 16, 2, 9),   # overlapping, selection block 2 l
+    (97, 2, 1, 8, 4, 4, 8, 3, 5),     # l = d, selection block 2 l
+    (64, 4, 2, 8, 8, 8, 4, 4, 7),     # selection block shorter than a compressed block
+    (50, 2, 1, 8, 6, 3, 5, 2, 4),     # sizes that share no factor
+    (5, 2, 1, 8, 4, 2, 2, 1, 2),      # barely one compressed block
+])
+def test_oracle_matches_dense_mask_statement_general_geometry(T, Hq, Hkv, D, l, d, lsel, n, w):
+    """Compression stride d and selection block l' independent of l: each
+    compressed block adds its probability to every selection block it
+    overlaps.  The oracle's row walk must agree with the dense-mask statement,
+    whose overlap is a [C, J] boolean matrix."""
+    p = OracleParams(D, Hq, Hkv, l, d, lsel, n, w)
+    q, k, v, gates, wk, wv = _rand_inputs(300 + T + d + lsel, T, Hq, Hkv, D, l)
+    r, kc, vc = _run(p, q, k, v, gates, wk, wv)
+    C = oracle.num_cmp_blocks(p, T)
+    assert C == (0 if T < l else (T - l) // d + 1)
+    ref = nsa_dense(bf16_to_f64(q), bf16_to_f64(k), bf16_to_f64(v), bf16_to_f64(kc[:max(C, 0)]),
+                    bf16_to_f64(vc[:max(C, 0)]), gates.astype(np.float64), D, Hq, Hkv, l, n, w,
+                    d=d, lsel=lsel)
+    for key in ("o_cmp", "o_slc", "o_win", "out"):
+        assert np.max(np.abs(r[key] - ref[key])) < 1e-12, key
+    J = T // lsel + 1
+    assert np.max(np.abs(r["scores"][:, :, :J] - ref["scores"][:, :, :J])) < 1e-12
+    for t in range(T):
+        for g in range(Hkv):
+            got = [j for j in r["sel"][t, g] if j >= 0]
+            assert got == list(ref["sel"][(t, g)]), (t, g)
+
+
+def test_selection_block_score_sums_its_compressed_blocks():
+    """With d = l and l' = 2 l every compressed block lies in exactly one
+    selection block: the score of selection block J is the sum of the scores
+    of compressed blocks 2J and 2J + 1 under l' = l."""
+    T, Hq, Hkv, D, l = 120, 4, 2, 8, 4
+    q, k, v, gates, wk, wv = _rand_inputs(77, T, Hq, Hkv, D, l)
+    r1, _, _ = _run(OracleParams(D, Hq, Hkv, l, l, l, 3, 5), q, k, v, gates, wk, wv)
+    r2, _, _ = _run(OracleParams(D, Hq, Hkv, l, l, 2 * l, 3, 5), q, k, v, gates, wk, wv)
+    s1 = r1["scores"]
+    J = T // (2 * l) + 1
+    for j in range(J):
+        want = s1[:, :, 2 * j] + (s1[:, :, 2 * j + 1] if 2 * j + 1 < s1.shape[2] else 0.0)
+        assert np.max(np.abs(r2["scores"][:, :, j] - want)) < 1e-13, j
+    # the compressed branch does not depend on the selection block
+    assert np.array_equal(r1["o_cmp"], r2["o_cmp"]) and np.array_equal(r1["lse"], r2["lse"])
+
+
+def test_overlapping_compression_worked_example():
+    """Eight tokens, one head, D = 2, l = 4, d = 2, l' = 4, n = 1, w = 1, zero
+    queries (uniform softmaxes) and mean pooling, worked out by hand:
+      compressed block i covers tokens 2i .. 2i + 3 and is visible once
+      2i + 3 <= t;  v = (1,0) (0,1) (2,2) (4,0) (0,0) (2,0) (0,4) (8,8), so
+      Vc0 = (7/4, 3/4), Vc1 = (2, 1/2), Vc2 = (5/2, 3);
+      t = 5: blocks 0, 1 visible, p = 1/2 each; block 0 meets selection block
+        0, block 1 (tokens 2..5) meets selection blocks 0 and 1: S = (1, 1/2);
+        O_cmp = (15/8, 5/8);
+      t = 7: blocks 0, 1, 2, p = 1/3: S = (2/3, 2/3), an exact tie the lower
+        block wins; O_cmp = (25/12, 17/12); O_slc = mean of v0..v3 = (7/4, 3/4);
+        O_win = v7."""
+    D, l, d, lsel = 2, 4, 2, 4
+    p = OracleParams(D, 1, 1, l, d, lsel, 1, 1)
+    q = wl.bf16_bits(np.zeros((8, 1, D), dtype=np.float32))
+    k = wl.bf16_bits(np.arange(16, dtype=np.float32).reshape(8, 1, D))
+    v = wl.bf16_bits(np.array([[[1, 0]], [[0, 1]], [[2, 2]], [[4, 0]], [[0, 0]], [[2, 0]],
+                               [[0, 4]], [[8, 8]]], dtype=np.float32))
+    gates = np.tile(np.array([1.0, 0.0, 0.0], dtype=np.float32), (8, 1, 1))
+    w = np.zeros((1, D, l * D), dtype=np.float32)
+    for c in range(D):
+        for pos in range(l):
+            w[0, c, pos * D + c] = 1.0 / l
+    _, kc = oracle.compress(p, k, w)
+    _, vc = oracle.compress(p, v, w)
+    assert np.array_equal(bf16_to_f64(vc)[:, 0], [[1.75, 0.75], [2.0, 0.5], [2.5, 3.0]])
+    r = oracle.nsa_rows(p, q, k, v, kc, vc, gates, np.array([5, 7], dtype=np.int32), cmax=2)
+    assert np.allclose(r["scores"][:, 0, :], [[1.0, 0.5], [2 / 3, 2 / 3]], rtol=0, atol=1e-15)
+    assert np.array_equal(r["sel"][:, 0, 0], [0, 0])
+    assert np.allclose(r["o_cmp"][:, 0], [[15 / 8, 5 / 8], [25 / 12, 17 / 12]], rtol=0, atol=1e-15)
+    assert np.allclose(r["o_slc"][1, 0], [1.75, 0.75], rtol=0, atol=1e-15)
+    assert np.array_equal(r["o_win"][1, 0], [8.0, 8.0])
+    assert r["gap"][1, 0] == 0.0
+
+
+@pytest.mark.parametrize("l,d,lsel", [(8, 8, 8), (8, 4, 16)])
+def test_decode_query_equals_last_prefill_row(l, d, lsel):
+    T, Hq, Hkv, D = 128, 4, 2, 8
+    p = OracleParams(D, Hq, Hkv, l, d, lsel, 3, 16)
     q, k, v, gates, wk, wv = _rand_inputs(15, T, Hq, Hkv, D, l)
     r, kc, vc = _run(p, q, k, v, gates, wk, wv)
-    for L in (T, T - 3):  # L % l == 0 exercises the block completed by the new token
+    for L in (T, T - 3):  # L = T completes the last compressed block with the new token
         inputs = {"q": q[L - 1][None], "k": k[None, :L], "v": v[None, :L],
                   "kc": kc[None], "vc": vc[None], "gates": gates[L - 1][None],
                   "seqlens": np.array([L]), "w_k": wk, "w_v": wv}
-        if L % l == 0:
+        C = oracle.num_cmp_blocks(p, L)
+        if (C - 1) * d + l == L:
             inputs["kc"] = inputs["kc"].copy()
-            inputs["kc"][0, L // l - 1] = 0  # must be recomputed from the cache
+            inputs["kc"][0, C - 1] = 0  # must be recomputed from the cache
             inputs["vc"] = inputs["vc"].copy()
-            inputs["vc"][0, L // l - 1] = 0
-        d = oracle.decode_reference(p, inputs, 0)
-        assert np.array_equal(d["out"], r["out"][L - 1])
-        assert np.array_equal(d["sel"], r["sel"][L - 1])
+            inputs["vc"][0, C - 1] = 0
+        dr = oracle.decode_reference(p, inputs, 0)
+        assert np.array_equal(dr["out"], r["out"][L - 1])
+        assert np.array_equal(dr["sel"], r["sel"][L - 1])
 
 
 def test_workload_generator_is_seeded_and_bf16():
