@@ -58,7 +58,8 @@ def prefill_config(cfg, T, world):
     """The workload description both arms print."""
     return {"workload": cfg.name, "batch": len(wl.seqlens_of(cfg)), "seq_len": T,
             "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
-            "cmp_block": cfg.cmp_block, "sel_block": cfg.sel_block, "top_n": cfg.top_n,
+            "cmp_block": cfg.cmp_block, "cmp_stride": cfg.cmp_stride, "sel_block": cfg.sel_block,
+            "top_n": cfg.top_n,
             "window": cfg.window, "out": "bf16",
             "l2": "flushed (256 MB write) before every timed step",
             "parallelism": f"replicas x{world} (independent sequences)"}
@@ -98,18 +99,20 @@ def algorithmic_flops(cfg, T, sel):
     """Exact FLOPs of the method on one sequence (the work it does, not the
     dense work it avoids): per (t, head) 4 D (|cmp(t)| + |slc(t)| + |win(t)|),
     plus compression 4 l D^2 per complete block per KV head."""
-    D, G, l, w = cfg.head_dim, cfg.group, cfg.cmp_block, cfg.window
+    D, G, l, d, ls, w = (cfg.head_dim, cfg.group, cfg.cmp_block, cfg.cmp_stride, cfg.sel_block,
+                         cfg.window)
     t = np.arange(T, dtype=np.int64)
-    ncmp = (t + 1) // l
+    ncmp = np.where(t + 1 >= l, (t + 1 - l) // d + 1, 0)  # complete compressed blocks
     nwin = np.minimum(w, t + 1)
     blk = sel.astype(np.int64)                            # [T, Hkv, n]
-    keys = np.where(blk >= 0, np.minimum(l, t[:, None, None] - blk * l + 1), 0)
+    keys = np.where(blk >= 0, np.minimum(ls, t[:, None, None] - blk * ls + 1), 0)
     nslc = keys.clip(min=0).sum(axis=2)                   # [T, Hkv]
     per_head = 4 * D
     f_cmp = per_head * G * cfg.num_kv_heads * int(ncmp.sum())
     f_win = per_head * G * cfg.num_kv_heads * int(nwin.sum())
     f_slc = per_head * G * int(nslc.sum())
-    f_compress = 4 * (T // l) * cfg.num_kv_heads * l * D * D
+    n_blocks = (T - l) // d + 1 if T >= l else 0
+    f_compress = 4 * n_blocks * cfg.num_kv_heads * l * D * D
     return {"cmp": f_cmp, "slc": f_slc, "win": f_win, "compress": f_compress,
             "total": f_cmp + f_slc + f_win + f_compress}
 
@@ -185,12 +188,12 @@ def oracle_sample(cfg, inputs, nrows=512):
     rows = np.linspace(T - 1, 0, num=nrows).astype(np.int32)[::-1].copy()
     t0 = time.perf_counter()
     oracle.nsa_rows(p, inputs["q"], inputs["k"], inputs["v"], kc, vc, inputs["gates"], rows,
-                    cmax=max(1, T // cfg.cmp_block))
+                    cmax=max(1, T // cfg.cmp_block, T // cfg.sel_block + 1))
     t_rows = time.perf_counter() - t0
     sec_per_token = t_rows / nrows + t_cmp / T
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": 1.0 / sec_per_token, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"fp64 oracle on the {cfg.name} input: compression of all {T // cfg.cmp_block} "
+            "sample": (f"fp64 oracle on the {cfg.name} input: compression of all {oracle.num_cmp_blocks(p, T)} "
                        f"blocks ({t_cmp:.2f} s, amortised over {T} tokens) + {nrows} evenly spaced "
                        f"query rows ({t_rows:.2f} s)")}
 
@@ -378,7 +381,8 @@ def run_ours(args, rank, world):
     if not args.no_legs:
         torch.cuda.empty_cache()
         result["legs"] = {name: run_prefill_leg(name, dev, world)
-                          for name in ("prefill_8k", "varlen") if name != args.workload}
+                          for name in ("prefill_8k", "varlen", "prefill_8k_overlap")
+                          if name != args.workload}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(cfg, inputs)
         result["cpu_baseline_1core"] = oracle_single_core()
@@ -475,17 +479,19 @@ def decode_bytes(cfg, lens, sel):
     the compressed keys and values of the complete blocks, the selected blocks'
     keys and values and the window's (their union counted once), plus q,
     gates and out."""
-    D, Hq, Hkv, l, w = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads, cfg.cmp_block, cfg.window
+    D, Hq, Hkv, w = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads, cfg.window
+    l, d, ls = cfg.cmp_block, cfg.cmp_stride, cfg.sel_block
     total = 0
     for b, L in enumerate(lens):
         t = L - 1
+        C = (L - l) // d + 1 if L >= l else 0
         win = set(range(max(0, t - w + 1), t + 1))
         for g in range(Hkv):
             keys = set(win)
             for blk in sel[b, g]:
                 if blk >= 0:
-                    keys.update(range(blk * l, min(blk * l + l, t + 1)))
-            total += (L // l) * D * 2 * 2 + len(keys) * D * 2 * 2
+                    keys.update(range(blk * ls, min(blk * ls + ls, t + 1)))
+            total += C * D * 2 * 2 + len(keys) * D * 2 * 2
         total += Hq * D * 2 + Hq * 3 * 4 + Hq * D * 2
     return total
 
@@ -537,16 +543,20 @@ def run_decode_leg(args, dev, world=1):
     nbytes = decode_bytes(cfg, [int(x) for x in d["seqlens"].cpu()], sel.cpu().numpy())
     hbm, _, _, src = _peaks()
     gbs = nbytes / (med / 1e3) / 1e9
-    kgbs = nbytes / (stage[1] / 1e3) / 1e9
+    kern_ms = stage[1] + stage[2]  # the two decode kernels (after the block compression)
+    kgbs = nbytes / (kern_ms / 1e3) / 1e9
     return {"metric": "NSA decode tokens/s", "value": round(job_rate(B, world, med), 1), "unit": "tokens/s",
             "ms_per_step_median": round(med, 5), "steps": steps,
             "config": {"workload": cfg.name, "batch": B, "context": int(cfg.decode_len),
                        "q_heads": cfg.num_q_heads, "kv_heads": cfg.num_kv_heads, "head_dim": cfg.head_dim,
-                       "l": cfg.cmp_block, "top_n": cfg.top_n, "window": cfg.window,
+                       "l": cfg.cmp_block, "d": cfg.cmp_stride, "l_sel": cfg.sel_block,
+                       "top_n": cfg.top_n, "window": cfg.window,
                        "l2": "flushed before every timed step"},
             "stage_ms": {"nsa_decode_compress_kernel": round(stage[0], 5),
-                         "nsa_decode_kernel": round(stage[1], 5)},
-            "roofline": {"bound": "hbm", "kernel": "nsa_decode_kernel", "achieved": round(kgbs, 1),
+                         "nsa_decode_a_kernel": round(stage[1], 5),
+                         "nsa_decode_b_kernel": round(stage[2], 5)},
+            "roofline": {"bound": "hbm", "kernel": "nsa_decode_a_kernel + nsa_decode_b_kernel",
+                         "achieved": round(kgbs, 1),
                          "peak": hbm, "unit": "GB/s", "frac": round(kgbs / hbm, 4),
                          "algorithmic_bytes": int(nbytes), "step_gbs": round(gbs, 1),
                          "peak_source": f"{src} copy bandwidth"}}
@@ -584,7 +594,8 @@ def main():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill_64k", choices=["prefill_64k", "prefill_8k", "varlen"])
+    ap.add_argument("--workload", default="prefill_64k",
+                    choices=["prefill_64k", "prefill_8k", "varlen", "prefill_8k_overlap"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true",

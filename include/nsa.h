@@ -7,17 +7,22 @@
  *   1. compression ("DeepSeek NSA config.toml" page, section 3,
  *      compress_block_size; "DeepSeek NSA in manufacturing" page, section on
  *      what dynamic sparsity sparsifies: one learned linear map over each
- *      flattened key block):
- *        Kc[i,g,:] = W_K[g] . vec(K[i*l .. i*l+l-1, g, :]),  Vc likewise,
+ *      flattened key block), blocks of l tokens at a stride of d:
+ *        Kc[i,g,:] = W_K[g] . vec(K[i*d .. i*d+l-1, g, :]),  Vc likewise,
  *      vec index p*D + c (token p of the block, channel c), stored in bf16;
  *   2. compressed branch (config page, section 1): softmax over the complete
- *      blocks i (i*l + l - 1 <= t) of s * q_h . Kc[i,g]; O_cmp = sum p Vc;
+ *      blocks i (i*d + l - 1 <= t) of s * q_h . Kc[i,g]; O_cmp = sum p Vc;
  *   3. block scores (manufacturing page, same section: coarse attention of
- *      the query to every compressed block ranks the blocks):
- *        S[t,g,j] = sum over the G heads of group g of p_h[j];
+ *      the query to every compressed block ranks the blocks): selection
+ *      block j covers tokens [j*l', j*l' + l' - 1] and
+ *        S[t,g,j] = sum over the G heads of group g of the probabilities
+ *                   p_h[i] of every complete compressed block i that
+ *                   overlaps it
+ *      (with l == d == l' that is the sum over heads of p_h[j]);
  *   4. selection (config page, section 3, select_top_k): the top_n blocks
- *      among j*l <= t by (score descending, index ascending); the block
- *      holding t, while incomplete, competes with score 0;
+ *      among j*l' <= t by (score descending, index ascending); the block
+ *      holding t competes with whatever score step 3 gives it (0 when no
+ *      complete compressed block overlaps it);
  *   5. selected branch (config page, section 3, select_block_size): softmax
  *      attention over the tokens u <= t of the chosen blocks;
  *   6. window branch (config page, section 3, sliding_window): softmax
@@ -25,11 +30,11 @@
  *   7. gate (config page, sections 1 and 3, gate_type learned):
  *        out = g_cmp * O_cmp + g_slc * O_slc + g_win * O_win,
  *      with the gate values given per token and head (post-sigmoid).
- * An empty branch contributes 0.  This version supports l == d == l'
- * (compress block == stride == select block) in {32, 64}, head_dim in
- * {64, 128}, G in {1, 2, 4, 8, 16}, 1 <= top_n <= 1024 / l (16 blocks of 64
- * or 32 of 32 tokens: a token's selected keys fit in 8 chunks of 128),
- * window >= 1; other valid geometries return NSA_ERR_UNSUPPORTED.
+ * An empty branch contributes 0.  This version supports compression blocks
+ * l in {32, 64} with a stride d in {16, 32, 64} that divides l, selection
+ * blocks l' in {32, 64}, head_dim in {64, 128}, G in {1, 2, 4, 8, 16},
+ * 1 <= top_n <= min(32, 1024 / l') (a token's selected keys fit in 8 chunks
+ * of 128), window >= 1; other valid geometries return NSA_ERR_UNSUPPORTED.
  *
  * Memory: every pointer except the plan is caller-owned device memory (bf16
  * is passed as raw 16-bit storage).  The library never allocates device
@@ -74,8 +79,8 @@ typedef struct {
   int num_q_heads;       /* Hq */
   int num_kv_heads;      /* Hkv; Hq / Hkv must be 1, 2, 4, 8 or 16 */
   int cmp_block;         /* l  (compress_block_size) */
-  int cmp_stride;        /* d  (compression stride; must equal l here) */
-  int sel_block;         /* l' (select_block_size; must equal l here) */
+  int cmp_stride;        /* d  (compression stride: 16, 32 or 64, dividing l) */
+  int sel_block;         /* l' (select_block_size: 32 or 64) */
   int top_n;             /* n  (select_top_k) */
   int window;            /* w  (sliding_window) */
   float softmax_scale;   /* s; 0 selects 1/sqrt(D) */
@@ -107,15 +112,21 @@ typedef enum {
   NSA_WS_STATUS = 0,  /* int32 status word */
   NSA_WS_O_CMP = 1,   /* fp32 [T_total, Hq, D] compressed-branch output */
   NSA_WS_LSE = 2,     /* fp32 [T_total, Hq] compressed-branch log-sum-exp (natural log) */
-  NSA_WS_SCORES = 3,  /* fp32 [T_total, Hkv, max_seqlen / l] block scores; entry j
-                         of row t is defined for j < number of complete blocks */
+  NSA_WS_SCORES = 3,  /* fp32 [T_total, Hkv, (max_seqlen - l) / d + 1] compressed-block
+                         scores (sum over the group's heads of the compressed softmax
+                         probabilities); entry i of row t is defined for i < the
+                         number of complete compressed blocks */
   NSA_WS_SEL = 4,     /* int32 [T_total, Hkv, top_n] selection (when sel_idx is NULL) */
-  NSA_WS_WIN = 5      /* fp32 [T_total, Hq, D] window-branch output times its gate */
+  NSA_WS_WIN = 5,     /* fp32 [T_total, Hq, D] window-branch output times its gate */
+  NSA_WS_SEL_SCORES = 6 /* fp32 [T_total, Hkv, max_seqlen / l' + 1] selection-block scores
+                           (entry j of row t defined for j <= t / l'); empty (0 bytes)
+                           when l == d == l', where NSA_WS_SCORES already holds them */
 } nsa_ws_region;
 int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, size_t* bytes);
 
 /* Rows of the packed compressed-KV output of a prefill over `total_tokens`
- * tokens: floor(total_tokens / l), an upper bound on sum_b floor(T_b / l). */
+ * tokens: floor(total_tokens / d), an upper bound on the sum over the
+ * sequences of their complete compressed blocks, (T_b - l) / d + 1. */
 int nsa_cmp_rows(nsa_plan_t plan, int total_tokens);
 
 /*
@@ -128,7 +139,8 @@ int nsa_cmp_rows(nsa_plan_t plan, int total_tokens);
  *                                cu_seqlens[batch] = total_tokens, each length <= max_seqlen
  *   out        [T_total, Hq, D]  bf16 or fp32 (plan out_dtype)
  *   k_cmp, v_cmp [nsa_cmp_rows, Hkv, D] bf16, written: the compressed keys and
- *              values of sequence b occupy rows sum_{b'<b} floor(T_b'/l) onward
+ *              values of sequence b occupy rows sum_{b'<b} C(T_b') onward,
+ *              C(T) = (T - l) / d + 1 complete blocks (0 when T < l)
  *   sel_idx    [T_total, Hkv, top_n] int32 or NULL: selected block indices of
  *              each token, ascending, -1 padded
  *   workspace  >= nsa_workspace_size(plan, NSA_MODE_PREFILL) bytes, 256-byte aligned
@@ -177,21 +189,29 @@ int nsa_noalloc_read_device_status(void* stream);
  * each sequence, which the caller has already written into the caches).
  *   q           [batch, Hq, D]             bf16, query of the newest token
  *   k_cache, v_cache [batch, cache_capacity, Hkv, D] bf16
- *   k_cmp_cache, v_cmp_cache [batch, cache_capacity / l, Hkv, D] bf16: the
+ *   k_cmp_cache, v_cmp_cache [batch, cache_capacity / d, Hkv, D] bf16: the
  *               compressed blocks of every complete block before the newest
- *               token; when the newest token completes a block (len % l == 0)
- *               that block is compressed here from the cache and written back
+ *               token; when the newest token completes a block (len >= l and
+ *               (len - l) % d == 0) that block, number (len - l) / d, is
+ *               compressed here from the cache and written back
  *   seqlens     [batch] int32 device, tokens in the cache including the newest,
- *               1 <= len <= cache_capacity and len < 1025 * l (all of a query's
- *               compressed scores are kept on chip); cache rows at or past
- *               len are never read
- *   cache_capacity  multiple of l, <= plan max_seqlen and <= 1025 * l; the
+ *               1 <= len <= cache_capacity; cache rows at or past len are never
+ *               read
+ *   cache_capacity  multiple of l and of l', <= plan max_seqlen, holding at
+ *               most 4096 compressed blocks (all of a query's compressed
+ *               scores are kept on chip: 262144 tokens at l = d = 64); the
  *               window must be at most 1024 tokens
  *   gates       [batch, Hq, 3] fp32
  *   w_k, w_v    [Hkv, D, l*D] fp32
  *   out         [batch, Hq, D] bf16 or fp32
  *   sel_idx     [batch, Hkv, top_n] int32 or NULL
- *   workspace   >= nsa_workspace_size(plan, NSA_MODE_DECODE) bytes
+ *   workspace   >= nsa_workspace_size(plan, NSA_MODE_DECODE) bytes (per
+ *               (sequence, KV group): the selection, the compressed branch's
+ *               probabilities and the fp32 partial results the last kernel
+ *               merges; about 6 MB for 32 sequences of 64k tokens)
+ * Three launches: the compression of a block the newest token completed,
+ * then two kernels that split every (sequence, group) into units of about
+ * 128-256 KB of cache reads; the last unit of each pair merges the branches.
  */
 int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* v_cache,
                void* k_cmp_cache, void* v_cmp_cache, const int* seqlens, int batch,

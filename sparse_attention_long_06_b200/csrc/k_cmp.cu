@@ -5,7 +5,11 @@
 //   compressed blocks of s * q . Kc, output O_cmp = sum p Vc;
 //   step 3 ("DeepSeek NSA in manufacturing" page, section on what dynamic
 //   sparsity sparsifies: the query's coarse attention to every compressed
-//   block ranks the blocks): S[t, g, j] = sum over the heads of group g of p.
+//   block ranks the blocks): S[t, g, i] = sum over the heads of group g of p
+//   for compressed block i (the top-n kernel sums these over each selection
+//   block when the block sizes and stride differ).
+// Compressed block i covers tokens [i d, i d + l - 1] and is visible to the
+// queries t >= i d + l - 1.
 //
 // One persistent CTA per SM walks dense tiles of 128 MMA rows = (128 / G)
 // consecutive tokens x the G query heads of one KV group.  The compressed
@@ -67,7 +71,8 @@ __device__ __forceinline__ CmpItem cmp_item(const PrefillArgs& a, int k) {
   it.T = __ldg(a.cu + it.b + 1) - c0;
   it.row0 = c0 + it.t0;
   const int tend = min(it.t0 + a.geo.tpt, it.T);
-  const int ncmp_max = tend / a.geo.l;  // (t + 1) / l at t = tend - 1
+  // compressed blocks visible to the tile's last token (t = tend - 1)
+  const int ncmp_max = num_cmp_blocks(tend, a.geo.l, a.geo.d);
   it.nc = (ncmp_max + kChunk - 1) / kChunk;
   it.cmp0 = a.cmp_off[it.b];
   return it;
@@ -197,7 +202,7 @@ __global__ void __launch_bounds__(kCmpThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(sm);
   int* status = a.status;
-  const int G = a.geo.G, l = a.geo.l;
+  const int G = a.geo.G, l = a.geo.l, dstride = a.geo.d;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(kCmpThreads, 1)
       const int i_row = r >> lgG, h_row = r & (G - 1);
       const int t_row = it.t0 + i_row;
       const bool row_ok = t_row < it.T;
-      const int ncmp_row = row_ok ? (t_row + 1) / l : 0;
+      const int ncmp_row = row_ok ? num_cmp_blocks(t_row + 1, l, dstride) : 0;
       const size_t orow = ((size_t)(it.row0 + i_row) * Hq + it.g * G + h_row);
       if (it.nc == 0) {
         if (row_ok && !*abort_flag) {
@@ -439,8 +444,8 @@ __global__ void __launch_bounds__(kCmpThreads, 1)
         if (p_use > 0) mbar_wait(p_empty + w, (p_use - 1) & 1, abort_flag, status, kWaitCycles);
         const int key = c * kChunk + r;
         // rows (token, head) that see compressed block `key`: tokens t with
-        // (t + 1) / l > key, inside the sequence
-        const int tok_lo = max(0, (key + 1) * l - 1 - it.t0);
+        // key * d + l - 1 <= t, inside the sequence
+        const int tok_lo = max(0, key * dstride + l - 1 - it.t0);
         const int tok_hi = min(a.geo.tpt, it.T - it.t0);
         const int row_lo = tok_lo * G, row_hi = tok_hi * G;
         const uint32_t prow = sbase + L::kP + w * L::kPBytes + (r >> 3) * 1024 + (r & 7) * 128;

@@ -3,27 +3,34 @@
 // config page separates prefill from decode in its benchmarking advice,
 // section 5).
 //
-// nsa_decode_compress_kernel: when the newest token completes a block
-// (len % l == 0), that block is compressed from the cache (step 1) and
-// written into the compressed cache; all other blocks were compressed before.
-//
-// nsa_decode_kernel: one CTA per (sequence, KV group), the group's G heads
-// sharing every load.  All products are swap-AB tcgen05 MMAs with 128 keys on
-// the TMEM lanes and the heads on 16 columns (S^T = K Q^T, O^T += V^T P^T):
-//   compressed all complete blocks (chunks end at the last one), two-sweep
-//             softmax, O_cmp, and a third sweep for the block scores
-//             S_j = sum over heads of the normalised probabilities;
-//   top-n     one warp selects n blocks from the scores in shared memory
-//             (the window's keys and values stream in meanwhile);
-//   window    the w tokens ending at t (chunks end at t, so no cache row past
-//             the sequence is read), two-sweep softmax, O_win;
-//   selected  the chosen blocks (the incomplete block is loaded as the l rows
-//             ending at t), two-sweep softmax, O_slc;
-//   epilogue  out = g_cmp O_cmp + g_slc O_slc + g_win O_win, lane = channel.
-// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2..5 = softmax / top-n /
-// epilogue.  Memory per (sequence, group) at the 64k shape: 512 KB of
-// compressed KV, 512 KB of selected blocks and 256 KB of window, streamed
-// through a 4-stage ring of 32 KB chunks.
+// A decode step reads every compressed block, the window and the selected
+// blocks of each (sequence, KV group) once: an HBM-bound stream of about
+// 1.3 MB per pair at the 64k shape.  It is cut into units of similar size so
+// that every SM streams, with no unit waiting for another:
+//   nsa_decode_compress_kernel  when the newest token completes a
+//              compressed block (len >= l, (len - l) % d == 0), that block
+//              is compressed from the cache (step 1) into the compressed
+//              cache;
+//   nsa_decode_a_kernel  two units per pair:
+//     scores   all compressed keys: S^T = Kc Q^T (keys on TMEM lanes, the
+//              group's heads on 16 columns), per-head log-sum-exp, the
+//              normalised probabilities P^T (bf16, to the workspace), the
+//              block scores (step 3: the sum over heads of p, summed over
+//              the compressed blocks overlapping each selection block when
+//              l, d and l' differ) and the top-n (step 4, one warp, to the
+//              workspace and sel_idx);
+//     window   the w tokens ending at t (step 6): O_win, normalised;
+//   nsa_decode_b_kernel  units of at most two 128-key chunks per pair:
+//     cmp      O_cmp partial sums P Vc over a range of compressed blocks
+//              (step 2, with the probabilities of the scores unit);
+//     selected a range of the selected blocks (step 5; the incomplete
+//              block holding t is loaded as the l' rows ending at t): a
+//              softmax partial (row max, sum, unnormalised O);
+//   the last unit of a pair to finish (an atomic counter per pair) merges
+//   the partials and applies the gates (step 7):
+//     out = g_cmp O_cmp + g_slc O_slc + g_win O_win.
+// Both kernels: warp 0 = TMA producer, warp 1 = tcgen05.mma issuer,
+// warps 2..5 = softmax / epilogue (thread = key lane of a chunk, or channel).
 #include <cuda_bf16.h>
 
 #include "nsa_internal.cuh"
@@ -37,18 +44,19 @@ using namespace sm100;
 namespace {
 
 // ------------------------------------------------------------------ step 1 for decode
-// Kc[blk, h, c] = sum_k W[h, c, k] * X[b, blk*l + k / D, h, k % D] for the
-// block the newest token completed.  One warp per 16 output channels; lanes
-// split the l*D inputs (coalesced rows of W) and reduce with shuffles.
+// Kc[blk, h, c] = sum_k W[h, c, k] * X[b, blk*d + k / D, h, k % D] for the
+// block the newest token completed.  One warp per output channel at a time;
+// lanes split the l*D inputs (coalesced rows of W) and reduce with shuffles.
 __global__ void __launch_bounds__(256) nsa_decode_compress_kernel(DecodeArgs a) {
   const int b = blockIdx.x, h = blockIdx.y;
   const bool is_v = blockIdx.z != 0;
   const int L = __ldg(a.seqlens + b);
-  const int l = a.geo.l, D = a.geo.D, H = a.geo.Hkv;
-  if (L < l || L > a.cap || (L % l) != 0) return;
-  const int blk = L / l - 1;
+  const int l = a.geo.l, dstride = a.geo.d, D = a.geo.D, H = a.geo.Hkv;
+  if (L < l || L > a.cap || (L - l) % dstride != 0) return;
+  const int blk = (L - l) / dstride;
   extern __shared__ float xs[];  // l*D inputs of the block
-  const uint16_t* X = (is_v ? a.v_cache : a.k_cache) + ((size_t)b * a.cap + (size_t)blk * l) * H * D;
+  const uint16_t* X =
+      (is_v ? a.v_cache : a.k_cache) + ((size_t)b * a.cap + (size_t)blk * dstride) * H * D;
   const int K = l * D;
   for (int k = threadIdx.x; k < K; k += blockDim.x) {
     const int p = k / D, c = k - p * D;
@@ -59,9 +67,16 @@ __global__ void __launch_bounds__(256) nsa_decode_compress_kernel(DecodeArgs a) 
   uint16_t* out = (is_v ? a.v_cmp : a.k_cmp) + (((size_t)b * a.ccap + blk) * H + h) * D;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nwarps = blockDim.x / 32;
   for (int c = warp; c < D; c += nwarps) {
-    const float* wrow = W + (size_t)c * K;
+    const float4* wrow = reinterpret_cast<const float4*>(W + (size_t)c * K);
+    const float4* x4 = reinterpret_cast<const float4*>(xs);
     float acc = 0.f;
-    for (int k = lane; k < K; k += 32) acc = fmaf(__ldg(wrow + k), xs[k], acc);
+    for (int k = lane; k < K / 4; k += 32) {
+      const float4 wv = __ldg(wrow + k), xv = x4[k];
+      acc = fmaf(wv.x, xv.x, acc);
+      acc = fmaf(wv.y, xv.y, acc);
+      acc = fmaf(wv.z, xv.z, acc);
+      acc = fmaf(wv.w, xv.w, acc);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) {
@@ -71,113 +86,220 @@ __global__ void __launch_bounds__(256) nsa_decode_compress_kernel(DecodeArgs a) 
   }
 }
 
-// ------------------------------------------------------------------ fused decode
-template <int D>
-struct DecLayout {
-  static constexpr int kStages = 4;
-  static constexpr int kQBytes = 16 * D * 2;          // 16 head rows
-  static constexpr int kChunkBytes = kChunk * D * 2;  // 128 keys
-  static constexpr int kPBytes = 8 * 4096;            // 8 chunks of P^T (128 keys x 16 heads)
-  static constexpr int kQ = 0;
-  static constexpr int kRing = 4096;                  // Q needs at most 4 KB
-  static constexpr int kP = kRing + kStages * kChunkBytes;  // 2 buffers
-  static constexpr int kScores = kP + 2 * kPBytes;          // float[1024]
-  static constexpr int kRed = kScores + kDecodeMaxCmp * 4;  // float[2][64]
-  static constexpr int kSel = kRed + 2 * 64 * 4;            // int[64]
-  static constexpr int kHist = kSel + 64 * 4;               // unsigned[256]
-  static constexpr int kBars = kHist + 256 * 4;
-  static constexpr int kEnd = kBars + 32 * 8;
-  static constexpr int kSmem = kEnd + 1024;
-  static_assert(kSmem <= 232448, "shared memory budget");
+// ------------------------------------------------------------------ shared pieces
+constexpr int kDecThreads = 192;
+// at most 16 compressed-value units (32 chunks of 128 blocks) and 8 selected
+// units (16 chunks: top_n <= 32 blocks of 32 or 16 of 64) per pair
+constexpr int kMaxCmpUnits = 16;
+constexpr int kMaxSlcUnits = 8;
+constexpr int kPChunkBytes = 4096;  // P^T of one chunk: 128 keys x 16 heads, bf16
+
+// Per-(sequence, group) quantities of one decode query.
+struct DecPair {
+  int ok, b, g, L, t, C, ncc, nwc, nsc, ncand, cmp_row0, win_row0;
 };
 
-constexpr uint32_t kColSW = 0, kColSC = 128, kColSS = 256;
-constexpr uint32_t kColOW = 384, kColOC = 400, kColOS = 416;
-
-struct DecItem {
-  int ok, b, g, L, t, C, nwc, ncc, nsc, ncand;
-};
-
-__device__ __forceinline__ DecItem dec_item(const DecodeArgs& a) {
-  DecItem it{};
-  it.b = blockIdx.x / a.geo.Hkv;
-  it.g = blockIdx.x % a.geo.Hkv;
-  it.L = __ldg(a.seqlens + it.b);
-  it.ok = it.L >= 1 && it.L <= a.cap && it.L / a.geo.l <= kDecodeMaxCmp;
-  if (!it.ok) return it;
-  it.t = it.L - 1;
-  it.C = it.L / a.geo.l;
-  const int wn = min(a.geo.w, it.L);
-  it.nwc = (wn + kChunk - 1) / kChunk;
-  it.ncc = (it.C + kChunk - 1) / kChunk;
-  const int bpc = kChunk >> a.geo.lg_l;
-  it.nsc = (a.geo.n + bpc - 1) / bpc;
-  it.ncand = it.t / a.geo.l + 1;
-  return it;
+__device__ __forceinline__ DecPair dec_pair(const DecodeArgs& a, int pair) {
+  DecPair p{};
+  p.b = pair / a.geo.Hkv;
+  p.g = pair % a.geo.Hkv;
+  p.L = __ldg(a.seqlens + p.b);
+  p.ok = p.L >= 1 && p.L <= a.cap;
+  if (!p.ok) return p;
+  p.t = p.L - 1;
+  p.C = num_cmp_blocks(p.L, a.geo.l, a.geo.d);
+  p.ncc = (p.C + kChunk - 1) / kChunk;
+  const int wn = min(a.geo.w, p.L);
+  p.nwc = (wn + kChunk - 1) / kChunk;
+  const int bpc = kChunk >> a.geo.lg_ls;
+  p.nsc = (a.geo.n + bpc - 1) / bpc;
+  p.ncand = p.t / a.geo.ls + 1;
+  p.cmp_row0 = p.C - kChunk * p.ncc;      // compressed chunks end at the last block
+  p.win_row0 = p.t - kChunk * p.nwc + 1;  // window chunks end at t
+  return p;
 }
 
-// First cache row of the selected block `blk` as loaded (the incomplete block
-// holding t is loaded as the l rows ending at t).
+// First cache row of the selected block `blk` of l tokens as loaded (the
+// incomplete block holding t is loaded as the l rows ending at t).
 __device__ __forceinline__ int sel_row0(int blk, int l, int t) {
   return (blk * l + l - 1 > t) ? t - l + 1 : blk * l;
 }
 
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Sweep over `nchunks` S^T chunks of 16 columns starting at TMEM column
+// `col` (lane = key): op(c, v[16]) for each chunk, the loads of four chunks
+// in flight before one wait.
+template <int kMaxChunks, typename Op>
+__device__ __forceinline__ void sweep_chunks(uint32_t lane_addr, uint32_t col, int nchunks, Op op) {
+#pragma unroll
+  for (int c0 = 0; c0 < kMaxChunks; c0 += 4) {
+    if (c0 >= nchunks) break;
+    float v[64];
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      float u16[16];
+      tmem_ld16(lane_addr + col + (c0 + cc) * 16, u16);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[cc * 16 + j] = u16[j];
+    }
+    tmem_ld_wait();
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      if (c0 + cc >= nchunks) break;
+      float u16[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) u16[j] = v[cc * 16 + j];
+      op(c0 + cc, u16);
+    }
+  }
+}
+
+// Stores 16 bf16 head values of key r into a P^T chunk laid out as the B
+// operand of O^T += V^T P^T: [head half][key / 8][key % 8][8 heads].
+__device__ __forceinline__ void store_pt(uint8_t* chunk, int r, const float (&p)[16]) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
+  uint8_t* base = chunk + (r >> 3) * 128 + (r & 7) * 16;
+  *reinterpret_cast<uint4*>(base) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  *reinterpret_cast<uint4*>(base + 2048) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
-    nsa_decode_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
-  using L = DecLayout<D>;
-  constexpr int KSTEPS = D / 16;
+__device__ __forceinline__ void issue_qk(uint32_t tmem_col, uint32_t stage, uint32_t qs) {
+  constexpr uint32_t id_qk = idesc_bf16(128, 16, false, false);
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    const uint32_t qoff = (ks >> 2) * 2048 + (ks & 3) * 32;   // Q^T halves: 16 rows
+    const uint32_t soff = (ks >> 2) * 16384 + (ks & 3) * 32;  // chunk halves: 128 rows
+    mma_bf16_ss(tmem_col, smem_desc(stage + soff, 16, 1024, kLayoutSw128),
+                smem_desc(qs + qoff, 16, 1024, kLayoutSw128), id_qk, ks > 0);
+  }
+}
+
+// O^T (D x 16 at tmem_col) (+)= V^T P^T for one 128-key chunk.
+__device__ __forceinline__ void issue_pv(uint32_t tmem_col, uint32_t stage, uint32_t pchunk,
+                                         bool accumulate) {
+  constexpr uint32_t id_pv = idesc_bf16(128, 16, true, true);
+#pragma unroll
+  for (int ks = 0; ks < kChunk / 16; ++ks)
+    mma_bf16_ss(tmem_col, smem_desc(stage + ks * 2048, 16384, 1024, kLayoutSw128),
+                smem_desc(pchunk + ks * 256, 128, 2048, kLayoutNone), id_pv,
+                (accumulate || ks > 0) ? 1u : 0u);
+}
+
+// Workspace records of one pair (fp32): window output [G][D], compressed
+// partial sums [ncv][G][D], selected partials [nsl][G*D + 32] (O [G][D], then
+// the row maximum m[16] and the sum[16] per head; every record 16-byte
+// aligned).
+struct PairRecs {
+  float* win;
+  float* cmp;
+  float* slc;
+  uint8_t* pt;
+  int* sel;
+};
+
+__device__ __forceinline__ PairRecs pair_recs(const DecodeArgs& a, int pair) {
+  const int G = a.geo.G, D = a.geo.D;
+  PairRecs r;
+  r.win = a.ws_win + (size_t)pair * G * D;
+  r.cmp = a.ws_cmp + (size_t)pair * a.ncv_max * G * D;
+  r.slc = a.ws_slc + (size_t)pair * a.nsl * (G * D + 32);
+  r.pt = a.ws_pt + (size_t)pair * a.ncc_max * kPChunkBytes;
+  r.sel = a.ws_sel + (size_t)pair * a.geo.n;
+  return r;
+}
+
+// ------------------------------------------------------------------ kernel A
+// The PV products read a ring stage as a 128-channel operand (two 64-channel
+// halves 16 KB apart).  With D = 64 only the first half exists: the second
+// feeds output channels that are never read, and the pad after the ring keeps
+// that read of the last stage inside the CTA's shared memory.
+template <int D>
+constexpr int ring_pad() { return D == 64 ? 16384 : 0; }
+
+template <int D>
+struct DecALayout {
+  static constexpr int kStages = 2;
+  static constexpr int kChunkBytes = kChunk * D * 2;
+  static constexpr int kQ = 0;                                   // 16 x D bf16 (4 KB max)
+  static constexpr int kRing = 4096;
+  static constexpr int kU = kRing + kStages * kChunkBytes + ring_pad<D>();  // P^T (window) | scores
+  static constexpr int kUBytes = 8 * kPChunkBytes > kDecodeMaxCmp * 4 ? 8 * kPChunkBytes
+                                                                     : kDecodeMaxCmp * 4;
+  static constexpr int kRed = kU + kUBytes;                      // float [2][64]
+  static constexpr int kSel = kRed + 2 * 64 * 4;                 // int [64]
+  static constexpr int kHist = kSel + 64 * 4;                    // unsigned [256]
+  static constexpr int kCand = kHist + 256 * 4;                  // u64 [kTopnCand]
+  static constexpr int kBars = kCand + kTopnCand * 8;
+  static constexpr int kEnd = kBars + 16 * 8;
+  static constexpr int kSmem = kEnd + 1024;  // manual 1024-byte alignment
+  static_assert(kU % 1024 == 0, "alignment");
+  // a PV operand spans 32 KB from the start of its stage
+  static_assert(kRing + (kStages - 1) * kChunkBytes + 32768 <= kEnd, "PV operand inside smem");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
+    nsa_decode_a_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
+  using L = DecALayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* st_full = bars + 1;   // [4]
-  uint64_t* st_empty = bars + 5;  // [4]
-  uint64_t* sW_full = bars + 9;
-  uint64_t* sC_full = bars + 10;
-  uint64_t* sS_full = bars + 11;
-  uint64_t* pW_full = bars + 12;
-  uint64_t* pC_full = bars + 13;
-  uint64_t* pS_full = bars + 14;
-  uint64_t* pW_empty = bars + 15;
-  uint64_t* idx_ready = bars + 16;
-  uint64_t* o_done = bars + 17;
-  uint64_t* fin = bars + 18;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
-  float* scores = reinterpret_cast<float*>(sm + L::kScores);
+  uint64_t* st_full = bars + 1;   // [2]
+  uint64_t* st_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* o_done = bars + 7;
+  uint64_t* fin = bars + 8;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   float* red = reinterpret_cast<float*>(sm + L::kRed);
-  int* sel_s = reinterpret_cast<int*>(sm + L::kSel);
   unsigned* hist = reinterpret_cast<unsigned*>(sm + L::kHist);
+  unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + L::kCand);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const DecItem it = dec_item(a);
-  if (!it.ok) {
+  // kernel B may be scheduled now: its CTAs wait for this grid's results
+  // (griddepcontrol.wait) and only take the SM slots this grid leaves free
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int pair = blockIdx.x >> 1;
+  const bool is_win = blockIdx.x & 1;
+  const DecPair P = dec_pair(a, pair);
+  if (!P.ok) {
     if (threadIdx.x == 0) atomicCAS(a.status, 0, kDeviceBadInputCode);
     return;
   }
+  const int nchunks = is_win ? P.nwc : P.ncc;
+  const PairRecs rec = pair_recs(a, pair);
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < L::kStages; ++i) {
       mbar_init(st_full + i, 1);
       mbar_init(st_empty + i, 1);
     }
-    mbar_init(sW_full, 1);
-    mbar_init(sC_full, 1);
-    mbar_init(sS_full, 1);
-    mbar_init(pW_full, 4);
-    mbar_init(pC_full, 4);
-    mbar_init(pS_full, 4);
-    mbar_init(pW_empty, 1);
-    mbar_init(idx_ready, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
     mbar_init(o_done, 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // TMEM: scores unit S^T of up to 32 chunks; window unit S^T of up to 8
+  // chunks and O^T (16 columns at 128)
+  const uint32_t ncols = is_win ? 256u : (nchunks <= 8 ? 128u : (nchunks <= 16 ? 256u : 512u));
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -186,67 +308,35 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(sm);
   int* status = a.status;
-  const int G = a.geo.G, l = a.geo.l, n = a.geo.n, lg_l = a.geo.lg_l;
-  const int bpc = kChunk >> lg_l;
-  const int t = it.t, b = it.b, g = it.g;
-  const int win_row0 = t - kChunk * it.nwc + 1;  // first row of window chunk 0
-  const int cmp_row0 = it.C - kChunk * it.ncc;   // first row of compressed chunk 0
+  const int G = a.geo.G, n = a.geo.n;
+  const int b = P.b, g = P.g, t = P.t;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int sc = 0;
       bool ok = true;
-      auto acquire = [&]() -> uint8_t* {
-        const int s = sc % L::kStages, u = sc / L::kStages;
-        if (u > 0 && !mbar_wait(st_empty + s, (u - 1) & 1, abort_flag, status, kWaitCycles)) {
-          ok = false;
-          return nullptr;
-        }
-        mbar_arrive_expect_tx(st_full + s, L::kChunkBytes);
-        return sm + L::kRing + s * L::kChunkBytes;
-      };
-      // 128 rows of a [rows, Hkv, D] cache slab starting at row0 (rows < 0 read 0)
-      auto load_rows = [&](const CUtensorMap* map, int row0) {
-        uint8_t* dst = acquire();
-        if (!dst) return;
-        const int s = sc % L::kStages;
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) tma_load_4d(dst + h * 16384, map, st_full + s, h * 64, g, row0, b);
-        ++sc;
-      };
-      auto load_sel = [&](bool is_v) {
-        for (int c = 0; c < it.nsc && ok; ++c) {
-          uint8_t* dst = acquire();
-          if (!dst) return;
-          const int s = sc % L::kStages;
-          for (int sub = 0; sub < bpc; ++sub) {
-            const int bs = c * bpc + sub;
-            const int blk = bs < n ? sel_s[bs] : -1;
-            const int row = blk >= 0 ? sel_row0(blk, l, t) : -(1 << 24);
-#pragma unroll
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_4d(dst + h * 16384 + sub * l * 128, is_v ? &maps.v_blk : &maps.k_blk,
-                          st_full + s, h * 64, g, row, b);
-          }
-          ++sc;
-        }
-      };
-      // 16 head rows per 64-channel half (fewer when Hq < 16; the rows the box
-      // leaves untouched only feed result columns that are never read)
       const int qrows = a.geo.Hq < 16 ? a.geo.Hq : 16;
       mbar_arrive_expect_tx(q_full, qrows * D * 2);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) tma_load_3d(sm + L::kQ + h * 2048, &maps.q, q_full, h * 64, g * G, b);
-      // compressed keys first: the block scores (and the top-n that the
-      // selected loads wait for) are computed while the rest streams in
-      for (int c = 0; c < it.ncc && ok; ++c) load_rows(&maps.kc, cmp_row0 + c * kChunk);
-      for (int c = 0; c < it.nwc && ok; ++c) load_rows(&maps.k_win, win_row0 + c * kChunk);
-      for (int c = 0; c < it.ncc && ok; ++c) load_rows(&maps.vc, cmp_row0 + c * kChunk);
-      for (int c = 0; c < it.nwc && ok; ++c) load_rows(&maps.v_win, win_row0 + c * kChunk);
-      if (ok && mbar_wait(idx_ready, 0, abort_flag, status, kWaitCycles)) {
-        load_sel(false);
-        if (ok) load_sel(true);
+      auto load_rows = [&](const CUtensorMap* map, int row0) {
+        const int s = sc % L::kStages, u = sc / L::kStages;
+        if (u > 0 && !mbar_wait(st_empty + s, (u - 1) & 1, abort_flag, status, kWaitCycles)) {
+          ok = false;
+          return;
+        }
+        mbar_arrive_expect_tx(st_full + s, L::kChunkBytes);
+        uint8_t* dst = sm + L::kRing + s * L::kChunkBytes;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) tma_load_4d(dst + h * 16384, map, st_full + s, h * 64, g, row0, b);
+        ++sc;
+      };
+      if (is_win) {
+        for (int c = 0; c < nchunks && ok; ++c) load_rows(&maps.k_win, P.win_row0 + c * kChunk);
+        for (int c = 0; c < nchunks && ok; ++c) load_rows(&maps.v_win, P.win_row0 + c * kChunk);
+      } else {
+        for (int c = 0; c < nchunks && ok; ++c) load_rows(&maps.kc, P.cmp_row0 + c * kChunk);
       }
       volatile int never = 0;
       for (int s = 0; s < L::kStages && s < sc; ++s) {
@@ -258,9 +348,6 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t id_qk = idesc_bf16(128, 16, false, false);
-      constexpr uint32_t id_pv = idesc_bf16(128, 16, true, true);
-      const uint32_t Qs = sbase + L::kQ, Ps = sbase + L::kP;
       int sc = 0;
       bool ok = mbar_wait(q_full, 0, abort_flag, status, kWaitCycles);
       tc_fence_after();
@@ -273,60 +360,23 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         return sbase + L::kRing + s * L::kChunkBytes;
       };
-      auto release_stage = [&]() {
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const uint32_t st = wait_stage();
+        if (!ok) break;
+        issue_qk<D>(tmem + c * 16, st, sbase + L::kQ);
         mma_commit(st_empty + (sc % L::kStages));
         ++sc;
-      };
-      auto qk = [&](int nchunks, uint32_t col) {
+      }
+      mma_commit(s_full);
+      if (is_win && ok && mbar_wait(p_full, 0, abort_flag, status, kWaitCycles)) {
+        tc_fence_after();
         for (int c = 0; c < nchunks && ok; ++c) {
           const uint32_t st = wait_stage();
-          if (!ok) return;
-#pragma unroll
-          for (int ks = 0; ks < KSTEPS; ++ks) {
-            const uint32_t qoff = (ks >> 2) * 2048 + (ks & 3) * 32;   // Q^T halves: 16 rows
-            const uint32_t soff = (ks >> 2) * 16384 + (ks & 3) * 32;  // chunk halves: 128 rows
-            mma_bf16_ss(tmem + col + c * 16, smem_desc(st + soff, 16, 1024, kLayoutSw128),
-                        smem_desc(Qs + qoff, 16, 1024, kLayoutSw128), id_qk, ks > 0);
-          }
-          release_stage();
+          if (!ok) break;
+          issue_pv(tmem + 128, st, sbase + L::kU + c * kPChunkBytes, c > 0);
+          mma_commit(st_empty + (sc % L::kStages));
+          ++sc;
         }
-      };
-      auto pv = [&](int nchunks, uint32_t pbuf, uint32_t col) {
-        for (int c = 0; c < nchunks && ok; ++c) {
-          const uint32_t st = wait_stage();
-          if (!ok) return;
-#pragma unroll
-          for (int ks = 0; ks < kChunk / 16; ++ks)
-            mma_bf16_ss(tmem + col, smem_desc(st + ks * 2048, 16384, 1024, kLayoutSw128),
-                        smem_desc(pbuf + c * 4096 + ks * 256, 128, 2048, kLayoutNone), id_pv,
-                        (c > 0 || ks > 0) ? 1u : 0u);
-          release_stage();
-        }
-      };
-      if (ok && it.ncc > 0) {
-        qk(it.ncc, kColSC);
-        mma_commit(sC_full);
-      }
-      if (ok) {
-        qk(it.nwc, kColSW);
-        mma_commit(sW_full);
-      }
-      if (ok && it.ncc > 0 && mbar_wait(pC_full, 0, abort_flag, status, kWaitCycles)) {
-        tc_fence_after();
-        pv(it.ncc, Ps + L::kPBytes, kColOC);
-      }
-      if (ok && mbar_wait(pW_full, 0, abort_flag, status, kWaitCycles)) {
-        tc_fence_after();
-        pv(it.nwc, Ps, kColOW);
-        mma_commit(pW_empty);
-      }
-      if (ok) {
-        qk(it.nsc, kColSS);
-        mma_commit(sS_full);
-      }
-      if (ok && mbar_wait(pS_full, 0, abort_flag, status, kWaitCycles)) {
-        tc_fence_after();
-        pv(it.nsc, Ps, kColOS);
       }
       mma_commit(o_done);
       mma_commit(fin);
@@ -334,228 +384,115 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(fin, 0, &never, nullptr, kWaitCycles / 4);
     }
   } else {
-    // ------------------------------------------------------------ softmax / top-n / epilogue
+    // ------------------------------------------------------------ softmax / epilogue
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // key lane of every chunk; channel in the epilogue
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float sl2 = a.geo.scale_log2;
     const uint32_t colmask = (G >= 16) ? 0xFFFFu : ((1u << G) - 1u);
-    // Two-sweep softmax over the S^T chunks at `col` (keys on lanes, heads on
-    // columns): writes unnormalised P^T into `pbuf` and returns 1/sum per head.
-    auto softmax = [&](uint32_t col, int nchunks, const bool (&kok)[8], uint32_t pbuf,
-                       float (&inv)[16]) {
-      float mx[16];
+    // keys of this lane that take part, one bit per chunk
+    uint32_t kok = 0;
+    for (int c = 0; c < nchunks; ++c) {
+      const int row = (is_win ? P.win_row0 : P.cmp_row0) + c * kChunk + r;
+      const bool on = is_win ? row >= max(0, t - a.geo.w + 1) : row >= 0;
+      kok |= on ? (1u << c) : 0u;
+    }
+    mbar_wait(s_full, 0, abort_flag, status, kWaitCycles);
+    tc_fence_after();
+    // sweep 1: per-head maximum (log2 units)
+    float mx[16];
 #pragma unroll
-      for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
+    for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
+    sweep_chunks<32>(lane_addr, 0, nchunks, [&](int c, const float(&v)[16]) {
+      if ((kok >> c) & 1u) {
 #pragma unroll
-      for (int c0 = 0; c0 < 8; c0 += 4) {
-        if (c0 >= nchunks) break;
-        float v[64];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float u16[16];
-          tmem_ld16(lane_addr + col + (c0 + cc) * 16, u16);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[cc * 16 + j] = u16[j];
-        }
-        tmem_ld_wait();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          if (c0 + cc < nchunks && kok[c0 + cc]) {
-#pragma unroll
-            for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[cc * 16 + h] * sl2);
-          }
+        for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[h] * sl2);
       }
-      reduce16_across_128<1>(mx, red, q4, lane, true);
-      float sm16[16];
+    });
+    reduce16_across_128<1>(mx, red, q4, lane, true);
+    float sm16[16];
 #pragma unroll
-      for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
-      const uint32_t pb = pbuf + (r >> 3) * 128 + (r & 7) * 16;
-#pragma unroll
-      for (int c0 = 0; c0 < 8; c0 += 4) {
-        if (c0 >= nchunks) break;
-        float v[64];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float u16[16];
-          tmem_ld16(lane_addr + col + (c0 + cc) * 16, u16);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[cc * 16 + j] = u16[j];
-        }
-        tmem_ld_wait();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = c0 + cc;
-          if (c >= nchunks) break;
-          float p[16];
-#pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            p[h] = (kok[c] && ((colmask >> h) & 1u)) ? ex2(v[cc * 16 + h] * sl2 - mx[h]) : 0.f;
-            sm16[h] += p[h];
-          }
-          uint32_t pk[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
-          st_shared_v4(pb + c * 4096, pk[0], pk[1], pk[2], pk[3]);
-          st_shared_v4(pb + c * 4096 + 2048, pk[4], pk[5], pk[6], pk[7]);
-        }
-      }
-      fence_async_smem();
-      reduce16_across_128<1>(sm16, red + 64, q4, lane, false);
-#pragma unroll
-      for (int h = 0; h < 16; ++h) inv[h] = (((colmask >> h) & 1u) && sm16[h] > 0.f) ? 1.f / sm16[h] : 0.f;
-    };
-    const uint32_t P0 = sbase + L::kP, P1 = P0 + L::kPBytes;
-    float inv_w[16], inv_c[16], inv_s[16];
-    // ---- compressed branch and block scores
-#pragma unroll
-    for (int h = 0; h < 16; ++h) inv_c[h] = 0.f;
-    if (it.ncc > 0) {
-      bool kok[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) kok[c] = c < it.ncc && cmp_row0 + c * kChunk + r >= 0;
-      mbar_wait(sC_full, 0, abort_flag, status, kWaitCycles);
-      tc_fence_after();
-      // sweep 1: per-head maximum (kept for the scores of sweep 3)
-      float mx[16];
-#pragma unroll
-      for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
-      {
-#pragma unroll
-        for (int c0 = 0; c0 < 8; c0 += 4) {
-          if (c0 >= it.ncc) break;
-          float v[64];
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            float u16[16];
-            tmem_ld16(lane_addr + kColSC + (c0 + cc) * 16, u16);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[cc * 16 + j] = u16[j];
-          }
-          tmem_ld_wait();
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            if (c0 + cc < it.ncc && kok[c0 + cc]) {
-#pragma unroll
-              for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[cc * 16 + h] * sl2);
-            }
-        }
-      }
-      reduce16_across_128<1>(mx, red, q4, lane, true);
-      // sweep 2: P^T and sums; sweep 3: normalised probabilities summed over heads
-      float sm16[16];
-#pragma unroll
-      for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
-      const uint32_t pb = P1 + (r >> 3) * 128 + (r & 7) * 16;
-      for (int c = 0; c < it.ncc; ++c) {
-        float v[16];
-        tmem_ld16(lane_addr + kColSC + c * 16, v);
-        tmem_ld_wait();
+    for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
+    if (is_win) {
+      // sweep 2: unnormalised P^T into shared memory and the sums
+      uint8_t* pbase = sm + L::kU;
+      sweep_chunks<8>(lane_addr, 0, nchunks, [&](int c, const float(&v)[16]) {
+        const bool on = (kok >> c) & 1u;
         float p[16];
 #pragma unroll
         for (int h = 0; h < 16; ++h) {
-          p[h] = (kok[c] && ((colmask >> h) & 1u)) ? ex2(v[h] * sl2 - mx[h]) : 0.f;
+          p[h] = (on && ((colmask >> h) & 1u)) ? ex2(v[h] * sl2 - mx[h]) : 0.f;
           sm16[h] += p[h];
         }
-        uint32_t pk[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
-        st_shared_v4(pb + c * 4096, pk[0], pk[1], pk[2], pk[3]);
-        st_shared_v4(pb + c * 4096 + 2048, pk[4], pk[5], pk[6], pk[7]);
-      }
+        store_pt(pbase + c * kPChunkBytes, r, p);
+      });
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(pC_full);
+      if (lane == 0) mbar_arrive(p_full);
       reduce16_across_128<1>(sm16, red + 64, q4, lane, false);
-      // log2 of each head's normaliser: p_norm = 2^(s*sl2 - mx - log2(sum))
-      float lnorm[16];
+      // epilogue: O_win = O^T / sum, thread = channel
+      mbar_wait(o_done, 0, abort_flag, status, kWaitCycles);
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(lane_addr + 128, o);
+      tmem_ld_wait();
+      if (r < D && !*abort_flag) {
 #pragma unroll
-      for (int h = 0; h < 16; ++h) {
-        inv_c[h] = (((colmask >> h) & 1u) && sm16[h] > 0.f) ? 1.f / sm16[h] : 0.f;
-        lnorm[h] = sm16[h] > 0.f ? mx[h] + __log2f(sm16[h]) : INFINITY;
-      }
-      for (int c = 0; c < it.ncc; ++c) {
-        float v[16];
-        tmem_ld16(lane_addr + kColSC + c * 16, v);
-        tmem_ld_wait();
-        const int j = cmp_row0 + c * kChunk + r;
-        if (kok[c]) {
-          float s = 0.f;
-#pragma unroll
-          for (int h = 0; h < 16; ++h)
-            if ((colmask >> h) & 1u) s += ex2(v[h] * sl2 - lnorm[h]);
-          scores[j] = s;
+        for (int h = 0; h < 16; ++h) {
+          if (h >= G) break;
+          rec.win[h * D + r] = sm16[h] > 0.f ? o[h] / sm16[h] : 0.f;
         }
       }
-    }
-    // ---- top-n (one warp), indices to shared memory, global output and the producer
-    named_bar_128<1>();
-    if (warp == 2) {
-      int* gsel = a.sel ? a.sel + ((size_t)b * a.geo.Hkv + g) * n : nullptr;
-      warp_topn([&](int j) { return scores[j]; }, it.C, it.ncand, n, hist, [&](int i, int j) {
-        sel_s[i] = j;
-        if (gsel) gsel[i] = j;
+    } else {
+      // sweep 2: sums -> log2-sum-exp per head
+      sweep_chunks<32>(lane_addr, 0, nchunks, [&](int c, const float(&v)[16]) {
+        if ((kok >> c) & 1u) {
+#pragma unroll
+          for (int h = 0; h < 16; ++h)
+            if ((colmask >> h) & 1u) sm16[h] += ex2(v[h] * sl2 - mx[h]);
+        }
       });
-      __syncwarp();
-      if (lane == 0) mbar_arrive(idx_ready);
-    }
-    named_bar_128<1>();
-    // ---- window
-    {
-      bool kok[8];
-      const int lo = max(0, t - a.geo.w + 1);
+      reduce16_across_128<1>(sm16, red + 64, q4, lane, false);
+      float lse[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) kok[c] = c < it.nwc && win_row0 + c * kChunk + r >= lo;
-      mbar_wait(sW_full, 0, abort_flag, status, kWaitCycles);
-      tc_fence_after();
-      softmax(kColSW, it.nwc, kok, P0, inv_w);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pW_full);
-    }
-    // ---- selected branch
-    {
-      bool kok[8];
-      const int key_in_blk = r & (l - 1), slot_in_chunk = r >> lg_l;
+      for (int h = 0; h < 16; ++h) lse[h] = sm16[h] > 0.f ? mx[h] + __log2f(sm16[h]) : INFINITY;
+      // sweep 3: normalised probabilities -> P^T (workspace) and block scores
+      float* scores = reinterpret_cast<float*>(sm + L::kU);
+      const bool live = !*abort_flag;
+      sweep_chunks<32>(lane_addr, 0, nchunks, [&](int c, const float(&v)[16]) {
+        const bool on = (kok >> c) & 1u;
+        float p[16];
+        float s = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int bs = c * bpc + slot_in_chunk;
-        const int blk = (c < it.nsc && bs < n) ? sel_s[bs] : -1;
-        kok[c] = blk >= 0 && sel_row0(blk, l, t) + key_in_blk >= blk * l;
-      }
-      mbar_wait(sS_full, 0, abort_flag, status, kWaitCycles);
-      mbar_wait(pW_empty, 0, abort_flag, status, kWaitCycles);
-      tc_fence_after();
-      softmax(kColSS, it.nsc, kok, P0, inv_s);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pS_full);
-    }
-    // ---- epilogue: lane = channel
-    mbar_wait(o_done, 0, abort_flag, status, kWaitCycles);
-    tc_fence_after();
-    float ow[16], ocm[16], os[16];
-    tmem_ld16(lane_addr + kColOW, ow);
-    tmem_ld16(lane_addr + kColOC, ocm);
-    tmem_ld16(lane_addr + kColOS, os);
-    tmem_ld_wait();
-    if (r < D && !*abort_flag) {
-      const int Hq = a.geo.Hq;
-#pragma unroll
-      for (int h = 0; h < 16; ++h) {
-        if (h >= G) break;
-        const int gh = g * G + h;
-        const float* gt = a.gates + ((size_t)b * Hq + gh) * 3;
-        const float oc = it.ncc > 0 ? ocm[h] * inv_c[h] : 0.f;
-        const float val = __ldg(gt + 0) * oc + __ldg(gt + 1) * os[h] * inv_s[h] +
-                          __ldg(gt + 2) * ow[h] * inv_w[h];
-        const size_t oi = ((size_t)b * Hq + gh) * D + r;
-        if (a.geo.out_f32) {
-          static_cast<float*>(a.out)[oi] = val;
+        for (int h = 0; h < 16; ++h) {
+          p[h] = (on && ((colmask >> h) & 1u)) ? ex2(v[h] * sl2 - lse[h]) : 0.f;
+          s += p[h];
+        }
+        if (live) store_pt(rec.pt + (size_t)c * kPChunkBytes, r, p);
+        const int j = P.cmp_row0 + c * kChunk + r;
+        if (on) scores[j] = s;
+      });
+      named_bar_128<1>();
+      // top-n (one warp): the workspace copy feeds the selected units
+      if (warp == 2) {
+        int* gsel = a.sel ? a.sel + ((size_t)b * a.geo.Hkv + g) * n : nullptr;
+        auto put = [&](int i, int j) {
+          if (live) rec.sel[i] = j;
+          if (gsel && live) gsel[i] = j;
+        };
+        // the register selection for up to 1024 candidates, else (or when
+        // too many keys tie at its bound) the radix select
+        const bool regs_ok = P.ncand <= 1024 && n <= 32;
+        if (!a.geo.remap) {
+          auto score = [&](int j) { return scores[j]; };
+          if (!(regs_ok && warp_topn_regs(score, P.C, P.ncand, n, cand, put)))
+            warp_topn(score, P.C, P.ncand, n, hist, put);
         } else {
-          const __nv_bfloat16 bv = __float2bfloat16_rn(val);
-          static_cast<uint16_t*>(a.out)[oi] = *reinterpret_cast<const uint16_t*>(&bv);
+          const int C = P.C;
+          auto score = [&](int j) { return remap_score(a.geo, [&](int i) { return scores[i]; }, C, j); };
+          if (!(regs_ok && warp_topn_regs(score, P.ncand, P.ncand, n, cand, put)))
+            warp_topn(score, P.ncand, P.ncand, n, hist, put);
         }
       }
     }
@@ -564,24 +501,416 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, ncols);
   }
 }
 
+// ------------------------------------------------------------------ kernel B
 template <int D>
-cudaError_t launch_decode_t(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s) {
-  using L = DecLayout<D>;
-  static bool configured[64] = {};
+struct DecBLayout {
+  static constexpr int kStages = 3;
+  static constexpr int kChunkBytes = kChunk * D * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kRing = 4096;
+  static constexpr int kP = kRing + kStages * kChunkBytes + ring_pad<D>();  // 2 chunks of P^T
+  static constexpr int kRed = kP + 2 * kPChunkBytes;        // float [2][64]
+  static constexpr int kSel = kRed + 2 * 64 * 4;            // int [64]
+  static constexpr int kFlag = kSel + 64 * 4;               // int
+  static constexpr int kBars = kFlag + 16;
+  static constexpr int kEnd = kBars + 16 * 8;
+  static constexpr int kSmem = kEnd + 1024;
+  // a PV operand spans 32 KB from the start of its stage
+  static_assert(kRing + (kStages - 1) * kChunkBytes + 32768 <= kEnd, "PV operand inside smem");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
+    nsa_decode_b_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ DecodeMaps maps) {
+  using L = DecBLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
+  uint64_t* q_full = bars + 0;
+  uint64_t* st_full = bars + 1;   // [3]
+  uint64_t* st_empty = bars + 4;  // [3]
+  uint64_t* pt_full = bars + 7;   // P^T chunks of a cmp unit
+  uint64_t* s_full = bars + 8;
+  uint64_t* p_full = bars + 9;
+  uint64_t* o_done = bars + 10;
+  uint64_t* fin = bars + 11;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  float* red = reinterpret_cast<float*>(sm + L::kRed);
+  int* sel_s = reinterpret_cast<int*>(sm + L::kSel);
+  int* last_flag = reinterpret_cast<int*>(sm + L::kFlag);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int units = a.ncv_max + a.nsl;
+  const int pair = blockIdx.x / units, unit = blockIdx.x % units;
+  const DecPair P = dec_pair(a, pair);
+  if (!P.ok) return;  // kernel A has recorded the bad length
+  const bool is_cmp = unit < a.ncv_max;
+  const int u = is_cmp ? unit : unit - a.ncv_max;
+  // chunks [c_lo, c_hi) of the compressed blocks or of the selected keys
+  const int total_chunks = is_cmp ? P.ncc : P.nsc;
+  const int c_lo = min(2 * u, total_chunks), c_hi = min(2 * u + 2, total_chunks);
+  const int nch = c_hi - c_lo;
+  const PairRecs rec = pair_recs(a, pair);
+  // selection blocks of l' tokens
+  const int G = a.geo.G, l = a.geo.ls, n = a.geo.n, lg_l = a.geo.lg_ls;
+  const int bpc = kChunk >> lg_l;
+  const int b = P.b, g = P.g, t = P.t;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < L::kStages; ++i) {
+      mbar_init(st_full + i, 1);
+      mbar_init(st_empty + i, 1);
+    }
+    mbar_init(pt_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 4);
+    mbar_init(o_done, 1);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // everything below reads kernel A's results (selection, P^T, window).  The
+  // TMEM is allocated only after kernel A has finished: a CTA of this grid
+  // that waits here holds no TMEM that a CTA of kernel A could need.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 64);  // S^T of two chunks at 0 and 16, O^T at 32
+    tmem_relinquish();
+  }
+  if (threadIdx.x < 64) sel_s[threadIdx.x] = (!is_cmp && threadIdx.x < n) ? rec.sel[threadIdx.x] : -1;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t sbase = smem_u32(sm);
+  int* status = a.status;
+
+  if (nch > 0) {
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        int sc = 0;
+        bool ok = true;
+        auto acquire = [&]() -> uint8_t* {
+          const int s = sc % L::kStages, uu = sc / L::kStages;
+          if (uu > 0 && !mbar_wait(st_empty + s, (uu - 1) & 1, abort_flag, status, kWaitCycles)) {
+            ok = false;
+            return nullptr;
+          }
+          mbar_arrive_expect_tx(st_full + s, L::kChunkBytes);
+          return sm + L::kRing + s * L::kChunkBytes;
+        };
+        if (is_cmp) {
+          mbar_arrive_expect_tx(pt_full, nch * kPChunkBytes);
+          for (int c = 0; c < nch; ++c)
+            bulk_load(sm + L::kP + c * kPChunkBytes, rec.pt + (size_t)(c_lo + c) * kPChunkBytes,
+                      kPChunkBytes, pt_full);
+          for (int c = c_lo; c < c_hi && ok; ++c) {
+            uint8_t* dst = acquire();
+            if (!dst) break;
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(dst + h * 16384, &maps.vc, st_full + sc % L::kStages, h * 64, g,
+                          P.cmp_row0 + c * kChunk, b);
+            ++sc;
+          }
+        } else {
+          const int qrows = a.geo.Hq < 16 ? a.geo.Hq : 16;
+          mbar_arrive_expect_tx(q_full, qrows * D * 2);
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(sm + L::kQ + h * 2048, &maps.q, q_full, h * 64, g * G, b);
+          for (int pass = 0; pass < 2 && ok; ++pass) {  // keys, then values
+            for (int c = c_lo; c < c_hi && ok; ++c) {
+              uint8_t* dst = acquire();
+              if (!dst) break;
+              const int s = sc % L::kStages;
+              for (int sub = 0; sub < bpc; ++sub) {
+                const int bs = c * bpc + sub;
+                const int blk = bs < n ? sel_s[bs] : -1;
+                const int row = blk >= 0 ? sel_row0(blk, l, t) : -(1 << 24);
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                  tma_load_4d(dst + h * 16384 + sub * l * 128, pass ? &maps.v_blk : &maps.k_blk,
+                              st_full + s, h * 64, g, row, b);
+              }
+              ++sc;
+            }
+          }
+        }
+        volatile int never = 0;
+        for (int s = 0; s < L::kStages && s < sc; ++s) {
+          const int last = sc - 1 - ((sc - 1 - s) % L::kStages);
+          mbar_wait(st_full + s, (last / L::kStages) & 1, &never, nullptr, kWaitCycles / 4);
+        }
+        if (is_cmp) mbar_wait(pt_full, 0, &never, nullptr, kWaitCycles / 4);
+        else mbar_wait(q_full, 0, &never, nullptr, kWaitCycles / 4);
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        int sc = 0;
+        bool ok = true;
+        auto wait_stage = [&]() -> uint32_t {
+          const int s = sc % L::kStages;
+          if (!mbar_wait(st_full + s, (sc / L::kStages) & 1, abort_flag, status, kWaitCycles)) {
+            ok = false;
+            return 0;
+          }
+          tc_fence_after();
+          return sbase + L::kRing + s * L::kChunkBytes;
+        };
+        if (is_cmp) {
+          ok = mbar_wait(pt_full, 0, abort_flag, status, kWaitCycles);
+          for (int c = 0; c < nch && ok; ++c) {
+            const uint32_t st = wait_stage();
+            if (!ok) break;
+            issue_pv(tmem + 32, st, sbase + L::kP + c * kPChunkBytes, c > 0);
+            mma_commit(st_empty + (sc % L::kStages));
+            ++sc;
+          }
+        } else {
+          ok = mbar_wait(q_full, 0, abort_flag, status, kWaitCycles);
+          tc_fence_after();
+          for (int c = 0; c < nch && ok; ++c) {
+            const uint32_t st = wait_stage();
+            if (!ok) break;
+            issue_qk<D>(tmem + c * 16, st, sbase + L::kQ);
+            mma_commit(st_empty + (sc % L::kStages));
+            ++sc;
+          }
+          mma_commit(s_full);
+          if (ok && mbar_wait(p_full, 0, abort_flag, status, kWaitCycles)) {
+            tc_fence_after();
+            for (int c = 0; c < nch && ok; ++c) {
+              const uint32_t st = wait_stage();
+              if (!ok) break;
+              issue_pv(tmem + 32, st, sbase + L::kP + c * kPChunkBytes, c > 0);
+              mma_commit(st_empty + (sc % L::kStages));
+              ++sc;
+            }
+          }
+        }
+        mma_commit(o_done);
+        mma_commit(fin);
+        volatile int never = 0;
+        mbar_wait(fin, 0, &never, nullptr, kWaitCycles / 4);
+      }
+    } else {
+      // ---------------------------------------------------------- softmax / partial
+      const int q4 = warp & 3;
+      const int r = q4 * 32 + lane;
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+      const float sl2 = a.geo.scale_log2;
+      const uint32_t colmask = (G >= 16) ? 0xFFFFu : ((1u << G) - 1u);
+      float mx[16], sm16[16];
+      if (!is_cmp) {
+        // keys of this lane that are visible selected keys, per chunk
+        const int key_in_blk = r & (l - 1), slot_in_chunk = r >> lg_l;
+        uint32_t kok = 0;
+        for (int c = 0; c < nch; ++c) {
+          const int bs = (c_lo + c) * bpc + slot_in_chunk;
+          const int blk = bs < n ? sel_s[bs] : -1;
+          kok |= (blk >= 0 && sel_row0(blk, l, t) + key_in_blk >= blk * l) ? (1u << c) : 0u;
+        }
+        mbar_wait(s_full, 0, abort_flag, status, kWaitCycles);
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
+        sweep_chunks<4>(lane_addr, 0, nch, [&](int c, const float(&v)[16]) {
+          if ((kok >> c) & 1u) {
+#pragma unroll
+            for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[h] * sl2);
+          }
+        });
+        reduce16_across_128<1>(mx, red, q4, lane, true);
+#pragma unroll
+        for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
+        sweep_chunks<4>(lane_addr, 0, nch, [&](int c, const float(&v)[16]) {
+          const bool on = (kok >> c) & 1u;
+          float p[16];
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            p[h] = (on && ((colmask >> h) & 1u)) ? ex2(v[h] * sl2 - mx[h]) : 0.f;
+            sm16[h] += p[h];
+          }
+          store_pt(sm + L::kP + c * kPChunkBytes, r, p);
+        });
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+        reduce16_across_128<1>(sm16, red + 64, q4, lane, false);
+      }
+      mbar_wait(o_done, 0, abort_flag, status, kWaitCycles);
+      tc_fence_after();
+      float o[16];
+      tmem_ld16(lane_addr + 32, o);
+      tmem_ld_wait();
+      if (r < D && !*abort_flag) {
+        if (is_cmp) {
+          float* dst = rec.cmp + (size_t)u * G * D;
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            if (h >= G) break;
+            dst[h * D + r] = o[h];
+          }
+        } else {
+          float* dst = rec.slc + (size_t)u * (G * D + 32);
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            if (h >= G) break;
+            dst[h * D + r] = o[h];
+          }
+          if (r < G) {
+            float mv = 0.f, lv = 0.f;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) {
+              mv = (h == r) ? mx[h] : mv;
+              lv = (h == r) ? sm16[h] : lv;
+            }
+            dst[G * D + r] = mv;
+            dst[G * D + 16 + r] = lv;
+          }
+        }
+      }
+    }
+  } else if (warp >= 2 && !is_cmp) {
+    // a selected unit with no chunk: an empty partial
+    const int r = threadIdx.x - 64;
+    float* dst = rec.slc + (size_t)u * (G * D + 32);
+    if (r < D)
+      for (int h = 0; h < G; ++h) dst[h * D + r] = 0.f;
+    if (r < G) {
+      dst[G * D + r] = -INFINITY;
+      dst[G * D + 16 + r] = 0.f;
+    }
+  }
+  // ---- the last unit of the pair merges the partials (step 7)
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int done = atomicAdd(a.counters + pair, 1);
+    *last_flag = done == units - 1;
+  }
+  __syncthreads();
+  if (*last_flag) {
+    __threadfence();
+    // per-head statistics of the selected partials and the gates, staged in
+    // the (now idle) P^T region; then every (head, 4 channels) item issues
+    // all of its partial loads before combining them
+    float* ml = reinterpret_cast<float*>(sm + L::kP);  // [nsl][m[16], sum[16]]
+    float* gt = ml + 8 * 32;                            // [G][3]
+    const int Hq = a.geo.Hq;
+    for (int i = threadIdx.x; i < a.nsl * 32; i += blockDim.x)
+      ml[i] = __ldcg(rec.slc + (size_t)(i >> 5) * (G * D + 32) + G * D + (i & 31));
+    for (int i = threadIdx.x; i < G * 3; i += blockDim.x)
+      gt[i] = __ldg(a.gates + ((size_t)b * Hq + g * G) * 3 + i);
+    __syncthreads();
+    const int ncv = (P.ncc + 1) / 2;
+    for (int item = threadIdx.x; item < G * (D / 4); item += blockDim.x) {
+      const int h = item / (D / 4), c4 = (item - h * (D / 4)) * 4;
+      float4 vs[kMaxSlcUnits], vc[kMaxCmpUnits];
+#pragma unroll
+      for (int s2 = 0; s2 < kMaxSlcUnits; ++s2)
+        if (s2 < a.nsl)
+          vs[s2] = __ldcg(reinterpret_cast<const float4*>(rec.slc + (size_t)s2 * (G * D + 32) +
+                                                          h * D + c4));
+#pragma unroll
+      for (int u2 = 0; u2 < kMaxCmpUnits; ++u2)
+        if (u2 < ncv)
+          vc[u2] = __ldcg(reinterpret_cast<const float4*>(rec.cmp + ((size_t)u2 * G + h) * D + c4));
+      const float4 w4 = __ldcg(reinterpret_cast<const float4*>(rec.win + h * D + c4));
+      float M = -INFINITY;
+      for (int s2 = 0; s2 < a.nsl; ++s2) M = fmaxf(M, ml[s2 * 32 + h]);
+      float4 os = make_float4(0.f, 0.f, 0.f, 0.f);
+      float ls = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < kMaxSlcUnits; ++s2) {
+        if (s2 >= a.nsl) break;
+        const float ms = ml[s2 * 32 + h];
+        const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
+        ls += ml[s2 * 32 + 16 + h] * f;
+        os.x += vs[s2].x * f;
+        os.y += vs[s2].y * f;
+        os.z += vs[s2].z * f;
+        os.w += vs[s2].w * f;
+      }
+      float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u2 = 0; u2 < kMaxCmpUnits; ++u2) {
+        if (u2 >= ncv) break;
+        oc.x += vc[u2].x;
+        oc.y += vc[u2].y;
+        oc.z += vc[u2].z;
+        oc.w += vc[u2].w;
+      }
+      const float inv = ls > 0.f ? 1.f / ls : 0.f;
+      const float g0 = gt[h * 3 + 0], g1 = gt[h * 3 + 1] * inv, g2 = gt[h * 3 + 2];
+      const float e[4] = {g0 * oc.x + g1 * os.x + g2 * w4.x, g0 * oc.y + g1 * os.y + g2 * w4.y,
+                          g0 * oc.z + g1 * os.z + g2 * w4.z, g0 * oc.w + g1 * os.w + g2 * w4.w};
+      const size_t oi = ((size_t)b * Hq + g * G + h) * D + c4;
+      if (a.geo.out_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.out) + oi) = make_float4(e[0], e[1], e[2], e[3]);
+      } else {
+        *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + oi) =
+            make_uint2(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]));
+      }
+    }
+    if (threadIdx.x == 0) a.counters[pair] = 0;
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes, bool (&configured)[64]) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(nsa_decode_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  nsa_decode_kernel<D><<<a.batch * a.geo.Hkv, 192, L::kSmem, s>>>(a, m);
+  return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_decode_a_t(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s) {
+  static bool conf[64] = {};
+  cudaError_t e = set_smem(nsa_decode_a_kernel<D>, DecALayout<D>::kSmem, conf);
+  if (e != cudaSuccess) return e;
+  nsa_decode_a_kernel<D><<<a.batch * a.geo.Hkv * 2, kDecThreads, DecALayout<D>::kSmem, s>>>(a, m);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_decode_b_t(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s) {
+  static bool conf[64] = {};
+  cudaError_t e = set_smem(nsa_decode_b_kernel<D>, DecBLayout<D>::kSmem, conf);
+  if (e != cudaSuccess) return e;
+  // programmatic dependent launch: the CTAs of this grid start while kernel A
+  // runs and wait for its results inside the kernel (griddepcontrol.wait)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.batch * a.geo.Hkv * (a.ncv_max + a.nsl));
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = DecBLayout<D>::kSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, nsa_decode_b_kernel<D>, a, m);
 }
 
 }  // namespace
@@ -589,20 +918,18 @@ cudaError_t launch_decode_t(const DecodeArgs& a, const DecodeMaps& m, cudaStream
 cudaError_t launch_decode_compress(const DecodeArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)a.geo.l * a.geo.D * sizeof(float);
   static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(nsa_decode_compress_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 128 * 4);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
+  cudaError_t e = set_smem(nsa_decode_compress_kernel, 64 * 128 * 4, configured);
+  if (e != cudaSuccess) return e;
   nsa_decode_compress_kernel<<<dim3(a.batch, a.geo.Hkv, 2), 256, smem, s>>>(a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s) {
-  return a.geo.D == 128 ? launch_decode_t<128>(a, m, s) : launch_decode_t<64>(a, m, s);
+cudaError_t launch_decode_a(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s) {
+  return a.geo.D == 128 ? launch_decode_a_t<128>(a, m, s) : launch_decode_a_t<64>(a, m, s);
+}
+
+cudaError_t launch_decode_b(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s) {
+  return a.geo.D == 128 ? launch_decode_b_t<128>(a, m, s) : launch_decode_b_t<64>(a, m, s);
 }
 
 }  // namespace nsa

@@ -32,7 +32,7 @@ __global__ void nsa_meta_kernel(PrefillArgs a, int max_seqlen) {
       bad = 1;
       break;
     }
-    c += T / a.geo.l;
+    c += num_cmp_blocks(T, a.geo.l, a.geo.d);
     tl += (T + a.geo.tpt - 1) / a.geo.tpt;
     a.cmp_off[b + 1] = c;
     a.tile_off[b + 1] = tl;
@@ -52,7 +52,7 @@ cudaError_t launch_meta(const PrefillArgs& a, cudaStream_t s) {
 // ------------------------------------------------------------------ compression
 // Kc[r, h, c] = sum_{p < l, c' < D} W[h, c, p*D + c'] * X[tok0(r) + p, h, c']
 // for every complete block r of every sequence (tok0 = first token of the
-// block).  A tiled fp32 GEMM: CTA tile 32 blocks x D outputs, k-step 32.
+// block: the sequence start plus d times the block's index in it).  A tiled fp32 GEMM: CTA tile 32 blocks x D outputs, k-step 32.
 // Rows in [cmp_total, cmp_rows) are zero-filled so that later tiles reading
 // past the last sequence see finite values.
 template <int D>
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(256) nsa_compress_kernel(PrefillArgs a) {
     int t0 = -1;
     if (r < C) {
       const int b = seq_of_offset(a.cmp_off, a.batch, r);
-      t0 = __ldg(a.cu + b) + (r - a.cmp_off[b]) * l;
+      t0 = __ldg(a.cu + b) + (r - a.cmp_off[b]) * a.geo.d;
     }
     tok0[tid] = t0;
   }
@@ -157,13 +157,16 @@ cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s) {
 }
 
 // ------------------------------------------------------------------ top-n
-// One warp per (token, KV group); the selection itself is warp_topn.
+// One warp per (token, KV group); the selection itself is warp_topn.  With
+// l == d == l' the candidates' scores are the compressed-block scores; else
+// each selection block's score is first summed from the compressed blocks
+// that overlap it (written to the selection-score table, then ranked).
 __global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
   __shared__ unsigned long long cand_all[8][kTopnCand];
-  const int warp = threadIdx.x / 32;
-  const int H = a.geo.Hkv, l = a.geo.l, n = a.geo.n;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int H = a.geo.Hkv, n = a.geo.n;
   const long long row = (long long)blockIdx.x * 8 + warp;
   if (row >= (long long)a.total_tokens * H) return;
   const int tg = (int)(row / H), g = (int)(row % H);
@@ -171,11 +174,23 @@ __global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   const int t = tg - __ldg(a.cu + b);
   const float* S = a.scores + ((size_t)tg * H + g) * a.geo.cmp_cap;
   int* out = a.sel + ((size_t)tg * H + g) * n;
-  const int ncmp = (t + 1) / l, ncand = t / l + 1;
-  auto score = [&](int j) { return S[j]; };
+  const int ncmp = num_cmp_blocks(t + 1, a.geo.l, a.geo.d), ncand = t / a.geo.ls + 1;
   auto put = [&](int i, int j) { out[i] = j; };
-  if (ncand <= 1024 && n <= 32 && warp_topn_regs(score, ncmp, ncand, n, cand_all[warp], put)) return;
-  warp_topn(score, ncmp, ncand, n, hist_all[warp], put);
+  if (!a.geo.remap) {
+    auto score = [&](int j) { return S[j]; };
+    if (ncand <= 1024 && n <= 32 && warp_topn_regs(score, ncmp, ncand, n, cand_all[warp], put))
+      return;
+    warp_topn(score, ncmp, ncand, n, hist_all[warp], put);
+    return;
+  }
+  float* Ssel = a.sel_scores + ((size_t)tg * H + g) * a.geo.sel_cap;
+  for (int j = lane; j < ncand; j += 32)
+    Ssel[j] = remap_score(a.geo, [&](int i) { return S[i]; }, ncmp, j);
+  __syncwarp();
+  auto score = [&](int j) { return Ssel[j]; };
+  if (ncand <= 1024 && n <= 32 && warp_topn_regs(score, ncand, ncand, n, cand_all[warp], put))
+    return;
+  warp_topn(score, ncand, ncand, n, hist_all[warp], put);
 }
 
 cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s) {

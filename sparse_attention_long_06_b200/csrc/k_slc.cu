@@ -60,6 +60,10 @@ struct SlcLayout {
   static constexpr int kSmem = kEnd;
   static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kP % 1024 == 0, "swizzle alignment");
   static_assert(kSmem <= 232448, "shared memory budget");
+  // the PV operand V^T is 128 channels (two 64-channel halves kVBytes / 2
+  // apart); with D = 64 its second half reads past the slot, still inside
+  // shared memory
+  static_assert(kV + kVSlots * kVBytes + (D == 64 ? kVBytes : 0) <= kEnd, "PV operand inside smem");
 };
 
 constexpr int kSlcThreads = 384;
@@ -166,7 +170,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t sbase = smem_u32(sm);
   int* status = a.status;
-  const int G = a.geo.G, l = a.geo.l, lg_l = a.geo.lg_l, n = a.geo.n;
+  // selection blocks of l' tokens
+  const int G = a.geo.G, l = a.geo.ls, lg_l = a.geo.lg_ls, n = a.geo.n;
   const int bpc = kChunk >> lg_l;        // blocks per 128-key chunk
   const int nsc = (n + bpc - 1) / bpc;   // chunks per job
   const int njobs = slc_jobs_of_cta(a);
@@ -427,6 +432,17 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         kok |= (blk_next[c] >= 0 && (blk_next[c] << lg_l) + key_in_blk <= jb.t) ? (1u << c) : 0u;
       nj = slc_job(a, blockIdx.x + (long long)(j + 2) * gridDim.x);
       load_blk(nj, blk_next);
+      // the epilogue of job j (one job from now) reads its G rows of O_cmp
+      // and g_win O_win from HBM: bring them into L2 now, one 128-byte line
+      // per thread (G * D * 4 bytes each)
+      if (jb.valid) {
+        const size_t base = ((size_t)jb.row * Hq + jb.g * G) * D;
+        const int lines = (G * D * 4) >> 7;
+        if (r < lines) {
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.o_cmp + base + r * 32) : "memory");
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.o_win + base + r * 32) : "memory");
+        }
+      }
 
       mbar_wait(s_full + w, k & 1, abort_flag, status, kWaitCycles);
       tc_fence_after();

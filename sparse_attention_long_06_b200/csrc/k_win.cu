@@ -10,16 +10,23 @@
 // One persistent CTA per SM walks dense tiles of 128 MMA rows = (128 / G)
 // consecutive tokens x the G query heads of one KV group (all tiles of group
 // 0 first).  The tile's window keys [t0 - w + 1, t0 + 128 / G - 1] are shared
-// by all of its rows and are streamed in chunks of 128 keys:
-//   pass 1: S = Q K^T (rows on TMEM lanes), masked to each row's window:
-//           row maximum;
-//   pass 2: S again, P = exp(s - max) (largest element exactly 1, K-major A
-//           operand in shared memory) and its row sum in fp32, O += P V in
-//           TMEM; the epilogue scales row r by g_win / sum.
-// Warp roles: 0 = TMA producer, 1 = tcgen05.mma issuer, 2..5 and 6..9 = two
-// softmax warpgroups that take alternate key chunks of both passes (each with
-// its own TMEM score buffer and P buffer) and split the epilogue's columns
-// (thread i of warp w owns TMEM lane 32 * (w % 4) + i).
+// by all of its rows and are streamed once, in chunks of 128 keys (the last
+// one only as wide as the keys it holds, rounded up to 16).  One pass with an
+// online softmax:
+//   S = Q K^T (rows on TMEM lanes), masked to each row's window; the chunk's
+//   row maximum raises the running maximum m only when it grows by more than
+//   2^8 (then the row's accumulator and sum are rescaled), so that most
+//   chunks keep m; P = exp2(s - m) (bf16, K-major A operand in shared
+//   memory), its row sum in fp32, O += P V in TMEM.
+// Two softmax warpgroups take alternate key chunks, each with its own TMEM
+// score buffer, P buffer, running (m, sum) and O accumulator; the epilogue
+// merges the two accumulators of a row and stores g_win * O / sum.
+// Warp roles (three warpgroups): 0 = TMA producer, 1 = tcgen05.mma issuer,
+// 2..3 idle; 4..7 and 8..11 = the two softmax warpgroups (thread i of warp w
+// owns TMEM lane 32 * (w % 4) + i; in the epilogue, softmax warpgroup w
+// stores columns [w D/2, (w+1) D/2) of the rows).  The first warpgroup gives
+// registers to the softmax warpgroups (setmaxnreg 56 / 224), which hold a
+// whole 128-key row of scores in registers.
 #include <type_traits>
 
 #include "nsa_internal.cuh"
@@ -39,7 +46,7 @@ struct WinLayout {
   static constexpr int kQ = 0;                              // 2 buffers
   static constexpr int kRing = kQ + 2 * kQBytes;            // kStages
   static constexpr int kP = kRing + kStages * kChunkBytes;  // 2 buffers (one per warpgroup)
-  static constexpr int kStat = kP + 2 * kPBytes;            // float m, l, m1, l1 [128]
+  static constexpr int kStat = kP + 2 * kPBytes;            // float m[2][128], l[2][128]
   static constexpr int kBars = kStat + 4 * 128 * 4;
   static constexpr int kEnd = kBars + 32 * 8;
   // at least 116 KB so that one CTA owns an SM (it allocates all 512 TMEM columns)
@@ -47,7 +54,9 @@ struct WinLayout {
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-constexpr int kWinThreads = 320;
+constexpr int kWinThreads = 384;
+constexpr uint32_t kRegsControl = 56;   // producer / MMA warpgroup
+constexpr uint32_t kRegsSoftmax = 224;  // softmax warpgroups: 56 + 2 * 224 = 3 * 168
 
 struct WinItem {
   int valid, b, g, t0, T, row0, ntok, ws, nc, cu0, span;
@@ -106,10 +115,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   uint64_t* fin = bars + 20;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 22);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
-  float* m_s = reinterpret_cast<float*>(sm + L::kStat);  // merged row max (scaled, log2)
-  float* l_s = m_s + 128;                                 // row sum, warpgroup 0's part
-  float* m1_s = m_s + 256;
-  float* l1_s = m_s + 384;                                // row sum, warpgroup 1's part
+  float* m_s = reinterpret_cast<float*>(sm + L::kStat);  // [warpgroup][row] running max (log2)
+  float* l_s = m_s + 256;                                 // [warpgroup][row] running sum
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (a.meta->bad) return;
@@ -147,7 +154,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
   const uint32_t sbase = smem_u32(sm);
   int* status = a.status;
   const int G = a.geo.G;
-
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -180,12 +188,13 @@ __global__ void __launch_bounds__(kWinThreads, 1)
           tma_load_3d(sm + L::kQ + qb * L::kQBytes + h * 16384, &maps.q, q_full + qb, h * 64,
                       it.g * G, it.row0);
         ++qc;
-        for (int c = 0; c < it.nc && ok; ++c) load_chunk(&maps.k_win, it, c);
-        if (ok) load_chunk(&maps.k_win, it, 0);
-        for (int c = 0; c < it.nc && ok; ++c) {
-          if (c + 1 < it.nc) load_chunk(&maps.k_win, it, c + 1);
-          if (ok) load_chunk(&maps.v_win, it, c);
+        // the MMA issuer's order: K(0), then K(c) and V(c-1), then V(nc-1)
+        load_chunk(&maps.k_win, it, 0);
+        for (int c = 1; c < it.nc && ok; ++c) {
+          load_chunk(&maps.k_win, it, c);
+          if (ok) load_chunk(&maps.v_win, it, c - 1);
         }
+        if (ok) load_chunk(&maps.v_win, it, it.nc - 1);
       }
       // drain: every issued copy has landed before the CTA retires (also
       // after an abort, hence a private never-set abort flag)
@@ -233,6 +242,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         ++sc;
         ++s_use[buf];
       };
+      // chunk c accumulates into the O of warpgroup c & 1 (TMEM columns
+      // 256 + (c & 1) * D); the first chunk of each warpgroup overwrites it
       auto pv = [&](int c, int cw) {
         const int s = sc % L::kStages, pb = c & 1;
         if (!mbar_wait(st_full + s, (sc / L::kStages) & 1, abort_flag, status, kWaitCycles) ||
@@ -247,10 +258,11 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         tc_fence_after();
         const uint32_t stage = sbase + L::kRing + s * L::kChunkBytes;
         const uint32_t P = sbase + L::kP + pb * L::kPBytes;
+        const uint32_t ocol = 256 + pb * D;
         for (int ks = 0; ks < cw / 16; ++ks)
-          mma_bf16_ss(tmem + 256, smem_desc(P + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSw128),
+          mma_bf16_ss(tmem + ocol, smem_desc(P + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSw128),
                       smem_desc(stage + ks * 2048, 16384, 1024, kLayoutSw128), id_pv,
-                      (c > 0 || ks > 0) ? 1u : 0u);
+                      (c > 1 || ks > 0) ? 1u : 0u);
         mma_commit(st_empty + s);
         mma_commit(p_empty + pb);
         ++sc;
@@ -261,12 +273,13 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         if (!it.valid) break;
         const int qb = qc & 1;
         if (!mbar_wait(q_full + qb, (qc >> 1) & 1, abort_flag, status, kWaitCycles)) break;
-        for (int c = 0; c < it.nc && ok; ++c) qk(qb, c, chunk_width(it, c));
-        if (ok) qk(qb, 0, chunk_width(it, 0));
-        for (int c = 0; c < it.nc && ok; ++c) {
-          if (c + 1 < it.nc) qk(qb, c + 1, chunk_width(it, c + 1));
-          if (ok) pv(c, chunk_width(it, c));
+        // QK^T of chunk c runs ahead of the PV of chunk c - 1
+        qk(qb, 0, chunk_width(it, 0));
+        for (int c = 1; c < it.nc && ok; ++c) {
+          qk(qb, c, chunk_width(it, c));
+          if (ok) pv(c - 1, chunk_width(it, c - 1));
         }
+        if (ok) pv(it.nc - 1, chunk_width(it, it.nc - 1));
         if (!ok) break;
         mma_commit(o_full);
         mma_commit(q_empty + qb);
@@ -277,16 +290,18 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       volatile int never = 0;
       mbar_wait(fin, 0, &never, nullptr, kWaitCycles / 4);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax / epilogue
-    // Two warpgroups; warpgroup w handles the chunks c with c % 2 == w in both
-    // passes and columns [w D/2, (w+1) D/2) of the output rows.
-    const int w = (warp - 2) >> 2;
+    const int w = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;  // TMEM lane = tile row owned by this thread
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t o_col = 256 + w * D;  // this warpgroup's accumulator
     const float sl2 = a.geo.scale_log2;
     const int Hq = a.geo.Hq, lgG = a.geo.lg_G, wlen = a.geo.w;
+    const int tpt = a.geo.tpt;
     int s_use = 0, p_use = 0, oc = 0;
     auto both_bar = [&]() { asm volatile("bar.sync 3, 256;" ::: "memory"); };
     for (int k = blockIdx.x;; k += gridDim.x) {
@@ -297,137 +312,138 @@ __global__ void __launch_bounds__(kWinThreads, 1)
       const bool row_ok = i_row < it.ntok;
       // window keys of this row as offsets from the tile's first chunk key
       const int o_lo = max(t_row - wlen + 1, 0) - it.ws, o_hi = t_row - it.ws;
+      // offsets seen by every row of the tile (tile-uniform)
+      const int all_lo = max(it.t0 + tpt - 1 - wlen + 1, 0) - it.ws, all_hi = it.t0 - it.ws;
       const size_t orow = ((size_t)(it.row0 + i_row) * Hq + it.g * G + h_row);
-      // ---- pass 1: row maximum over this warpgroup's chunks (scaled, log2 units)
-      float m = -INFINITY;
+      float m_run = -INFINITY;  // running maximum of s * scale * log2(e)
+      float l_run = 0.f;        // sum of exp2(s * scale * log2(e) - m_run)
       for (int c = w; c < it.nc; c += 2) {
         mbar_wait(s_full + w, s_use & 1, abort_flag, status, kWaitCycles);
         tc_fence_after();
-        const int lo = o_lo - c * kChunk, hi = o_hi - c * kChunk;
-        // 16-column groups holding keys, and 64-column halves holding them
-        // (tile-uniform: the TMEM loads below are warp-wide)
-        const int ngc = chunk_width(it, c) >> 4;
-        auto chunk_max = [&](auto full_tag) {
-          constexpr bool kFull = decltype(full_tag)::value;
-          const int ng = kFull ? 8 : ngc, nh = kFull ? 2 : (ngc + 3) >> 2;
+        const int cw = chunk_width(it, c);
+        const int ngc = cw >> 4;  // 16-column groups holding keys (tile-uniform)
+        const bool full = it.ntok == tpt && cw == kChunk && all_lo <= c * kChunk &&
+                          all_hi >= c * kChunk + kChunk - 1;
+        float v[128];
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            if (!kFull && half >= nh) break;
-            float x[64];
+        for (int g16 = 0; g16 < 8; ++g16) {
+          float u16[16];
+          if (g16 < ngc) {
+            tmem_ld16(lane_addr + w * 128 + g16 * 16, u16);
+          } else {
 #pragma unroll
-            for (int g4 = 0; g4 < 4; ++g4) {
-              float v[16];
-              if (kFull || half * 4 + g4 < ng) {
-                tmem_ld16(lane_addr + w * 128 + half * 64 + g4 * 16, v);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = 0.f;  // past the span: masked below
-              }
-#pragma unroll
-              for (int j = 0; j < 16; ++j) x[g4 * 16 + j] = v[j];
-            }
-            tmem_ld_wait();
-            if (half == nh - 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(s_empty + w);
-            }
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-              const int o = half * 64 + j;
-              if (row_ok && o >= lo && o <= hi) m = fmaxf(m, x[j]);
-            }
+            for (int j = 0; j < 16; ++j) u16[j] = 0.f;  // past the chunk: masked below
           }
-        };
-        if (ngc == 8) chunk_max(std::true_type{});
-        else chunk_max(std::false_type{});
-        ++s_use;
-      }
-      m *= sl2;
-      // merge the two warpgroups' row maxima
-      if (w == 1) m1_s[r] = m;
-      both_bar();  // every thread is also done with the previous tile's m_s / l_s / l1_s
-      if (w == 0) m_s[r] = fmaxf(m, m1_s[r]);
-      both_bar();
-      const float mrow = m_s[r];
-      float lsum = 0.f;  // this warpgroup's part of the row sum
-      // ---- pass 2: P = exp2(s - max) into this warpgroup's P buffer (row r)
-      for (int c = w; c < it.nc; c += 2) {
-        mbar_wait(s_full + w, s_use & 1, abort_flag, status, kWaitCycles);
-        tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[g16 * 16 + j] = u16[j];
+        }
+        tmem_ld_wait();
+        // the scores are in registers: the buffer can take the next chunk
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_empty + w);
+        float cm = -INFINITY;
+        if (full) {
+#pragma unroll
+          for (int j = 0; j < 128; ++j) cm = fmaxf(cm, v[j]);
+        } else {
+          const int lo = o_lo - c * kChunk, hi = o_hi - c * kChunk;
+#pragma unroll
+          for (int j = 0; j < 128; ++j) {
+            v[j] = (row_ok && j >= lo && j <= hi) ? v[j] : -INFINITY;
+            cm = fmaxf(cm, v[j]);
+          }
+        }
+        cm *= sl2;
+        // P buffer free, and the previous PV into this warpgroup's O done
         if (p_use > 0) mbar_wait(p_empty + w, (p_use - 1) & 1, abort_flag, status, kWaitCycles);
-        const int lo = o_lo - c * kChunk, hi = o_hi - c * kChunk;
-        const uint32_t prow = sbase + L::kP + w * L::kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
-        const int ngc = chunk_width(it, c) >> 4;
-        auto chunk_p = [&](auto full_tag) {
-          constexpr bool kFull = decltype(full_tag)::value;
-          const int ng = kFull ? 8 : ngc, nh = kFull ? 2 : (ngc + 3) >> 2;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            if (!kFull && half >= nh) break;
-            float v[64];
-#pragma unroll
-            for (int g4 = 0; g4 < 4; ++g4) {
-              float u16[16];
-              if (kFull || half * 4 + g4 < ng) {
-                tmem_ld16(lane_addr + w * 128 + half * 64 + g4 * 16, u16);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) u16[j] = 0.f;
-              }
-#pragma unroll
-              for (int j = 0; j < 16; ++j) v[g4 * 16 + j] = u16[j];
-            }
+        // the maximum grew by more than 2^8: rescale the sum and O.  The TMEM
+        // pass is warp-collective (.sync.aligned), so the whole warp takes it
+        // when any of its rows needs it; the other rows scale by 1.
+        const bool grow = cm > m_run + 8.f;
+        const bool rescale = grow && m_run != -INFINITY;
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float f = rescale ? ex2(m_run - cm) : 1.f;
+          l_run *= f;
+          tc_fence_after();
+          // 16 columns at a time (the chunk's scores stay in registers)
+          for (int g16 = 0; g16 < D / 16; ++g16) {
+            float u16[16];
+            tmem_ld16(lane_addr + o_col + g16 * 16, u16);
             tmem_ld_wait();
 #pragma unroll
-            for (int g8 = 0; g8 < 8; ++g8) {  // 8 keys per 16-byte chunk of the row
-              if (!kFull && half * 8 + g8 >= 2 * ng) break;  // columns the PV does not read
-              uint32_t pk[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int o0 = half * 64 + g8 * 8 + 2 * j;
-                const float p0 = (row_ok && o0 >= lo && o0 <= hi) ? ex2(v[g8 * 8 + 2 * j] * sl2 - mrow) : 0.f;
-                const float p1 = (row_ok && o0 + 1 >= lo && o0 + 1 <= hi)
-                                     ? ex2(v[g8 * 8 + 2 * j + 1] * sl2 - mrow)
-                                     : 0.f;
-                lsum += p0 + p1;
-                pk[j] = pack_bf16x2(p0, p1);
-              }
-              st_shared_v4(prow + half * 16384 + ((g8 ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3]);
-            }
+            for (int j = 0; j < 16; ++j) u16[j] *= f;
+            tmem_st16(lane_addr + o_col + g16 * 16, u16);
           }
-        };
-        if (ngc == 8) chunk_p(std::true_type{});
-        else chunk_p(std::false_type{});
+          tmem_st_wait();
+        }
+        if (grow) m_run = cm;
+        // P = exp2(s * sl2 - m_run): masked keys hold -inf and give 0 (and
+        // when m_run is still -inf every key of the row is masked)
+        const float nm = m_run == -INFINITY ? 0.f : -m_run;
+        const uint32_t prow = sbase + L::kP + w * L::kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int g8 = 0; g8 < 16; ++g8) {  // 8 keys per 16-byte chunk of the row
+          if (g8 >= 2 * ngc) break;        // columns the PV does not read
+          uint32_t pk[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float p0 = ex2(fmaf(v[g8 * 8 + 2 * j], sl2, nm));
+            const float p1 = ex2(fmaf(v[g8 * 8 + 2 * j + 1], sl2, nm));
+            l_run += p0 + p1;
+            pk[j] = pack_bf16x2(p0, p1);
+          }
+          st_shared_v4(prow + (g8 >> 3) * 16384 + (((g8 & 7) ^ (r & 7)) << 4), pk[0], pk[1], pk[2],
+                       pk[3]);
+        }
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(s_empty + w);
-          mbar_arrive(p_full + w);
-        }
+        if (lane == 0) mbar_arrive(p_full + w);
         ++s_use;
         ++p_use;
       }
-      // ---- epilogue: this warpgroup's half of the row, g_win * O / sum
-      (w == 0 ? l_s : l1_s)[r] = lsum;
+      // ---- epilogue: merge the two warpgroups' (m, sum, O) of each row and
+      // store this warpgroup's half of g_win * O / sum
+      m_s[w * 128 + r] = m_run;
+      l_s[w * 128 + r] = l_run;
       both_bar();
-      const float ls = l_s[r] + l1_s[r];
+      const float m0 = m_s[r], m1 = m_s[128 + r], l0 = l_s[r], l1 = l_s[128 + r];
+      both_bar();  // both have read: the arrays may be rewritten by the next tile
+      const float mm = fmaxf(m0, m1);
+      const float f0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+      const float f1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
+      const float ls = l0 * f0 + l1 * f1;
+      const bool has1 = it.nc > 1;  // warpgroup 1's accumulator was written this tile
       mbar_wait(o_full, oc & 1, abort_flag, status, kWaitCycles);
       tc_fence_after();
       const float gw = row_ok ? __ldg(a.gates + orow * 3 + 2) : 0.f;
       const float scale = ls > 0.f ? gw / ls : 0.f;
+      const float s0 = f0 * scale, s1 = f1 * scale;
 #pragma unroll
       for (int grp = 0; grp < D / 32; ++grp) {
-        float v[16];
-        tmem_ld16(lane_addr + 256 + w * (D / 2) + grp * 16, v);
+        const uint32_t col = w * (D / 2) + grp * 16;
+        float x0[16], x1[16];
+        tmem_ld16(lane_addr + 256 + col, x0);
+        if (has1) {
+          tmem_ld16(lane_addr + 256 + D + col, x1);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x1[j] = 0.f;
+        }
         tmem_ld_wait();
         if (row_ok && !*abort_flag) {
-          float4* o = reinterpret_cast<float4*>(a.o_win + orow * D + w * (D / 2) + grp * 16);
+          float4* o = reinterpret_cast<float4*>(a.o_win + orow * D + col);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            o[j] = make_float4(v[4 * j] * scale, v[4 * j + 1] * scale, v[4 * j + 2] * scale,
-                               v[4 * j + 3] * scale);
+          for (int j = 0; j < 4; ++j) {
+            float e[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float y1 = has1 ? x1[4 * j + q] * s1 : 0.f;
+              e[q] = x0[4 * j + q] * s0 + y1;
+            }
+            o[j] = make_float4(e[0], e[1], e[2], e[3]);
+          }
         }
       }
       tc_fence_before();
@@ -457,6 +473,18 @@ cudaError_t launch_win_t(const PrefillArgs& a, const PrefillMaps& m, int num_sms
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
+  // the warpgroups' setmaxnreg shares add up to the launch allocation only
+  // when the kernel is launched with 168 registers a thread: any other count
+  // would leave setmaxnreg.inc waiting, so refuse to launch
+  static int regs[64] = {};
+  if (dev < 64 && regs[dev] == 0) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, nsa_win_kernel<D>);
+    if (e != cudaSuccess) return e;
+    regs[dev] = fa.numRegs;
+  }
+  if (dev < 64 && regs[dev] * (kWinThreads / 128) != kRegsControl + 2 * kRegsSoftmax)
+    return cudaErrorInvalidConfiguration;
   const int grid = num_sms < kMaxPersistentCtas ? num_sms : kMaxPersistentCtas;
   nsa_win_kernel<D><<<grid, kWinThreads, L::kSmem, s>>>(a, m);
   return cudaGetLastError();

@@ -45,7 +45,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool is_pow2_le16(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
 
 struct PrefillLayout {
-  size_t meta, o_cmp, lse, scores, sel, o_win, total;
+  size_t meta, o_cmp, lse, scores, sel_scores, sel, o_win, total;
 };
 
 PrefillLayout prefill_layout(const nsa_plan_s* pl) {
@@ -64,8 +64,43 @@ PrefillLayout prefill_layout(const nsa_plan_s* pl) {
   L.o_cmp = take(T * g.Hq * g.D * sizeof(float));
   L.lse = take(T * g.Hq * sizeof(float));
   L.scores = take(T * g.Hkv * (size_t)g.cmp_cap * sizeof(float));
+  L.sel_scores = take(g.remap ? T * g.Hkv * (size_t)g.sel_cap * sizeof(float) : 0);
   L.sel = take(T * g.Hkv * (size_t)g.n * sizeof(int));
   L.o_win = take(T * g.Hq * g.D * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+struct DecodeLayout {
+  size_t counters, sel, pt, win, cmp, slc, total;
+  int ncc_max, ncv_max, nsl;
+};
+
+// Decode workspace for `batch` sequences in a cache of `cap` tokens:
+// status header, per-pair unit counters, selection, compressed P^T and the
+// fp32 partial records of the second decode kernel.
+DecodeLayout decode_layout(const nsa_plan_s* pl, int batch, int cap) {
+  const Geometry& g = pl->geo;
+  DecodeLayout L{};
+  const size_t pairs = (size_t)batch * g.Hkv;
+  const int ccap = cap / g.d;
+  L.ncc_max = (ccap + kChunk - 1) / kChunk;
+  L.ncv_max = (L.ncc_max + 1) / 2;
+  const int nsc = (g.n + (kChunk >> g.lg_ls) - 1) / (kChunk >> g.lg_ls);
+  L.nsl = (nsc + 1) / 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  take(kHeaderBytes);
+  L.counters = take(pairs * sizeof(int));
+  L.sel = take(pairs * g.n * sizeof(int));
+  L.pt = take(pairs * (size_t)L.ncc_max * 4096);
+  L.win = take(pairs * g.G * g.D * sizeof(float));
+  L.cmp = take(pairs * (size_t)L.ncv_max * g.G * g.D * sizeof(float));
+  L.slc = take(pairs * (size_t)L.nsl * (g.G * g.D + 32) * sizeof(float));
   L.total = off;
   return L;
 }
@@ -202,15 +237,19 @@ int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out) {
       (p.out_dtype != NSA_OUT_BF16 && p.out_dtype != NSA_OUT_F32))
     return NSA_ERR_INVALID_ARG;
   if (p.num_q_heads % p.num_kv_heads != 0) return NSA_ERR_INVALID_ARG;
-  if (p.cmp_stride > p.cmp_block) return NSA_ERR_INVALID_ARG;
+  if (p.cmp_stride > p.cmp_block || p.cmp_block % p.cmp_stride != 0) return NSA_ERR_INVALID_ARG;
   const int G = p.num_q_heads / p.num_kv_heads;
   if (p.head_dim != 64 && p.head_dim != 128) return NSA_ERR_UNSUPPORTED;
   if (!is_pow2_le16(G)) return NSA_ERR_UNSUPPORTED;
-  if (p.cmp_block != p.cmp_stride || p.sel_block != p.cmp_block) return NSA_ERR_UNSUPPORTED;
+  // compression blocks of 32 or 64 tokens at a stride of 16, 32 or 64 that
+  // divides them; selection blocks of 32 or 64 tokens
   if (p.cmp_block != 32 && p.cmp_block != 64) return NSA_ERR_UNSUPPORTED;
-  // the selected branch keeps all of one token's selected keys in TMEM:
-  // at most 8 chunks of 128 keys
-  if (p.top_n > 8 * (kChunk / p.sel_block)) return NSA_ERR_UNSUPPORTED;
+  if (p.cmp_stride != 16 && p.cmp_stride != 32 && p.cmp_stride != 64) return NSA_ERR_UNSUPPORTED;
+  if (p.sel_block != 32 && p.sel_block != 64) return NSA_ERR_UNSUPPORTED;
+  // the selected branch keeps all of one token's selected keys in TMEM (at
+  // most 8 chunks of 128 keys) and deals the selection to the 32 lanes of a
+  // warp
+  if (p.top_n > 8 * (kChunk / p.sel_block) || p.top_n > 32) return NSA_ERR_UNSUPPORTED;
   if (p.max_seqlen < p.cmp_block) return NSA_ERR_INVALID_ARG;
   nsa_plan_s* pl = new (std::nothrow) nsa_plan_s;
   if (!pl) return NSA_ERR_INVALID_ARG;
@@ -223,10 +262,14 @@ int nsa_plan_create(const nsa_params* params, nsa_plan_t* plan_out) {
   g.lg_G = __builtin_ctz(G);
   g.tpt = kTileRows / G;
   g.l = p.cmp_block;
-  g.lg_l = __builtin_ctz(p.cmp_block);
+  g.d = p.cmp_stride;
+  g.ls = p.sel_block;
+  g.lg_ls = __builtin_ctz(p.sel_block);
+  g.remap = !(g.d == g.l && g.ls == g.l);
   g.n = p.top_n;
   g.w = p.window;
-  g.cmp_cap = p.max_seqlen / p.cmp_block;
+  g.cmp_cap = num_cmp_blocks(p.max_seqlen, g.l, g.d);
+  g.sel_cap = p.max_seqlen / g.ls + 1;
   g.max_seqlen = p.max_seqlen;
   g.scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / std::sqrt((float)p.head_dim);
   g.scale_log2 = g.scale * 1.4426950408889634f;
@@ -244,7 +287,11 @@ void nsa_plan_destroy(nsa_plan_t plan) { delete plan; }
 size_t nsa_workspace_size(nsa_plan_t plan, int mode) {
   if (!plan) return 0;
   if (mode == NSA_MODE_PREFILL) return prefill_layout(plan).total;
-  if (mode == NSA_MODE_DECODE) return kHeaderBytes;
+  if (mode == NSA_MODE_DECODE) {
+    const int unit = plan->geo.l > plan->geo.ls ? plan->geo.l : plan->geo.ls;
+    const int cap = plan->p.max_seqlen / unit * unit;
+    return decode_layout(plan, plan->p.max_batch, cap).total;
+  }
   return 0;
 }
 
@@ -258,6 +305,10 @@ int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, 
     case NSA_WS_O_CMP: *offset = L.o_cmp; *bytes = T * g.Hq * g.D * sizeof(float); break;
     case NSA_WS_LSE: *offset = L.lse; *bytes = T * g.Hq * sizeof(float); break;
     case NSA_WS_SCORES: *offset = L.scores; *bytes = T * g.Hkv * (size_t)g.cmp_cap * sizeof(float); break;
+    case NSA_WS_SEL_SCORES:
+      *offset = L.sel_scores;
+      *bytes = g.remap ? T * g.Hkv * (size_t)g.sel_cap * sizeof(float) : 0;
+      break;
     case NSA_WS_SEL: *offset = L.sel; *bytes = T * g.Hkv * (size_t)g.n * sizeof(int); break;
     case NSA_WS_WIN: *offset = L.o_win; *bytes = T * g.Hq * g.D * sizeof(float); break;
     default: return NSA_ERR_INVALID_ARG;
@@ -267,7 +318,8 @@ int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, 
 
 int nsa_cmp_rows(nsa_plan_t plan, int total_tokens) {
   if (!plan || total_tokens < 0) return -1;
-  return total_tokens / plan->geo.l;
+  // sum_b ((T_b - l) / d + 1) <= T_total / d for l >= d
+  return total_tokens / plan->geo.d;
 }
 
 int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, const float* gates,
@@ -285,7 +337,7 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   const PrefillLayout L = prefill_layout(plan);
   if (workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return NSA_ERR_WORKSPACE;
-  const int cmp_rows = total_tokens / geo.l;
+  const int cmp_rows = total_tokens / geo.d;
   if (total_tokens > 0) {
     if (!q || !k || !v || !gates || !w_k || !w_v || !out) return NSA_ERR_INVALID_ARG;
     if (cmp_rows > 0 && (!k_cmp || !v_cmp)) return NSA_ERR_INVALID_ARG;
@@ -320,6 +372,7 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   a.o_cmp = reinterpret_cast<float*>(ws + L.o_cmp);
   a.lse = reinterpret_cast<float*>(ws + L.lse);
   a.scores = reinterpret_cast<float*>(ws + L.scores);
+  a.sel_scores = reinterpret_cast<float*>(ws + L.sel_scores);
   a.sel = sel_idx ? sel_idx : reinterpret_cast<int*>(ws + L.sel);
   a.o_win = reinterpret_cast<float*>(ws + L.o_win);
 
@@ -334,17 +387,17 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
             encode3d(&m.q_tok, q, geo.D, geo.Hq, total_tokens, geo.Hq < 16 ? geo.Hq : 16, 1) &&
             encode3d(&m.kc, k_cmp, geo.D, geo.Hkv, cmp_rows, 1, kChunk) &&
             encode3d(&m.vc, v_cmp, geo.D, geo.Hkv, cmp_rows, 1, kChunk) &&
-            encode3d(&m.k_blk, k, geo.D, geo.Hkv, total_tokens, 1, geo.l) &&
-            encode3d(&m.v_blk, v, geo.D, geo.Hkv, total_tokens, 1, geo.l) &&
+            encode3d(&m.k_blk, k, geo.D, geo.Hkv, total_tokens, 1, geo.ls) &&
+            encode3d(&m.v_blk, v, geo.D, geo.Hkv, total_tokens, 1, geo.ls) &&
             encode3d(&m.k_win, k, geo.D, geo.Hkv, total_tokens, 1, kChunk) &&
             encode3d(&m.v_win, v, geo.D, geo.Hkv, total_tokens, 1, kChunk);
   if (!ok) return NSA_ERR_CUDA;
   // one-copy query rows (16 heads) and one-copy V blocks (64 keys), when the
   // driver accepts the channel-split maps
   a.split_q = geo.Hq >= 16 && encode_split4d(&m.q_split, q, geo.D, geo.Hq, total_tokens, false, 16);
-  a.split_v = geo.l == 64 && encode_split4d(&m.v_split, v, geo.D, geo.Hkv, total_tokens, true, 64);
+  a.split_v = geo.ls == 64 && encode_split4d(&m.v_split, v, geo.D, geo.Hkv, total_tokens, true, 64);
   static std::once_flag split_note;
-  if ((geo.Hq >= 16 && !a.split_q) || (geo.l == 64 && !a.split_v))
+  if ((geo.Hq >= 16 && !a.split_q) || (geo.ls == 64 && !a.split_v))
     std::call_once(split_note, [] {
       fprintf(stderr, "nsa_prefill: channel-split tensor maps rejected by the driver; "
                       "using one copy per 64-channel half\n");
@@ -379,13 +432,16 @@ int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* 
   const nsa_params& p = plan->p;
   const Geometry& geo = plan->geo;
   if (batch <= 0 || batch > p.max_batch || cache_capacity <= 0 ||
-      cache_capacity > p.max_seqlen || cache_capacity % geo.l != 0)
+      cache_capacity > p.max_seqlen || cache_capacity % geo.l != 0 ||
+      cache_capacity % geo.ls != 0)
     return NSA_ERR_INVALID_ARG;
-  // all of one query's compressed scores, window and selected keys stay in
-  // TMEM: at most 1024 compressed blocks, 8 window chunks of 128 keys
-  if (cache_capacity / geo.l > kDecodeMaxCmp + 1 || geo.w > 8 * kChunk) return NSA_ERR_UNSUPPORTED;
+  // all of one query's compressed scores and window keys stay in TMEM: at
+  // most 4096 compressed blocks, 8 window chunks of 128 keys
+  if (num_cmp_blocks(cache_capacity, geo.l, geo.d) > kDecodeMaxCmp || geo.w > 8 * kChunk)
+    return NSA_ERR_UNSUPPORTED;
   if (!workspace) return NSA_ERR_WORKSPACE;
-  if (workspace_bytes < kHeaderBytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  const DecodeLayout DL = decode_layout(plan, batch, cache_capacity);
+  if (workspace_bytes < DL.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return NSA_ERR_WORKSPACE;
   if (!q || !k_cache || !v_cache || !k_cmp_cache || !v_cmp_cache || !seqlens || !gates || !w_k ||
       !w_v || !out)
@@ -400,7 +456,7 @@ int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* 
   a.geo = geo;
   a.batch = batch;
   a.cap = cache_capacity;
-  a.ccap = cache_capacity / geo.l;
+  a.ccap = cache_capacity / geo.d;
   a.q = static_cast<const uint16_t*>(q);
   a.k_cache = static_cast<const uint16_t*>(k_cache);
   a.v_cache = static_cast<const uint16_t*>(v_cache);
@@ -412,30 +468,46 @@ int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* 
   a.w_v = w_v;
   a.out = out;
   a.sel = sel_idx;
-  a.status = static_cast<int*>(workspace);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.status = reinterpret_cast<int*>(ws);
+  a.ncc_max = DL.ncc_max;
+  a.ncv_max = DL.ncv_max;
+  a.nsl = DL.nsl;
+  a.counters = reinterpret_cast<int*>(ws + DL.counters);
+  a.ws_sel = reinterpret_cast<int*>(ws + DL.sel);
+  a.ws_pt = ws + DL.pt;
+  a.ws_win = reinterpret_cast<float*>(ws + DL.win);
+  a.ws_cmp = reinterpret_cast<float*>(ws + DL.cmp);
+  a.ws_slc = reinterpret_cast<float*>(ws + DL.slc);
   DecodeMaps m;
   bool ok = encode3d(&m.q, q, geo.D, geo.Hq, batch, geo.Hq < 16 ? geo.Hq : 16, 1) &&
             encode4d(&m.kc, k_cmp_cache, geo.D, geo.Hkv, a.ccap, batch, kChunk) &&
             encode4d(&m.vc, v_cmp_cache, geo.D, geo.Hkv, a.ccap, batch, kChunk) &&
-            encode4d(&m.k_blk, k_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.l) &&
-            encode4d(&m.v_blk, v_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.l) &&
+            encode4d(&m.k_blk, k_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.ls) &&
+            encode4d(&m.v_blk, v_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.ls) &&
             encode4d(&m.k_win, k_cache, geo.D, geo.Hkv, cache_capacity, batch, kChunk) &&
             encode4d(&m.v_win, v_cache, geo.D, geo.Hkv, cache_capacity, batch, kChunk);
   if (!ok) return NSA_ERR_CUDA;
-  if (cudaMemsetAsync(a.status, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
+  // status word and per-pair unit counters start at zero
+  if (cudaMemsetAsync(ws, 0, DL.counters + (size_t)batch * geo.Hkv * sizeof(int), s) != cudaSuccess)
+    return NSA_ERR_CUDA;
   prof_reset();
   prof_mark(s);
   cudaError_t e = launch_decode_compress(a, s);
   if (e == cudaSuccess) {
     prof_mark(s);
-    e = launch_decode(a, m, s);
+    e = launch_decode_a(a, m, s);
+  }
+  if (e == cudaSuccess) {
+    prof_mark(s);
+    e = launch_decode_b(a, m, s);
   }
   prof_mark(s);
   if (e != cudaSuccess) {
     fprintf(stderr, "nsa_decode: launch failed: %s\n", cudaGetErrorString(e));
     return NSA_ERR_CUDA;
   }
-  g_last_launches = 2;
+  g_last_launches = 3;
   return NSA_OK;
 }
 

@@ -24,11 +24,17 @@ struct Geometry {
   int G;        // Hq / Hkv
   int lg_G;     // log2(G)
   int tpt;      // tokens per dense tile = 128 / G
-  int l;        // block length (compress block == stride == select block)
-  int lg_l;     // log2(l)
+  int l;        // compression block length
+  int d;        // compression stride (d <= l, l % d == 0)
+  int ls;       // selection block length l'
+  int lg_ls;    // log2(l')
+  int remap;    // 1 unless l == d == l': selection scores are sums over the
+                // compressed blocks that overlap each selection block
   int n;        // top-n
   int w;        // window
-  int cmp_cap;  // row stride of the score table = max_seqlen / l
+  int cmp_cap;  // row stride of the score table: compressed blocks of the
+                // longest sequence, (max_seqlen - l) / d + 1
+  int sel_cap;  // row stride of the selection-score table, max_seqlen / l' + 1
   int max_seqlen;
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
@@ -68,19 +74,20 @@ struct PrefillArgs {
   float* o_cmp;   // [T, Hq, D]
   float* lse;     // [T, Hq]
   float* scores;  // [T, Hkv, cmp_cap]
+  float* sel_scores;  // [T, Hkv, sel_cap] selection-block scores (remap only)
   float* o_win;   // [T, Hq, D] g_win * O_win
   int split_q;    // PrefillMaps.q_split is valid (Hq >= 16)
-  int split_v;    // PrefillMaps.v_split is valid (l = 64)
+  int split_v;    // PrefillMaps.v_split is valid (l' = 64)
 };
 
 struct PrefillMaps {
   CUtensorMap q;      // (D, Hq, T) box (64, G, tpt)
   CUtensorMap q_tok;  // (D, Hq, T) box (64, min(16, Hq), 1)
   CUtensorMap q_split;  // (64, Hq, D/64, T) box (64, 16, D/64, 1): [half][head][64]
-  CUtensorMap v_split;  // (64, T, D/64, Hkv) box (64, l, D/64, 1): [half][key][64] (l = 64)
+  CUtensorMap v_split;  // (64, T, D/64, Hkv) box (64, l', D/64, 1): [half][key][64] (l' = 64)
   CUtensorMap kc;     // (D, Hkv, cmp_rows) box (64, 1, 128)
   CUtensorMap vc;
-  CUtensorMap k_blk;  // (D, Hkv, T) box (64, 1, l)
+  CUtensorMap k_blk;  // (D, Hkv, T) box (64, 1, l')
   CUtensorMap v_blk;
   CUtensorMap k_win;  // (D, Hkv, T) box (64, 1, 128)
   CUtensorMap v_win;
@@ -89,8 +96,8 @@ struct PrefillMaps {
 struct DecodeArgs {
   Geometry geo;
   int batch;
-  int cap;   // cache capacity in tokens (multiple of l)
-  int ccap;  // compressed-cache capacity = cap / l
+  int cap;   // cache capacity in tokens (multiple of l and of l')
+  int ccap;  // compressed-cache capacity = cap / d
   const uint16_t* q;        // [B, Hq, D]
   const uint16_t* k_cache;  // [B, cap, Hkv, D]
   const uint16_t* v_cache;
@@ -103,21 +110,54 @@ struct DecodeArgs {
   void* out;                // [B, Hq, D]
   int* sel;                 // [B, Hkv, n] or null
   int* status;
+  // units of the second decode kernel and its workspace records (per
+  // (sequence, group) pair: see nsa_decode_b_kernel)
+  int ncc_max;              // ceil(ccap / 128): compressed chunks of the longest sequence
+  int ncv_max;              // ceil(ncc_max / 2): compressed-value units per pair
+  int nsl;                  // ceil(selected chunks / 2): selected units per pair
+  int* counters;            // [B * Hkv] finished units per pair (zero at launch)
+  int* ws_sel;              // [B * Hkv, n]
+  uint8_t* ws_pt;           // [B * Hkv, ncc_max, 4096 B] normalised compressed P^T, bf16
+  float* ws_win;            // [B * Hkv, G, D]
+  float* ws_cmp;            // [B * Hkv, ncv_max, G, D]
+  float* ws_slc;            // [B * Hkv, nsl, G * D + 32]
 };
 
 struct DecodeMaps {
   CUtensorMap q;      // (D, Hq, B) box (64, 16, 1)
   CUtensorMap kc;     // (D, Hkv, ccap, B) box (64, 1, 128, 1)
   CUtensorMap vc;
-  CUtensorMap k_blk;  // (D, Hkv, cap, B) box (64, 1, l, 1)
+  CUtensorMap k_blk;  // (D, Hkv, cap, B) box (64, 1, l', 1)
   CUtensorMap v_blk;
   CUtensorMap k_win;  // (D, Hkv, cap, B) box (64, 1, 128, 1)
   CUtensorMap v_win;
 };
 
 // Largest number of compressed blocks one decode query may see (all of its
-// compressed scores stay in TMEM: 8 chunks of 128).
-constexpr int kDecodeMaxCmp = 1024;
+// compressed scores stay in TMEM: 32 chunks of 128 keys x 16 columns).
+constexpr int kDecodeMaxCmp = 4096;
+
+// Complete compressed blocks among the first `len` tokens of a sequence
+// (block i covers tokens [i d, i d + l - 1]).
+__host__ __device__ __forceinline__ int num_cmp_blocks(int len, int l, int d) {
+  return len >= l ? (len - l) / d + 1 : 0;
+}
+
+// Selection score of block j (tokens [j l', j l' + l' - 1]) from the group's
+// compressed-block scores S(i), i < ncmp: the sum over the visible
+// compressed blocks that overlap it, in increasing i.  With l == d == l' it
+// is S(j) itself (0 for the incomplete block).
+template <typename ScoreFn>
+__device__ __forceinline__ float remap_score(const Geometry& g, ScoreFn S, int ncmp, int j) {
+  // i d <= (j + 1) l' - 1  and  i d + l - 1 >= j l'
+  const int lo_num = j * g.ls - g.l + 1;
+  int i0 = lo_num <= 0 ? 0 : (lo_num + g.d - 1) / g.d;
+  int i1 = ((j + 1) * g.ls - 1) / g.d;
+  if (i1 > ncmp - 1) i1 = ncmp - 1;
+  float s = 0.f;
+  for (int i = i0; i <= i1; ++i) s += S(i);
+  return s;
+}
 
 // Sequence of token `tok` (binary search over cu[0..B]).
 __device__ __forceinline__ int seq_of_token(const int* cu, int B, int tok) {
@@ -148,6 +188,7 @@ cudaError_t launch_win(const PrefillArgs& a, const PrefillMaps& m, int num_sms, 
 cudaError_t launch_slc(const PrefillArgs& a, const PrefillMaps& m, int num_sms, cudaStream_t s);
 cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s);
 cudaError_t launch_decode_compress(const DecodeArgs& a, cudaStream_t s);
-cudaError_t launch_decode(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);
+cudaError_t launch_decode_a(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);
+cudaError_t launch_decode_b(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);
 
 }  // namespace nsa

@@ -30,9 +30,16 @@ __device__ __forceinline__ void warp_topn(ScoreFn score, int ncmp, int ncand, in
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = lane; i < 256; i += 32) hist[i] = 0;
     __syncwarp();
-    for (int j = lane; j < ncand; j += 32) {
-      const uint32_t x = bits(j);
-      if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+    // warp-aggregated counting: the lanes holding the same digit add their
+    // count with one atomic (scores of one row share their high bits, so
+    // per-lane atomics would serialise on a few bins)
+    for (int base = 0; base < ncand; base += 32) {
+      const int j = base + lane;
+      const uint32_t x = j < ncand ? bits(j) : 0u;
+      const bool in = j < ncand && (x & pmask) == prefix;
+      const uint32_t digit = in ? ((x >> shift) & 255u) : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (in && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], (unsigned)__popc(peers));
     }
     __syncwarp();
     unsigned c[8];

@@ -24,7 +24,7 @@ NSA_ERR_DEVICE_TIMEOUT = 6
 NSA_ERR_DEVICE_BAD_INPUT = 7
 OUT_BF16, OUT_F32 = 0, 1
 MODE_PREFILL, MODE_DECODE = 0, 1
-WS_STATUS, WS_O_CMP, WS_LSE, WS_SCORES, WS_SEL, WS_WIN = 0, 1, 2, 3, 4, 5
+WS_STATUS, WS_O_CMP, WS_LSE, WS_SCORES, WS_SEL, WS_WIN, WS_SEL_SCORES = 0, 1, 2, 3, 4, 5, 6
 
 EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_workspace_region",
             "nsa_cmp_rows", "nsa_prefill", "nsa_decode", "nsa_read_device_status",

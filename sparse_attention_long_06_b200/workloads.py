@@ -75,6 +75,11 @@ CONFIGS = {
     "decode_64k": NsaConfig("decode_64k", 4, 128, 64, 4, 64, 64, 64, 16, 512,
                             decode_batch=32, decode_len=65537),
     "varlen": NsaConfig("varlen", 5, 128, 64, 4, 64, 64, 64, 16, 512, varlen=True, planted=True),
+    # overlapping compression (blocks of 32 at a stride of 16) ranked over
+    # selection blocks of 64, on the 8k shape: the geometry the pages leave
+    # open (compression stride and selection block as separate knobs)
+    "prefill_8k_overlap": NsaConfig("prefill_8k_overlap", 6, 128, 64, 4, 32, 16, 64, 16, 512,
+                                    seqlens=(8192,)),
 }
 
 
@@ -209,9 +214,10 @@ def make_keys_periodic(cfg: NsaConfig, inputs: dict, period_blocks: int) -> dict
 
 
 def decode_sequence(cfg: NsaConfig, b: int, length: int, capacity: int) -> dict:
-    """One decode sequence: q [Hq,D], caches [capacity,Hkv,D] and compressed caches."""
+    """One decode sequence: q [Hq,D], caches [capacity,Hkv,D] and compressed
+    caches [capacity // d, Hkv, D]."""
     D, Hq, Hkv = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads
-    ccap = capacity // cfg.cmp_block
+    ccap = capacity // cfg.cmp_stride
     rng_q = _rng(cfg.seed, "q", b)
     q = bf16_bits(rng_q.standard_normal((Hq, D), dtype=np.float32))
     k = np.zeros((capacity, Hkv, D), dtype=np.uint16)
@@ -230,7 +236,8 @@ def decode_inputs(cfg: NsaConfig, lengths: list[int] | None = None, capacity: in
     B = cfg.decode_batch
     lens = list(lengths) if lengths is not None else [cfg.decode_len] * B
     cap = capacity if capacity is not None else max(lens)
-    cap = ((cap + cfg.cmp_block - 1) // cfg.cmp_block) * cfg.cmp_block
+    unit = max(cfg.cmp_block, cfg.sel_block)  # both are powers of two
+    cap = ((cap + unit - 1) // unit) * unit
     seqs = [decode_sequence(cfg, b, L, cap) for b, L in enumerate(lens)]
     wk, wv = compressor_weights(cfg)
     out = {key: np.stack([s[key] for s in seqs]) for key in ("q", "k", "v", "kc", "vc", "gates")}

@@ -31,7 +31,7 @@ def run_prefill(cfg, inputs, out_dtype=nsa.OUT_F32, max_seqlen=None, both_dtypes
     import torch
     lens = inputs["seqlens"]
     total = int(inputs["cu_seqlens"][-1])
-    max_seqlen = max_seqlen or max(max(lens), cfg.cmp_block)
+    max_seqlen = max_seqlen or max(max(lens), cfg.cmp_block, cfg.sel_block)
     D, Hq, Hkv, n = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads, cfg.top_n
     dev = {k: to_dev(inputs[k]) for k in ("q", "k", "v", "gates", "w_k", "w_v", "cu_seqlens")}
     res = {}
@@ -67,18 +67,33 @@ def run_prefill(cfg, inputs, out_dtype=nsa.OUT_F32, max_seqlen=None, both_dtypes
             count = int(np.prod(shape))
             return wsn[off:off + count * 4].view(dtype).reshape(shape).copy()
 
-        cap = max_seqlen // cfg.cmp_block
+        cap = num_cmp(cfg, max_seqlen)
         res["o_cmp"] = region(nsa.WS_O_CMP, np.float32, (total, Hq, D)).astype(np.float64)
         res["lse"] = region(nsa.WS_LSE, np.float32, (total, Hq)).astype(np.float64)
         res["scores"] = region(nsa.WS_SCORES, np.float32, (total, Hkv, cap))
+        if remaps(cfg):
+            res["sel_scores"] = region(nsa.WS_SEL_SCORES, np.float32,
+                                       (total, Hkv, max_seqlen // cfg.sel_block + 1))
+        res["o_win_g"] = region(nsa.WS_WIN, np.float32, (total, Hq, D)).astype(np.float64)
         res["cap"] = cap
         del ws
     return res
 
 
+def num_cmp(cfg, T):
+    """Complete compressed blocks of a sequence of T tokens (block l, stride d)."""
+    return 0 if T < cfg.cmp_block else (T - cfg.cmp_block) // cfg.cmp_stride + 1
+
+
+def remaps(cfg) -> bool:
+    """Whether selection scores are sums over overlapping compressed blocks
+    (any geometry other than l == d == l')."""
+    return not (cfg.cmp_stride == cfg.cmp_block == cfg.sel_block)
+
+
 def cmp_offsets(cfg, lens):
     off = np.zeros(len(lens) + 1, dtype=np.int64)
-    off[1:] = np.cumsum([T // cfg.cmp_block for T in lens])
+    off[1:] = np.cumsum([num_cmp(cfg, T) for T in lens])
     return off
 
 
@@ -127,7 +142,7 @@ def check_prefill(cfg, inputs, res, rows_per_seq, check_e2e=True):
         rows = rows_per_seq[b]
         if len(rows) == 0:
             continue
-        C = T // cfg.cmp_block
+        C = num_cmp(cfg, T)
         kc_gpu = res["kc"][coff[b]:coff[b] + C]
         vc_gpu = res["vc"][coff[b]:coff[b] + C]
         # step 1: compressed KV = bf16 rounding of an fp32 accumulation: within
@@ -136,7 +151,7 @@ def check_prefill(cfg, inputs, res, rows_per_seq, check_e2e=True):
             blocks = np.unique(np.concatenate([np.arange(min(C, 4)), np.arange(max(0, C - 4), C),
                                                np.linspace(0, C - 1, num=min(C, 24)).astype(int)]))
             for blk in blocks:
-                seg = slice(s + blk * cfg.cmp_block, s + (blk + 1) * cfg.cmp_block)
+                seg = slice(s + blk * cfg.cmp_stride, s + blk * cfg.cmp_stride + cfg.cmp_block)
                 kf, kb = oracle.compress(p, inputs["k"][seg], inputs["w_k"])
                 vf, vb = oracle.compress(p, inputs["v"][seg], inputs["w_v"])
                 for exact, ref, got in ((kf[0], kb[0], kc_gpu[blk]), (vf[0], vb[0], vc_gpu[blk])):
@@ -148,22 +163,35 @@ def check_prefill(cfg, inputs, res, rows_per_seq, check_e2e=True):
         # stage A: the oracle's selection replayed on the GPU's fp32 scores
         tg = s + rows
         ncand = rows // cfg.sel_block + 1
-        ncmp = (rows + 1) // cfg.cmp_block
+        ncmp = np.array([num_cmp(cfg, t + 1) for t in rows], dtype=np.int32)
         for g in range(cfg.num_kv_heads):
-            selA, _ = oracle.select_f32(res["scores"][tg, g, :], ncand, ncmp, cfg.top_n)
+            if remaps(cfg):  # the GPU's selection-block scores, every candidate defined
+                selA, _ = oracle.select_f32(res["sel_scores"][tg, g, :], ncand, ncand, cfg.top_n)
+            else:
+                selA, _ = oracle.select_f32(res["scores"][tg, g, :], ncand, ncmp, cfg.top_n)
             assert np.array_equal(selA, res["sel"][tg, g, :]), f"stage A selection, seq {b} group {g}"
         # stage B: oracle steps 2-7 on the GPU's compressed KV
         kcb = kc_gpu if C else np.zeros((1, cfg.num_kv_heads, cfg.head_dim), np.uint16)
         vcb = vc_gpu if C else np.zeros((1, cfg.num_kv_heads, cfg.head_dim), np.uint16)
+        jmax = T // cfg.sel_block + 1
         r = oracle.nsa_rows(p, inputs["q"][s:s + T], inputs["k"][s:s + T], inputs["v"][s:s + T],
-                            kcb, vcb, inputs["gates"][s:s + T], rows, cmax=max(C, 1))
+                            kcb, vcb, inputs["gates"][s:s + T], rows, cmax=max(C, jmax, 1))
         # compressed branch and scores (fp32 vs fp64)
         assert np.max(np.abs(res["o_cmp"][tg] - r["o_cmp"])) < 1e-2
+        # window branch times its gate (the window kernel's own output)
+        win_ref = r["o_win"] * inputs["gates"][tg][:, :, 2:3].astype(np.float64)
+        rep["win_max_abs"] = max(rep.get("win_max_abs", 0.0),
+                                 float(np.max(np.abs(res["o_win_g"][tg] - win_ref))))
+        assert rep["win_max_abs"] < 1e-2
         vis = ncmp > 0
         if np.any(vis):
             assert np.max(np.abs(res["lse"][tg][vis] - r["lse"][vis])) < 1e-4
         for ri, t in enumerate(rows):
-            nc = (t + 1) // cfg.cmp_block
+            if remaps(cfg):  # selection-block scores
+                nj = t // cfg.sel_block + 1
+                assert np.max(np.abs(res["sel_scores"][s + t, :, :nj] - r["scores"][ri, :, :nj])) < 1e-5
+                continue
+            nc = num_cmp(cfg, t + 1)
             if nc:
                 assert np.max(np.abs(res["scores"][s + t, :, :nc] - r["scores"][ri, :, :nc])) < 1e-5
         for g in range(cfg.num_kv_heads):
@@ -183,7 +211,7 @@ def check_prefill(cfg, inputs, res, rows_per_seq, check_e2e=True):
             _, vco = oracle.compress(p, inputs["v"][s:s + T], inputs["w_v"])
             r2 = oracle.nsa_rows(p, inputs["q"][s:s + T], inputs["k"][s:s + T],
                                  inputs["v"][s:s + T], kco, vco, inputs["gates"][s:s + T], rows,
-                                 cmax=C)
+                                 cmax=max(C, jmax))
             for g in range(cfg.num_kv_heads):
                 same = np.all(r2["sel"][:, g, :] == res["sel"][tg, g, :], axis=1)
                 rep["e2e_idx_mismatch"] += int(np.count_nonzero(~same & (r2["gap"][:, g] >= 1e-6)))

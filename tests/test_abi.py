@@ -56,8 +56,10 @@ def _params(**kw):
     (dict(cmp_stride=128), nsa.NSA_ERR_INVALID_ARG),       # stride longer than the block
     (dict(head_dim=96), nsa.NSA_ERR_UNSUPPORTED),
     (dict(num_q_heads=96, num_kv_heads=4), nsa.NSA_ERR_UNSUPPORTED),  # G = 24
-    (dict(cmp_stride=32), nsa.NSA_ERR_UNSUPPORTED),        # overlapping compression
+    (dict(cmp_stride=48), nsa.NSA_ERR_INVALID_ARG),        # stride that does not divide the block
+    (dict(cmp_stride=8), nsa.NSA_ERR_UNSUPPORTED),         # overlap of 7/8 of a block
     (dict(sel_block=128), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(sel_block=32, top_n=33), nsa.NSA_ERR_UNSUPPORTED),  # more than one warp of blocks
     (dict(top_n=17), nsa.NSA_ERR_UNSUPPORTED),             # > 8 chunks of 128 keys
     (dict(max_seqlen=16), nsa.NSA_ERR_INVALID_ARG),
 ])
@@ -65,6 +67,19 @@ def test_plan_validation(L, kw, code):
     with pytest.raises(nsa.NsaError) as e:
         nsa.Plan(**_params(**kw))
     assert e.value.code == code
+
+
+def test_general_geometry_plans(L):
+    # overlapping compression and selection blocks other than l are planned
+    p = nsa.Plan(**_params(cmp_block=32, cmp_stride=16, sel_block=64))
+    assert p.cmp_rows(65536) == 65536 // 16
+    off, nb = p.workspace_region(nsa.WS_SEL_SCORES)
+    assert nb == 65536 * 4 * (65536 // 64 + 1) * 4
+    off, nb = p.workspace_region(nsa.WS_SCORES)
+    assert nb == 65536 * 4 * ((65536 - 32) // 16 + 1) * 4
+    # with l == d == l' the selection scores are the compressed-block scores
+    q = nsa.Plan(**_params())
+    assert q.workspace_region(nsa.WS_SEL_SCORES)[1] == 0
 
 
 def test_plan_sizes(L):
@@ -119,8 +134,10 @@ def test_prefill_rejects_bad_arguments_before_launch(L):
 def test_decode_rejects_bad_arguments_before_launch(L):
     p = nsa.Plan(**_params(max_batch=4, max_seqlen=65536 + 64))
     fake = 1 << 20  # an aligned address that is never dereferenced
+    wsb = p.workspace_size(nsa.MODE_DECODE)
+    assert wsb > 256  # status, counters, selection and the partial results
     args = dict(q=fake, k=fake, v=fake, kc=fake, vc=fake, lens=fake, batch=2, cap=4096,
-                gates=fake, w_k=fake, w_v=fake, out=fake, sel=None, ws=fake, wsb=256)
+                gates=fake, w_k=fake, w_v=fake, out=fake, sel=None, ws=fake, wsb=wsb)
 
     def call(**over):
         a = dict(args)
@@ -135,6 +152,7 @@ def test_decode_rejects_bad_arguments_before_launch(L):
     assert call(cap=65536 + 128) == nsa.NSA_ERR_INVALID_ARG     # above the plan's max_seqlen
     assert call(ws=None) == nsa.NSA_ERR_WORKSPACE
     assert call(wsb=255) == nsa.NSA_ERR_WORKSPACE
+    assert call(cap=65536 + 64, batch=4, wsb=wsb - 1) == nsa.NSA_ERR_WORKSPACE
     assert call(q=None) == nsa.NSA_ERR_INVALID_ARG
     assert call(k=fake + 2) == nsa.NSA_ERR_MISALIGNED
     assert call(lens=fake + 2) == nsa.NSA_ERR_MISALIGNED

@@ -52,8 +52,9 @@ def _assert_report(rep, res=None, e2e=True, name="prefill"):
         assert rep["e2e_max_abs"] <= 1e-2
 
 
-def _custom(name, D, Hq, Hkv, l, n, w, lens, seed=21):
-    return wl.NsaConfig(name, seed, D, Hq, Hkv, l, l, l, n, w, seqlens=tuple(lens))
+def _custom(name, D, Hq, Hkv, l, n, w, lens, seed=21, d=None, ls=None):
+    return wl.NsaConfig(name, seed, D, Hq, Hkv, l, l if d is None else d, l if ls is None else ls,
+                        n, w, seqlens=tuple(lens))
 
 
 def test_tiny_config_all_rows():
@@ -85,6 +86,47 @@ def test_edge_geometries(case):
     rows = [np.arange(T, dtype=np.int32) for T in lens]
     rep = gu.check_prefill(cfg, inputs, res, rows)
     _assert_report(rep, name=f"edge{case}")
+
+
+@pytest.mark.parametrize("case", [
+    # D, Hq, Hkv, l, d, l', n, w, lengths
+    (128, 64, 4, 32, 16, 64, 16, 512, [3000, 700]),     # overlapping compression, l' = 2 l
+    (64, 8, 2, 64, 32, 64, 8, 256, [2500, 33]),         # overlapping, l' = l
+    (128, 16, 1, 64, 64, 32, 16, 300, [2000, 64, 31]),  # l = d, l' < l (G = 16)
+    (64, 4, 1, 32, 32, 64, 4, 128, [1500, 200]),        # l = d, l' = 2 l
+    (128, 32, 4, 64, 16, 32, 32, 1000, [1800]),         # stride l / 4, l' < l, n = 32
+])
+def test_general_geometry(case):
+    """Compression stride d and selection block l' independent of the
+    compression block l: compressed block i covers tokens [i d, i d + l - 1],
+    and each selection block's score sums the compressed blocks overlapping
+    it.  Stage A replays the oracle's selection on the GPU's selection-block
+    scores (bit for bit); stage B and the outputs as for l == d == l'."""
+    D, Hq, Hkv, l, d, ls, n, w, lens = case
+    cfg = _custom("geo", D, Hq, Hkv, l, n, w, lens, seed=41, d=d, ls=ls)
+    inputs = wl.prefill_inputs(cfg)
+    res = gu.run_prefill(cfg, inputs, out_dtype=nsa.OUT_F32)
+    assert res["status"] == nsa.NSA_OK
+    rows = [np.arange(T, dtype=np.int32) for T in lens]
+    rep = gu.check_prefill(cfg, inputs, res, rows)
+    _assert_report(rep, name=f"geometry{case}")
+
+
+def test_window_running_maximum_rescale():
+    """The keys of every 8th block are scaled by 4 (exact in bf16), so a row's
+    window logits jump by far more than 2^8 in log2 units when its window
+    reaches such a block after ordinary keys: the window kernel must rescale
+    the running sum and its TMEM accumulator (for some rows of a warp and not
+    others) and still match the oracle."""
+    cfg = _custom("rescale", 128, 64, 4, 64, 16, 512, [4096], seed=43)
+    inputs = wl.prefill_inputs(cfg)
+    k = wl.bf16_to_f32(inputs["k"]).reshape(-1, 64, 4, 128)
+    k[3::8] *= 4.0
+    inputs["k"] = wl.bf16_bits(k.reshape(4096, 4, 128))
+    res = gu.run_prefill(cfg, inputs, out_dtype=nsa.OUT_F32)
+    assert res["status"] == nsa.NSA_OK
+    rep = gu.check_prefill(cfg, inputs, res, [np.arange(4096, dtype=np.int32)])
+    _assert_report(rep, name="window_rescale")
 
 
 def test_prefill_8k_sampled_rows():
