@@ -11,21 +11,23 @@
 //              compressed block (len >= l, (len - l) % d == 0), that block
 //              is compressed from the cache (step 1) into the compressed
 //              cache;
-//   nsa_decode_a_kernel  two units per pair:
-//     scores   all compressed keys: S^T = Kc Q^T (keys on TMEM lanes, the
-//              group's heads on 16 columns), per-head log-sum-exp, the
-//              normalised probabilities P^T (bf16, to the workspace), the
-//              block scores (step 3: the sum over heads of p, summed over
-//              the compressed blocks overlapping each selection block when
-//              l, d and l' differ) and the top-n (step 4, one warp, to the
-//              workspace and sel_idx);
-//     window   the w tokens ending at t (step 6): O_win, normalised;
-//   nsa_decode_b_kernel  units of at most two 128-key chunks per pair:
+//   nsa_decode_a_kernel  one CTA per pair, the dependency the selected
+//              keys wait for: all compressed keys through a six-stage ring,
+//              S^T = Kc Q^T (keys on TMEM lanes, the group's heads on 16
+//              columns), per-head log-sum-exp, the normalised probabilities
+//              P^T (bf16, to the workspace), the block scores (step 3: the
+//              sum over heads of p, summed over the compressed blocks
+//              overlapping each selection block when l, d and l' differ)
+//              and the top-n (step 4, one warp, to the workspace and
+//              sel_idx);
+//   nsa_decode_b_kernel  units of at most four 128-key chunks per pair:
 //     cmp      O_cmp partial sums P Vc over a range of compressed blocks
-//              (step 2, with the probabilities of the scores unit);
+//              (step 2, with the probabilities of kernel A);
+//     window   a range of the w keys ending at t (step 6);
 //     selected a range of the selected blocks (step 5; the incomplete
-//              block holding t is loaded as the l' rows ending at t): a
-//              softmax partial (row max, sum, unnormalised O);
+//              block holding t is loaded as the l' rows ending at t);
+//              window and selected units leave a softmax partial (row
+//              maximum, sum, unnormalised O);
 //   the last unit of a pair to finish (an atomic counter per pair) merges
 //   the partials and applies the gates (step 7):
 //     out = g_cmp O_cmp + g_slc O_slc + g_win O_win.
@@ -88,10 +90,12 @@ __global__ void __launch_bounds__(256) nsa_decode_compress_kernel(DecodeArgs a) 
 
 // ------------------------------------------------------------------ shared pieces
 constexpr int kDecThreads = 192;
-// at most 16 compressed-value units (32 chunks of 128 blocks) and 8 selected
-// units (16 chunks: top_n <= 32 blocks of 32 or 16 of 64) per pair
-constexpr int kMaxCmpUnits = 16;
-constexpr int kMaxSlcUnits = 8;
+// at most 8 compressed-value units (32 chunks of 128 blocks) and 4 selected
+// units (16 chunks: top_n <= 32 blocks of 32 or 16 of 64) per pair, each of
+// up to kUnitChunks chunks
+constexpr int kMaxCmpUnits = (kDecodeMaxCmp / kChunk + kUnitChunks - 1) / kUnitChunks;
+constexpr int kMaxSlcUnits = (16 + kUnitChunks - 1) / kUnitChunks;
+constexpr int kMaxWinUnits = (8 + kUnitChunks - 1) / kUnitChunks;  // window <= 1024 keys
 constexpr int kPChunkBytes = 4096;  // P^T of one chunk: 128 keys x 16 heads, bf16
 
 // Per-(sequence, group) quantities of one decode query.
@@ -196,10 +200,11 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_col, uint32_t stage, uint
                 (accumulate || ks > 0) ? 1u : 0u);
 }
 
-// Workspace records of one pair (fp32): window output [G][D], compressed
-// partial sums [ncv][G][D], selected partials [nsl][G*D + 32] (O [G][D], then
-// the row maximum m[16] and the sum[16] per head; every record 16-byte
-// aligned).
+// Workspace records of one pair (fp32): compressed partial sums
+// [ncv][G][D]; window and selected partials [nwu or nsl][G*D + 32] (O
+// [G][D], then the row maximum m[16] and the sum[16] per head; every record
+// 16-byte aligned).
+constexpr int partial_floats(int G, int D) { return G * D + 32; }
 struct PairRecs {
   float* win;
   float* cmp;
@@ -211,9 +216,9 @@ struct PairRecs {
 __device__ __forceinline__ PairRecs pair_recs(const DecodeArgs& a, int pair) {
   const int G = a.geo.G, D = a.geo.D;
   PairRecs r;
-  r.win = a.ws_win + (size_t)pair * G * D;
+  r.win = a.ws_win + (size_t)pair * a.nwu * partial_floats(G, D);
   r.cmp = a.ws_cmp + (size_t)pair * a.ncv_max * G * D;
-  r.slc = a.ws_slc + (size_t)pair * a.nsl * (G * D + 32);
+  r.slc = a.ws_slc + (size_t)pair * a.nsl * partial_floats(G, D);
   r.pt = a.ws_pt + (size_t)pair * a.ncc_max * kPChunkBytes;
   r.sel = a.ws_sel + (size_t)pair * a.geo.n;
   return r;
@@ -229,23 +234,20 @@ constexpr int ring_pad() { return D == 64 ? 16384 : 0; }
 
 template <int D>
 struct DecALayout {
-  static constexpr int kStages = 2;
+  static constexpr int kStages = 6;
   static constexpr int kChunkBytes = kChunk * D * 2;
   static constexpr int kQ = 0;                                   // 16 x D bf16 (4 KB max)
   static constexpr int kRing = 4096;
-  static constexpr int kU = kRing + kStages * kChunkBytes + ring_pad<D>();  // P^T (window) | scores
-  static constexpr int kUBytes = 8 * kPChunkBytes > kDecodeMaxCmp * 4 ? 8 * kPChunkBytes
-                                                                     : kDecodeMaxCmp * 4;
-  static constexpr int kRed = kU + kUBytes;                      // float [2][64]
+  static constexpr int kU = kRing + kStages * kChunkBytes;       // scores [kDecodeMaxCmp]
+  static constexpr int kRed = kU + kDecodeMaxCmp * 4;            // float [2][64]
   static constexpr int kSel = kRed + 2 * 64 * 4;                 // int [64]
   static constexpr int kHist = kSel + 64 * 4;                    // unsigned [256]
   static constexpr int kCand = kHist + 256 * 4;                  // u64 [kTopnCand]
   static constexpr int kBars = kCand + kTopnCand * 8;
-  static constexpr int kEnd = kBars + 16 * 8;
+  static constexpr int kEnd = kBars + 24 * 8;
   static constexpr int kSmem = kEnd + 1024;  // manual 1024-byte alignment
-  static_assert(kU % 1024 == 0, "alignment");
-  // a PV operand spans 32 KB from the start of its stage
-  static_assert(kRing + (kStages - 1) * kChunkBytes + 32768 <= kEnd, "PV operand inside smem");
+  static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(kStages <= 6, "barrier arrays");
 };
 
 template <int D>
@@ -257,30 +259,24 @@ __global__ void __launch_bounds__(kDecThreads)
                                            ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
   uint64_t* q_full = bars + 0;
-  uint64_t* st_full = bars + 1;   // [2]
-  uint64_t* st_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* o_done = bars + 7;
-  uint64_t* fin = bars + 8;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* st_full = bars + 1;   // [kStages]
+  uint64_t* st_empty = bars + 7;  // [kStages]
+  uint64_t* s_full = bars + 13;
+  uint64_t* fin = bars + 14;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   float* red = reinterpret_cast<float*>(sm + L::kRed);
   unsigned* hist = reinterpret_cast<unsigned*>(sm + L::kHist);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + L::kCand);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // kernel B may be scheduled now: its CTAs wait for this grid's results
-  // (griddepcontrol.wait) and only take the SM slots this grid leaves free
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int pair = blockIdx.x >> 1;
-  const bool is_win = blockIdx.x & 1;
+  const int pair = blockIdx.x;
   const DecPair P = dec_pair(a, pair);
   if (!P.ok) {
     if (threadIdx.x == 0) atomicCAS(a.status, 0, kDeviceBadInputCode);
     return;
   }
-  const int nchunks = is_win ? P.nwc : P.ncc;
+  const int nchunks = P.ncc;
   const PairRecs rec = pair_recs(a, pair);
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -289,15 +285,12 @@ __global__ void __launch_bounds__(kDecThreads)
       mbar_init(st_empty + i, 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
-    mbar_init(o_done, 1);
     mbar_init(fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // TMEM: scores unit S^T of up to 32 chunks; window unit S^T of up to 8
-  // chunks and O^T (16 columns at 128)
-  const uint32_t ncols = is_win ? 256u : (nchunks <= 8 ? 128u : (nchunks <= 16 ? 256u : 512u));
+  // TMEM: S^T of up to 32 chunks (16 columns each)
+  const uint32_t ncols = nchunks <= 8 ? 128u : (nchunks <= 16 ? 256u : 512u);
   if (warp == 1) {
     tmem_alloc(tmem_slot, ncols);
     tmem_relinquish();
@@ -332,12 +325,7 @@ __global__ void __launch_bounds__(kDecThreads)
         for (int h = 0; h < D / 64; ++h) tma_load_4d(dst + h * 16384, map, st_full + s, h * 64, g, row0, b);
         ++sc;
       };
-      if (is_win) {
-        for (int c = 0; c < nchunks && ok; ++c) load_rows(&maps.k_win, P.win_row0 + c * kChunk);
-        for (int c = 0; c < nchunks && ok; ++c) load_rows(&maps.v_win, P.win_row0 + c * kChunk);
-      } else {
-        for (int c = 0; c < nchunks && ok; ++c) load_rows(&maps.kc, P.cmp_row0 + c * kChunk);
-      }
+      for (int c = 0; c < nchunks && ok; ++c) load_rows(&maps.kc, P.cmp_row0 + c * kChunk);
       volatile int never = 0;
       for (int s = 0; s < L::kStages && s < sc; ++s) {
         const int last = sc - 1 - ((sc - 1 - s) % L::kStages);
@@ -368,17 +356,6 @@ __global__ void __launch_bounds__(kDecThreads)
         ++sc;
       }
       mma_commit(s_full);
-      if (is_win && ok && mbar_wait(p_full, 0, abort_flag, status, kWaitCycles)) {
-        tc_fence_after();
-        for (int c = 0; c < nchunks && ok; ++c) {
-          const uint32_t st = wait_stage();
-          if (!ok) break;
-          issue_pv(tmem + 128, st, sbase + L::kU + c * kPChunkBytes, c > 0);
-          mma_commit(st_empty + (sc % L::kStages));
-          ++sc;
-        }
-      }
-      mma_commit(o_done);
       mma_commit(fin);
       volatile int never = 0;
       mbar_wait(fin, 0, &never, nullptr, kWaitCycles / 4);
@@ -390,13 +367,9 @@ __global__ void __launch_bounds__(kDecThreads)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const float sl2 = a.geo.scale_log2;
     const uint32_t colmask = (G >= 16) ? 0xFFFFu : ((1u << G) - 1u);
-    // keys of this lane that take part, one bit per chunk
+    // keys of this lane that take part (complete blocks), one bit per chunk
     uint32_t kok = 0;
-    for (int c = 0; c < nchunks; ++c) {
-      const int row = (is_win ? P.win_row0 : P.cmp_row0) + c * kChunk + r;
-      const bool on = is_win ? row >= max(0, t - a.geo.w + 1) : row >= 0;
-      kok |= on ? (1u << c) : 0u;
-    }
+    for (int c = 0; c < nchunks; ++c) kok |= (P.cmp_row0 + c * kChunk + r >= 0) ? (1u << c) : 0u;
     mbar_wait(s_full, 0, abort_flag, status, kWaitCycles);
     tc_fence_after();
     // sweep 1: per-head maximum (log2 units)
@@ -413,38 +386,7 @@ __global__ void __launch_bounds__(kDecThreads)
     float sm16[16];
 #pragma unroll
     for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
-    if (is_win) {
-      // sweep 2: unnormalised P^T into shared memory and the sums
-      uint8_t* pbase = sm + L::kU;
-      sweep_chunks<8>(lane_addr, 0, nchunks, [&](int c, const float(&v)[16]) {
-        const bool on = (kok >> c) & 1u;
-        float p[16];
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          p[h] = (on && ((colmask >> h) & 1u)) ? ex2(v[h] * sl2 - mx[h]) : 0.f;
-          sm16[h] += p[h];
-        }
-        store_pt(pbase + c * kPChunkBytes, r, p);
-      });
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-      reduce16_across_128<1>(sm16, red + 64, q4, lane, false);
-      // epilogue: O_win = O^T / sum, thread = channel
-      mbar_wait(o_done, 0, abort_flag, status, kWaitCycles);
-      tc_fence_after();
-      float o[16];
-      tmem_ld16(lane_addr + 128, o);
-      tmem_ld_wait();
-      if (r < D && !*abort_flag) {
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          if (h >= G) break;
-          rec.win[h * D + r] = sm16[h] > 0.f ? o[h] / sm16[h] : 0.f;
-        }
-      }
-    } else {
+    {
       // sweep 2: sums -> log2-sum-exp per head
       sweep_chunks<32>(lane_addr, 0, nchunks, [&](int c, const float(&v)[16]) {
         if ((kok >> c) & 1u) {
@@ -481,17 +423,16 @@ __global__ void __launch_bounds__(kDecThreads)
           if (live) rec.sel[i] = j;
           if (gsel && live) gsel[i] = j;
         };
-        // the register selection for up to 1024 candidates, else (or when
-        // too many keys tie at its bound) the radix select
-        const bool regs_ok = P.ncand <= 1024 && n <= 32;
+        // the bound-and-rank selection over the shared-memory scores, else
+        // (when too many keys tie at its bound) the radix select
         if (!a.geo.remap) {
           auto score = [&](int j) { return scores[j]; };
-          if (!(regs_ok && warp_topn_regs(score, P.C, P.ncand, n, cand, put)))
+          if (!warp_topn_reread(score, P.C, P.ncand, n, cand, put))
             warp_topn(score, P.C, P.ncand, n, hist, put);
         } else {
           const int C = P.C;
           auto score = [&](int j) { return remap_score(a.geo, [&](int i) { return scores[i]; }, C, j); };
-          if (!(regs_ok && warp_topn_regs(score, P.ncand, P.ncand, n, cand, put)))
+          if (!warp_topn_reread(score, P.ncand, P.ncand, n, cand, put))
             warp_topn(score, P.ncand, P.ncand, n, hist, put);
         }
       }
@@ -508,12 +449,12 @@ __global__ void __launch_bounds__(kDecThreads)
 // ------------------------------------------------------------------ kernel B
 template <int D>
 struct DecBLayout {
-  static constexpr int kStages = 3;
+  static constexpr int kStages = 2;
   static constexpr int kChunkBytes = kChunk * D * 2;
   static constexpr int kQ = 0;
   static constexpr int kRing = 4096;
   static constexpr int kP = kRing + kStages * kChunkBytes + ring_pad<D>();  // 2 chunks of P^T
-  static constexpr int kRed = kP + 2 * kPChunkBytes;        // float [2][64]
+  static constexpr int kRed = kP + kUnitChunks * kPChunkBytes;  // float [2][64]
   static constexpr int kSel = kRed + 2 * 64 * 4;            // int [64]
   static constexpr int kFlag = kSel + 64 * 4;               // int
   static constexpr int kBars = kFlag + 16;
@@ -521,6 +462,8 @@ struct DecBLayout {
   static constexpr int kSmem = kEnd + 1024;
   // a PV operand spans 32 KB from the start of its stage
   static_assert(kRing + (kStages - 1) * kChunkBytes + 32768 <= kEnd, "PV operand inside smem");
+  // two CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA)
+  static_assert(2 * (kSmem + 1024) <= 233472, "two CTAs per SM");
 };
 
 template <int D>
@@ -546,15 +489,18 @@ __global__ void __launch_bounds__(kDecThreads)
   int* last_flag = reinterpret_cast<int*>(sm + L::kFlag);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int units = a.ncv_max + a.nsl;
+  const int units = a.ncv_max + a.nwu + a.nsl;
   const int pair = blockIdx.x / units, unit = blockIdx.x % units;
   const DecPair P = dec_pair(a, pair);
   if (!P.ok) return;  // kernel A has recorded the bad length
+  // unit kinds: compressed values, window, selected blocks
   const bool is_cmp = unit < a.ncv_max;
-  const int u = is_cmp ? unit : unit - a.ncv_max;
-  // chunks [c_lo, c_hi) of the compressed blocks or of the selected keys
-  const int total_chunks = is_cmp ? P.ncc : P.nsc;
-  const int c_lo = min(2 * u, total_chunks), c_hi = min(2 * u + 2, total_chunks);
+  const bool is_win = !is_cmp && unit < a.ncv_max + a.nwu;
+  const int u = is_cmp ? unit : (is_win ? unit - a.ncv_max : unit - a.ncv_max - a.nwu);
+  // chunks [c_lo, c_hi) of the compressed blocks, the window or the selected keys
+  const int total_chunks = is_cmp ? P.ncc : (is_win ? P.nwc : P.nsc);
+  const int c_lo = min(kUnitChunks * u, total_chunks);
+  const int c_hi = min(kUnitChunks * u + kUnitChunks, total_chunks);
   const int nch = c_hi - c_lo;
   const PairRecs rec = pair_recs(a, pair);
   // selection blocks of l' tokens
@@ -575,15 +521,12 @@ __global__ void __launch_bounds__(kDecThreads)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // everything below reads kernel A's results (selection, P^T, window).  The
-  // TMEM is allocated only after kernel A has finished: a CTA of this grid
-  // that waits here holds no TMEM that a CTA of kernel A could need.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 64);  // S^T of two chunks at 0 and 16, O^T at 32
+    tmem_alloc(tmem_slot, 128);  // S^T of four chunks at 0, 16, 32, 48; O^T at 64
     tmem_relinquish();
   }
-  if (threadIdx.x < 64) sel_s[threadIdx.x] = (!is_cmp && threadIdx.x < n) ? rec.sel[threadIdx.x] : -1;
+  if (threadIdx.x < 64)
+    sel_s[threadIdx.x] = (!is_cmp && !is_win && threadIdx.x < n) ? rec.sel[threadIdx.x] : -1;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -631,6 +574,14 @@ __global__ void __launch_bounds__(kDecThreads)
               uint8_t* dst = acquire();
               if (!dst) break;
               const int s = sc % L::kStages;
+              if (is_win) {  // 128 consecutive window rows ending at t
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+                  tma_load_4d(dst + h * 16384, pass ? &maps.v_win : &maps.k_win, st_full + s, h * 64,
+                              g, P.win_row0 + c * kChunk, b);
+                ++sc;
+                continue;
+              }
               for (int sub = 0; sub < bpc; ++sub) {
                 const int bs = c * bpc + sub;
                 const int blk = bs < n ? sel_s[bs] : -1;
@@ -671,7 +622,7 @@ __global__ void __launch_bounds__(kDecThreads)
           for (int c = 0; c < nch && ok; ++c) {
             const uint32_t st = wait_stage();
             if (!ok) break;
-            issue_pv(tmem + 32, st, sbase + L::kP + c * kPChunkBytes, c > 0);
+            issue_pv(tmem + 64, st, sbase + L::kP + c * kPChunkBytes, c > 0);
             mma_commit(st_empty + (sc % L::kStages));
             ++sc;
           }
@@ -691,7 +642,7 @@ __global__ void __launch_bounds__(kDecThreads)
             for (int c = 0; c < nch && ok; ++c) {
               const uint32_t st = wait_stage();
               if (!ok) break;
-              issue_pv(tmem + 32, st, sbase + L::kP + c * kPChunkBytes, c > 0);
+              issue_pv(tmem + 64, st, sbase + L::kP + c * kPChunkBytes, c > 0);
               mma_commit(st_empty + (sc % L::kStages));
               ++sc;
             }
@@ -711,19 +662,26 @@ __global__ void __launch_bounds__(kDecThreads)
       const uint32_t colmask = (G >= 16) ? 0xFFFFu : ((1u << G) - 1u);
       float mx[16], sm16[16];
       if (!is_cmp) {
-        // keys of this lane that are visible selected keys, per chunk
-        const int key_in_blk = r & (l - 1), slot_in_chunk = r >> lg_l;
+        // keys of this lane that take part, per chunk: window keys from
+        // max(0, t - w + 1), or visible keys of the selected blocks
         uint32_t kok = 0;
-        for (int c = 0; c < nch; ++c) {
-          const int bs = (c_lo + c) * bpc + slot_in_chunk;
-          const int blk = bs < n ? sel_s[bs] : -1;
-          kok |= (blk >= 0 && sel_row0(blk, l, t) + key_in_blk >= blk * l) ? (1u << c) : 0u;
+        if (is_win) {
+          const int lo = max(0, t - a.geo.w + 1);
+          for (int c = 0; c < nch; ++c)
+            kok |= (P.win_row0 + (c_lo + c) * kChunk + r >= lo) ? (1u << c) : 0u;
+        } else {
+          const int key_in_blk = r & (l - 1), slot_in_chunk = r >> lg_l;
+          for (int c = 0; c < nch; ++c) {
+            const int bs = (c_lo + c) * bpc + slot_in_chunk;
+            const int blk = bs < n ? sel_s[bs] : -1;
+            kok |= (blk >= 0 && sel_row0(blk, l, t) + key_in_blk >= blk * l) ? (1u << c) : 0u;
+          }
         }
         mbar_wait(s_full, 0, abort_flag, status, kWaitCycles);
         tc_fence_after();
 #pragma unroll
         for (int h = 0; h < 16; ++h) mx[h] = -INFINITY;
-        sweep_chunks<4>(lane_addr, 0, nch, [&](int c, const float(&v)[16]) {
+        sweep_chunks<kUnitChunks>(lane_addr, 0, nch, [&](int c, const float(&v)[16]) {
           if ((kok >> c) & 1u) {
 #pragma unroll
             for (int h = 0; h < 16; ++h) mx[h] = fmaxf(mx[h], v[h] * sl2);
@@ -732,7 +690,7 @@ __global__ void __launch_bounds__(kDecThreads)
         reduce16_across_128<1>(mx, red, q4, lane, true);
 #pragma unroll
         for (int h = 0; h < 16; ++h) sm16[h] = 0.f;
-        sweep_chunks<4>(lane_addr, 0, nch, [&](int c, const float(&v)[16]) {
+        sweep_chunks<kUnitChunks>(lane_addr, 0, nch, [&](int c, const float(&v)[16]) {
           const bool on = (kok >> c) & 1u;
           float p[16];
 #pragma unroll
@@ -751,7 +709,7 @@ __global__ void __launch_bounds__(kDecThreads)
       mbar_wait(o_done, 0, abort_flag, status, kWaitCycles);
       tc_fence_after();
       float o[16];
-      tmem_ld16(lane_addr + 32, o);
+      tmem_ld16(lane_addr + 64, o);
       tmem_ld_wait();
       if (r < D && !*abort_flag) {
         if (is_cmp) {
@@ -762,7 +720,7 @@ __global__ void __launch_bounds__(kDecThreads)
             dst[h * D + r] = o[h];
           }
         } else {
-          float* dst = rec.slc + (size_t)u * (G * D + 32);
+          float* dst = (is_win ? rec.win : rec.slc) + (size_t)u * partial_floats(G, D);
 #pragma unroll
           for (int h = 0; h < 16; ++h) {
             if (h >= G) break;
@@ -784,7 +742,7 @@ __global__ void __launch_bounds__(kDecThreads)
   } else if (warp >= 2 && !is_cmp) {
     // a selected unit with no chunk: an empty partial
     const int r = threadIdx.x - 64;
-    float* dst = rec.slc + (size_t)u * (G * D + 32);
+    float* dst = (is_win ? rec.win : rec.slc) + (size_t)u * partial_floats(G, D);
     if (r < D)
       for (int h = 0; h < G; ++h) dst[h * D + r] = 0.f;
     if (r < G) {
@@ -806,43 +764,54 @@ __global__ void __launch_bounds__(kDecThreads)
     // per-head statistics of the selected partials and the gates, staged in
     // the (now idle) P^T region; then every (head, 4 channels) item issues
     // all of its partial loads before combining them
-    float* ml = reinterpret_cast<float*>(sm + L::kP);  // [nsl][m[16], sum[16]]
-    float* gt = ml + 8 * 32;                            // [G][3]
-    const int Hq = a.geo.Hq;
+    float* ml = reinterpret_cast<float*>(sm + L::kP);  // selected [nsl][m[16], sum[16]]
+    float* wml = ml + kMaxSlcUnits * 32;                // window [nwu][m[16], sum[16]]
+    float* gt = wml + kMaxWinUnits * 32;                // [G][3]
+    const int Hq = a.geo.Hq, PF = partial_floats(G, D);
     for (int i = threadIdx.x; i < a.nsl * 32; i += blockDim.x)
-      ml[i] = __ldcg(rec.slc + (size_t)(i >> 5) * (G * D + 32) + G * D + (i & 31));
+      ml[i] = __ldcg(rec.slc + (size_t)(i >> 5) * PF + G * D + (i & 31));
+    for (int i = threadIdx.x; i < a.nwu * 32; i += blockDim.x)
+      wml[i] = __ldcg(rec.win + (size_t)(i >> 5) * PF + G * D + (i & 31));
     for (int i = threadIdx.x; i < G * 3; i += blockDim.x)
       gt[i] = __ldg(a.gates + ((size_t)b * Hq + g * G) * 3 + i);
     __syncthreads();
-    const int ncv = (P.ncc + 1) / 2;
+    const int ncv = (P.ncc + kUnitChunks - 1) / kUnitChunks;
     for (int item = threadIdx.x; item < G * (D / 4); item += blockDim.x) {
       const int h = item / (D / 4), c4 = (item - h * (D / 4)) * 4;
-      float4 vs[kMaxSlcUnits], vc[kMaxCmpUnits];
+      float4 vs[kMaxSlcUnits], vw[kMaxWinUnits], vc[kMaxCmpUnits];
 #pragma unroll
       for (int s2 = 0; s2 < kMaxSlcUnits; ++s2)
         if (s2 < a.nsl)
-          vs[s2] = __ldcg(reinterpret_cast<const float4*>(rec.slc + (size_t)s2 * (G * D + 32) +
-                                                          h * D + c4));
+          vs[s2] = __ldcg(reinterpret_cast<const float4*>(rec.slc + (size_t)s2 * PF + h * D + c4));
+#pragma unroll
+      for (int s2 = 0; s2 < kMaxWinUnits; ++s2)
+        if (s2 < a.nwu)
+          vw[s2] = __ldcg(reinterpret_cast<const float4*>(rec.win + (size_t)s2 * PF + h * D + c4));
 #pragma unroll
       for (int u2 = 0; u2 < kMaxCmpUnits; ++u2)
         if (u2 < ncv)
           vc[u2] = __ldcg(reinterpret_cast<const float4*>(rec.cmp + ((size_t)u2 * G + h) * D + c4));
-      const float4 w4 = __ldcg(reinterpret_cast<const float4*>(rec.win + h * D + c4));
-      float M = -INFINITY;
-      for (int s2 = 0; s2 < a.nsl; ++s2) M = fmaxf(M, ml[s2 * 32 + h]);
-      float4 os = make_float4(0.f, 0.f, 0.f, 0.f);
-      float ls = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < kMaxSlcUnits; ++s2) {
-        if (s2 >= a.nsl) break;
-        const float ms = ml[s2 * 32 + h];
-        const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
-        ls += ml[s2 * 32 + 16 + h] * f;
-        os.x += vs[s2].x * f;
-        os.y += vs[s2].y * f;
-        os.z += vs[s2].z * f;
-        os.w += vs[s2].w * f;
-      }
+      // softmax partials (row maximum m, sum, unnormalised O) -> normalised O
+      auto merge = [&](const float* mlv, const float4* v, int units_of, int max_units) {
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < units_of; ++s2) M = fmaxf(M, mlv[s2 * 32 + h]);
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        float ls = 0.f;
+        for (int s2 = 0; s2 < max_units; ++s2) {
+          if (s2 >= units_of) break;
+          const float ms = mlv[s2 * 32 + h];
+          const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
+          ls += mlv[s2 * 32 + 16 + h] * f;
+          o.x += v[s2].x * f;
+          o.y += v[s2].y * f;
+          o.z += v[s2].z * f;
+          o.w += v[s2].w * f;
+        }
+        const float inv = ls > 0.f ? 1.f / ls : 0.f;
+        return make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+      };
+      const float4 os = merge(ml, vs, a.nsl, kMaxSlcUnits);
+      const float4 ow = merge(wml, vw, a.nwu, kMaxWinUnits);
       float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u2 = 0; u2 < kMaxCmpUnits; ++u2) {
@@ -852,10 +821,9 @@ __global__ void __launch_bounds__(kDecThreads)
         oc.z += vc[u2].z;
         oc.w += vc[u2].w;
       }
-      const float inv = ls > 0.f ? 1.f / ls : 0.f;
-      const float g0 = gt[h * 3 + 0], g1 = gt[h * 3 + 1] * inv, g2 = gt[h * 3 + 2];
-      const float e[4] = {g0 * oc.x + g1 * os.x + g2 * w4.x, g0 * oc.y + g1 * os.y + g2 * w4.y,
-                          g0 * oc.z + g1 * os.z + g2 * w4.z, g0 * oc.w + g1 * os.w + g2 * w4.w};
+      const float g0 = gt[h * 3 + 0], g1 = gt[h * 3 + 1], g2 = gt[h * 3 + 2];
+      const float e[4] = {g0 * oc.x + g1 * os.x + g2 * ow.x, g0 * oc.y + g1 * os.y + g2 * ow.y,
+                          g0 * oc.z + g1 * os.z + g2 * ow.z, g0 * oc.w + g1 * os.w + g2 * ow.w};
       const size_t oi = ((size_t)b * Hq + g * G + h) * D + c4;
       if (a.geo.out_f32) {
         *reinterpret_cast<float4*>(static_cast<float*>(a.out) + oi) = make_float4(e[0], e[1], e[2], e[3]);
@@ -868,7 +836,7 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64);
+    tmem_dealloc(tmem, 128);
   }
 }
 
@@ -889,7 +857,7 @@ cudaError_t launch_decode_a_t(const DecodeArgs& a, const DecodeMaps& m, cudaStre
   static bool conf[64] = {};
   cudaError_t e = set_smem(nsa_decode_a_kernel<D>, DecALayout<D>::kSmem, conf);
   if (e != cudaSuccess) return e;
-  nsa_decode_a_kernel<D><<<a.batch * a.geo.Hkv * 2, kDecThreads, DecALayout<D>::kSmem, s>>>(a, m);
+  nsa_decode_a_kernel<D><<<a.batch * a.geo.Hkv, kDecThreads, DecALayout<D>::kSmem, s>>>(a, m);
   return cudaGetLastError();
 }
 
@@ -898,19 +866,9 @@ cudaError_t launch_decode_b_t(const DecodeArgs& a, const DecodeMaps& m, cudaStre
   static bool conf[64] = {};
   cudaError_t e = set_smem(nsa_decode_b_kernel<D>, DecBLayout<D>::kSmem, conf);
   if (e != cudaSuccess) return e;
-  // programmatic dependent launch: the CTAs of this grid start while kernel A
-  // runs and wait for its results inside the kernel (griddepcontrol.wait)
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.batch * a.geo.Hkv * (a.ncv_max + a.nsl));
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = DecBLayout<D>::kSmem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, nsa_decode_b_kernel<D>, a, m);
+  const int grid = a.batch * a.geo.Hkv * (a.ncv_max + a.nwu + a.nsl);
+  nsa_decode_b_kernel<D><<<grid, kDecThreads, DecBLayout<D>::kSmem, s>>>(a, m);
+  return cudaGetLastError();
 }
 
 }  // namespace

@@ -73,7 +73,7 @@ PrefillLayout prefill_layout(const nsa_plan_s* pl) {
 
 struct DecodeLayout {
   size_t counters, sel, pt, win, cmp, slc, total;
-  int ncc_max, ncv_max, nsl;
+  int ncc_max, ncv_max, nsl, nwu;
 };
 
 // Decode workspace for `batch` sequences in a cache of `cap` tokens:
@@ -85,9 +85,11 @@ DecodeLayout decode_layout(const nsa_plan_s* pl, int batch, int cap) {
   const size_t pairs = (size_t)batch * g.Hkv;
   const int ccap = cap / g.d;
   L.ncc_max = (ccap + kChunk - 1) / kChunk;
-  L.ncv_max = (L.ncc_max + 1) / 2;
+  L.ncv_max = (L.ncc_max + kUnitChunks - 1) / kUnitChunks;
   const int nsc = (g.n + (kChunk >> g.lg_ls) - 1) / (kChunk >> g.lg_ls);
-  L.nsl = (nsc + 1) / 2;
+  L.nsl = (nsc + kUnitChunks - 1) / kUnitChunks;
+  const int wmax = g.w < cap ? g.w : cap;
+  L.nwu = ((wmax + kChunk - 1) / kChunk + kUnitChunks - 1) / kUnitChunks;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -98,7 +100,7 @@ DecodeLayout decode_layout(const nsa_plan_s* pl, int batch, int cap) {
   L.counters = take(pairs * sizeof(int));
   L.sel = take(pairs * g.n * sizeof(int));
   L.pt = take(pairs * (size_t)L.ncc_max * 4096);
-  L.win = take(pairs * g.G * g.D * sizeof(float));
+  L.win = take(pairs * (size_t)L.nwu * (g.G * g.D + 32) * sizeof(float));
   L.cmp = take(pairs * (size_t)L.ncv_max * g.G * g.D * sizeof(float));
   L.slc = take(pairs * (size_t)L.nsl * (g.G * g.D + 32) * sizeof(float));
   L.total = off;
@@ -473,6 +475,7 @@ int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* 
   a.ncc_max = DL.ncc_max;
   a.ncv_max = DL.ncv_max;
   a.nsl = DL.nsl;
+  a.nwu = DL.nwu;
   a.counters = reinterpret_cast<int*>(ws + DL.counters);
   a.ws_sel = reinterpret_cast<int*>(ws + DL.sel);
   a.ws_pt = ws + DL.pt;

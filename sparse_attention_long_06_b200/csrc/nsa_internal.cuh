@@ -113,12 +113,13 @@ struct DecodeArgs {
   // units of the second decode kernel and its workspace records (per
   // (sequence, group) pair: see nsa_decode_b_kernel)
   int ncc_max;              // ceil(ccap / 128): compressed chunks of the longest sequence
-  int ncv_max;              // ceil(ncc_max / 2): compressed-value units per pair
-  int nsl;                  // ceil(selected chunks / 2): selected units per pair
+  int ncv_max;              // ceil(ncc_max / kUnitChunks): compressed-value units per pair
+  int nsl;                  // ceil(selected chunks / kUnitChunks): selected units per pair
+  int nwu;                  // ceil(window chunks / kUnitChunks): window units per pair
   int* counters;            // [B * Hkv] finished units per pair (zero at launch)
   int* ws_sel;              // [B * Hkv, n]
   uint8_t* ws_pt;           // [B * Hkv, ncc_max, 4096 B] normalised compressed P^T, bf16
-  float* ws_win;            // [B * Hkv, G, D]
+  float* ws_win;            // [B * Hkv, nwu, G * D + 32] window partials
   float* ws_cmp;            // [B * Hkv, ncv_max, G, D]
   float* ws_slc;            // [B * Hkv, nsl, G * D + 32]
 };
@@ -136,6 +137,8 @@ struct DecodeMaps {
 // Largest number of compressed blocks one decode query may see (all of its
 // compressed scores stay in TMEM: 32 chunks of 128 keys x 16 columns).
 constexpr int kDecodeMaxCmp = 4096;
+// 128-key chunks per unit of the second decode kernel
+constexpr int kUnitChunks = 4;
 
 // Complete compressed blocks among the first `len` tokens of a sequence
 // (block i covers tokens [i d, i d + l - 1]).

@@ -176,4 +176,75 @@ __device__ __forceinline__ bool warp_topn_regs(ScoreFn score, int ncmp, int ncan
   return true;
 }
 
+// The same selection as warp_topn_regs for any number of candidates whose
+// scores `score(j)` are cheap to re-read (shared memory): one pass finds each
+// lane's largest key (lane = j % 32), T0 = the n-th largest lane maximum; a
+// second pass gathers the keys >= T0 into `cand` and ranks them exactly; a
+// third writes every key >= the n-th largest in ascending block order.
+// Returns false, having written nothing, when more than kTopnCand keys reach
+// T0 (the caller then uses warp_topn).
+template <typename ScoreFn, typename OutFn>
+__device__ __forceinline__ bool warp_topn_reread(ScoreFn score, int ncmp, int ncand, int n,
+                                                 unsigned long long* cand, OutFn out) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  if (ncand <= n) {
+    for (int j = lane; j < n; j += 32) out(j, j < ncand ? j : -1);
+    return true;
+  }
+  auto key = [&](int j) -> unsigned long long {
+    const uint32_t b = j < ncmp ? __float_as_uint(score(j)) : 0u;
+    return ((unsigned long long)b << 32) | (0xFFFFFFFFu - (uint32_t)j);
+  };
+  unsigned long long lmax = 0;
+  for (int j = lane; j < ncand; j += 32) {
+    const unsigned long long k = key(j);
+    lmax = k > lmax ? k : lmax;
+  }
+  int rank = 0;
+#pragma unroll
+  for (int o = 0; o < 32; ++o) {
+    const unsigned long long other = __shfl_sync(0xffffffffu, lmax, o);
+    rank += other > lmax;
+  }
+  const unsigned tb = __ballot_sync(0xffffffffu, rank == n - 1 && lmax != 0ull);
+  const unsigned long long t0 = __shfl_sync(0xffffffffu, lmax, __ffs(tb) - 1);
+  int count = 0;
+  for (int base = 0; base < ncand; base += 32) {
+    const int j = base + lane;
+    const unsigned long long k = j < ncand ? key(j) : 0ull;
+    const bool p = k >= t0 && k != 0ull;
+    const unsigned m = __ballot_sync(0xffffffffu, p);
+    const int pos = count + __popc(m & lt_mask);
+    if (p && pos < kTopnCand) cand[pos] = k;
+    count += __popc(m);
+  }
+  if (count > kTopnCand) return false;
+  __syncwarp();
+  unsigned long long kth = 0ull;
+  bool have = false;
+  for (int c = lane; c < count; c += 32) {
+    const unsigned long long mine = cand[c];
+    int r = 0;
+    for (int e = 0; e < count; ++e) r += cand[e] > mine;
+    if (r == n - 1) {
+      kth = mine;
+      have = true;
+    }
+  }
+  const unsigned hb = __ballot_sync(0xffffffffu, have);
+  kth = __shfl_sync(0xffffffffu, kth, __ffs(hb) - 1);
+  __syncwarp();
+  int written = 0;
+  for (int base = 0; base < ncand; base += 32) {
+    const int j = base + lane;
+    const unsigned long long k = j < ncand ? key(j) : 0ull;
+    const bool take = k >= kth && k != 0ull;
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (take) out(written + __popc(m & lt_mask), j);
+    written += __popc(m);
+  }
+  return true;
+}
+
 }  // namespace nsa

@@ -14,8 +14,9 @@ bf16 arithmetic of the path):
     the same call (a bf16 store adds up to half a bf16 ulp, 0.0078 at |o| in
     [2, 4), so the 1e-2 bound applies to the fp32 result);
   * end to end (oracle's own compressed KV): index sets differ only where a
-    1-ulp difference of the compressed KV moves a near-tie (reported, under
-    2 % of rows), and rows with equal index sets agree within 1e-2.
+    1-ulp difference of the compressed KV moves a near-tie (counted and
+    logged; at most 0.5 % of a test's rows, six times the worst rate seen),
+    and rows with equal index sets agree within 1e-2.
 """
 import numpy as np
 import pytest
@@ -48,7 +49,8 @@ def _assert_report(rep, res=None, e2e=True, name="prefill"):
         assert np.array_equal(res["out_bf16"], wl.bf16_bits(res["out"].astype(np.float32)))
     assert rep["rel_l2"] <= 5e-3
     if e2e and rep["e2e_rows"]:
-        assert rep["e2e_idx_mismatch"] <= 0.02 * rep["e2e_rows"]
+        # observed over the suite: 12 of 117 914 rows (worst test 0.08 %)
+        assert rep["e2e_idx_mismatch"] <= max(1, 0.005 * rep["e2e_rows"])
         assert rep["e2e_max_abs"] <= 1e-2
 
 
