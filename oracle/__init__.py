@@ -11,7 +11,9 @@ header of that file cites the pages and lists the readings taken where the
 pages are silent.
 """
 from .oracle import (OracleParams, build, compress, nsa_rows, nsa_query, select_f32,
-                     num_cmp_blocks, prefill_reference, decode_reference, bf16_round_f64)
+                     num_cmp_blocks, prefill_reference, decode_reference, bf16_round_f64,
+                     block_means, block_select_rows, block_select_reference)
 
 __all__ = ["OracleParams", "build", "compress", "nsa_rows", "nsa_query", "select_f32",
-           "num_cmp_blocks", "prefill_reference", "decode_reference", "bf16_round_f64"]
+           "num_cmp_blocks", "prefill_reference", "decode_reference", "bf16_round_f64",
+           "block_means", "block_select_rows", "block_select_reference"]

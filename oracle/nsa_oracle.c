@@ -350,3 +350,138 @@ void oracle_select_f32(const float* S, int nrows, int cstride, const int* ncand,
     free(s);
   }
 }
+
+/* ------------------------------------------------------------ select-only block attention */
+/*
+ * Block attention with selection only, in the style of MoBA ("NSA vs MoBA"
+ * page (gtnt.cn/news/122266), section 1: the sequence is cut into blocks and
+ * a gate decides, per query, which key blocks it attends to, the way a
+ * mixture of experts routes tokens).  The page gives no formula; the readings
+ * (listed in the repository's design notes) are:
+ *  - a block's routing key is the mean of its l' keys, stored in bf16 (round
+ *    to nearest even);
+ *  - the routing score of block j for query t and KV group g is the sum over
+ *    the group's query heads of q . mean-key (the selection is shared by the
+ *    group, as in the NSA branch);
+ *  - the block holding t is always attended; the other n - 1 blocks are the
+ *    best-scoring complete blocks before it (ties to the lower index; all of
+ *    them when there are at most n - 1);
+ *  - the output is one softmax attention of each head over the tokens u <= t
+ *    of the chosen blocks (scale as in the NSA branches); no gate, no other
+ *    branch.
+ */
+
+/* Mean keys of the complete blocks of one sequence: X [T, Hkv, D] bf16 bits,
+ * out [T / l', Hkv, D] fp64 (unrounded) and bf16 (rounded); either may be NULL. */
+void oracle_block_means(const nsa_oracle_params* P, int T, const uint16_t* X, double* out_f64,
+                        uint16_t* out_bf16) {
+  const int L = P->lsel, nb = T / L, D = P->D, H = P->Hkv;
+  for (int j = 0; j < nb; ++j)
+    for (int h = 0; h < H; ++h)
+      for (int c = 0; c < D; ++c) {
+        double acc = 0.0;
+        for (int p = 0; p < L; ++p) acc += oracle_bf16_to_f64(X[((size_t)(j * L + p) * H + h) * D + c]);
+        const double m = acc / L;
+        const size_t o = ((size_t)j * H + h) * D + c;
+        if (out_f64) out_f64[o] = m;
+        if (out_bf16) out_bf16[o] = oracle_f64_to_bf16(m);
+      }
+}
+
+/*
+ * One query at position t of a sequence with keys/values k, v ([>= t+1, Hkv,
+ * D] bf16) and stored mean keys kbar ([>= t / l', Hkv, D] bf16).
+ *   q [Hq, D] bf16.  Outputs (any may be NULL):
+ *   out    [Hq, D]      attention output
+ *   scores [Hkv, cmax]  routing scores of the complete blocks before t's block
+ *                       (entries >= t / l' left 0)
+ *   sel    [Hkv, n]     attended blocks, ascending, -1 padded (t's block last)
+ *   gap    [Hkv]        (n-1)-th minus n-th ranked routing score (+inf when
+ *                       every candidate is taken)
+ * Returns 0, or -1 on an invalid geometry.
+ */
+int oracle_block_select_query(const nsa_oracle_params* P, int t, const uint16_t* q,
+                              const uint16_t* k, const uint16_t* v, const uint16_t* kbar,
+                              double* out, double* scores, int cmax, int* sel, double* gap) {
+  const int D = P->D, Hq = P->Hq, Hkv = P->Hkv, G = Hq / Hkv, L = P->lsel;
+  if (Hq % Hkv != 0 || L < 1 || P->n < 1) return -1;
+  const int cur = t / L;   /* the block holding t */
+  const int npast = cur;   /* complete blocks before it: the candidates */
+  const int m = P->n - 1;  /* blocks chosen by score */
+  double* S = (double*)malloc(sizeof(double) * (size_t)(npast > 0 ? npast : 1));
+  int* chosen = (int*)malloc(sizeof(int) * (size_t)(m > 0 ? m : 1));
+  int* rows = (int*)malloc(sizeof(int) * (size_t)P->n * L);
+  double* scratch = (double*)malloc(sizeof(double) * (size_t)P->n * L);
+  double* qh = (double*)malloc(sizeof(double) * (size_t)D);
+  double* o = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int g = 0; g < Hkv; ++g) {
+    for (int j = 0; j < npast; ++j) {
+      double s = 0.0;
+      for (int hh = 0; hh < G; ++hh) {
+        const int h = g * G + hh;
+        for (int c = 0; c < D; ++c)
+          s += oracle_bf16_to_f64(q[(size_t)h * D + c]) *
+               oracle_bf16_to_f64(kbar[((size_t)j * Hkv + g) * D + c]);
+      }
+      S[j] = s;
+    }
+    if (scores)
+      for (int j = 0; j < cmax; ++j) scores[(size_t)g * cmax + j] = (j < npast) ? S[j] : 0.0;
+    double gp = INFINITY;
+    int taken = 0;
+    if (m > 0) {
+      gp = oracle_select(S, npast, m, chosen);
+      taken = npast < m ? npast : m;
+    }
+    if (gap) gap[g] = gp;
+    if (sel) {
+      for (int i = 0; i < P->n; ++i) sel[(size_t)g * P->n + i] = -1;
+      for (int i = 0; i < taken; ++i) sel[(size_t)g * P->n + i] = chosen[i];
+      sel[(size_t)g * P->n + taken] = cur;
+    }
+    int nk = 0;
+    for (int i = 0; i < taken; ++i)
+      for (int u = chosen[i] * L; u < (chosen[i] + 1) * L; ++u) rows[nk++] = u;
+    for (int u = cur * L; u <= t; ++u) rows[nk++] = u;
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      for (int c = 0; c < D; ++c) qh[c] = oracle_bf16_to_f64(q[(size_t)h * D + c]);
+      attend(P, qh, k, v, g, rows, nk, o, NULL, scratch);
+      if (out)
+        for (int c = 0; c < D; ++c) out[(size_t)h * D + c] = o[c];
+    }
+  }
+  free(S);
+  free(chosen);
+  free(rows);
+  free(scratch);
+  free(qh);
+  free(o);
+  return 0;
+}
+
+/* oracle_block_select_query for a list of rows of one sequence:
+ * q [T, Hq, D], k, v [T, Hkv, D], kbar [T / l', Hkv, D]; outputs are indexed
+ * by the position in `rows`. */
+int oracle_block_select_rows(const nsa_oracle_params* P, int T, const uint16_t* q,
+                             const uint16_t* k, const uint16_t* v, const uint16_t* kbar,
+                             const int* rows, int nrows, double* out, double* scores, int cmax,
+                             int* sel, double* gap) {
+  const int D = P->D, Hq = P->Hq, Hkv = P->Hkv;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int r = 0; r < nrows; ++r) {
+    const int t = rows[r];
+    if (t < 0 || t >= T) {
+      bad |= 1;
+      continue;
+    }
+    const size_t hd = (size_t)Hq * D;
+    int rc = oracle_block_select_query(
+        P, t, q + (size_t)t * hd, k, v, kbar, out ? out + r * hd : NULL,
+        scores ? scores + (size_t)r * Hkv * cmax : NULL, cmax,
+        sel ? sel + (size_t)r * Hkv * P->n : NULL, gap ? gap + (size_t)r * Hkv : NULL);
+    bad |= (rc != 0);
+  }
+  return bad ? -1 : 0;
+}

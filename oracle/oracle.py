@@ -85,6 +85,11 @@ def _load():
             lib.oracle_f64_to_bf16.restype = ctypes.c_uint16
             lib.oracle_num_cmp_blocks.argtypes = [P, ctypes.c_int]
             lib.oracle_num_cmp_blocks.restype = ctypes.c_int
+            lib.oracle_block_means.argtypes = [P, ctypes.c_int, vp, vp, vp]
+            lib.oracle_block_means.restype = None
+            lib.oracle_block_select_rows.argtypes = [P, ctypes.c_int, vp, vp, vp, vp, vp,
+                                                     ctypes.c_int, vp, vp, ctypes.c_int, vp, vp]
+            lib.oracle_block_select_rows.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -232,3 +237,64 @@ def decode_reference(p: OracleParams, inputs: dict, b: int, kc=None, vc=None) ->
     r = nsa_query(p, t, inputs["q"][b], k, v, kc, vc, inputs["gates"][b], cmax=kc.shape[0])
     r.update(kc_used=kc, vc_used=vc, t=t)
     return r
+
+
+# ---------------------------------------------------------------- select-only block attention
+def block_means(p: OracleParams, x_bits: np.ndarray):
+    """Mean keys of the complete l'-token blocks of one sequence: x [T,Hkv,D]
+    bf16 bits.  Returns (fp64 [T//l',Hkv,D], bf16 bits [T//l',Hkv,D])."""
+    x = _c(x_bits, np.uint16)
+    nb = x.shape[0] // p.sel_block
+    f = np.zeros((nb, p.num_kv_heads, p.head_dim), dtype=np.float64)
+    b = np.zeros((nb, p.num_kv_heads, p.head_dim), dtype=np.uint16)
+    if nb:
+        _load().oracle_block_means(ctypes.byref(p.c()), x.shape[0], _ptr(x), _ptr(f), _ptr(b))
+    return f, b
+
+
+def block_select_rows(p: OracleParams, q, k, v, kbar, rows, cmax: int | None = None) -> dict:
+    """Select-only block attention for the query rows `rows` of one sequence.
+
+    q [T,Hq,D], k/v [T,Hkv,D], kbar [>=1,Hkv,D] (bf16 bits).  Returns fp64 out
+    [R,Hq,D], scores [R,Hkv,cmax] (routing scores of the complete blocks
+    before each row's block), sel [R,Hkv,n] (int32) and gap [R,Hkv]."""
+    q, k, v, kbar = _c(q, np.uint16), _c(k, np.uint16), _c(v, np.uint16), _c(kbar, np.uint16)
+    rows = _c(rows, np.int32)
+    T = q.shape[0]
+    R, Hq, Hkv, D, n = len(rows), p.num_q_heads, p.num_kv_heads, p.head_dim, p.top_n
+    if cmax is None:
+        cmax = max(1, T // p.sel_block)
+    res = {"out": np.zeros((R, Hq, D)), "scores": np.zeros((R, Hkv, cmax)),
+           "sel": np.zeros((R, Hkv, n), dtype=np.int32), "gap": np.zeros((R, Hkv))}
+    rc = _load().oracle_block_select_rows(ctypes.byref(p.c()), T, _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(kbar), _ptr(rows), R, _ptr(res["out"]),
+                                          _ptr(res["scores"]), cmax, _ptr(res["sel"]),
+                                          _ptr(res["gap"]))
+    if rc != 0:
+        raise ValueError("oracle rejected the geometry or a row index")
+    return res
+
+
+def block_select_reference(p: OracleParams, inputs: dict, rows_per_seq=None,
+                           kbar_override=None) -> list[dict]:
+    """Select-only block attention over a packed batch from
+    ``workloads.prefill_inputs`` (q, k, v, cu_seqlens are used).
+    kbar_override: packed [sum T_b // l', Hkv, D] bf16 mean keys to route with
+    instead of the oracle's own (stage-wise checks)."""
+    cu = inputs["cu_seqlens"]
+    out = []
+    boff = 0
+    for b in range(len(cu) - 1):
+        s, e = int(cu[b]), int(cu[b + 1])
+        T = e - s
+        nb = T // p.sel_block
+        kb64, kb16 = block_means(p, inputs["k"][s:e])
+        use = kb16 if kbar_override is None else kbar_override[boff:boff + nb]
+        boff += nb
+        rows = np.arange(T) if rows_per_seq is None else np.asarray(rows_per_seq[b])
+        r = block_select_rows(p, inputs["q"][s:e], inputs["k"][s:e], inputs["v"][s:e],
+                              use if nb else np.zeros((1, p.num_kv_heads, p.head_dim), np.uint16),
+                              rows)
+        r.update(rows=rows, kbar64=kb64, kbar16=kb16)
+        out.append(r)
+    return out
