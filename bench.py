@@ -383,6 +383,8 @@ def run_ours(args, rank, world):
         result["legs"] = {name: run_prefill_leg(name, dev, world)
                           for name in ("prefill_8k", "varlen", "prefill_8k_overlap")
                           if name != args.workload}
+        torch.cuda.empty_cache()
+        result["legs"]["block_select_64k"] = run_block_select_leg(dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(cfg, inputs)
         result["cpu_baseline_1core"] = oracle_single_core()
@@ -454,6 +456,94 @@ def run_prefill_leg(name, dev, world, steps=10, warmup=3):
             "config": prefill_config(cfg, T, world) | {"seqlens": lens},
             "algorithmic_flop_per_step": flops,
             "stage_ms": dict(zip(KERNEL_NAMES, [round(x, 4) for x in stage_ms])),
+            "rooflines": roof}
+
+
+BLOCK_SELECT_KERNELS = ["nsa_meta_kernel", "nsa_block_mean_kernel", "nsa_block_score_kernel",
+                        "nsa_topn_kernel", "nsa_slc_kernel"]
+
+
+def block_select_flops(cfg, lens, sel):
+    """Exact FLOPs of select-only block attention on a packed batch: routing
+    2 D per (token, head, candidate block) over the t // l' blocks before the
+    own block, plus attention 4 D per (token, head, attended key)."""
+    D, G, ls, Hkv = cfg.head_dim, cfg.group, cfg.sel_block, cfg.num_kv_heads
+    f_route = f_attn = 0
+    s = 0
+    for T in lens:
+        t = np.arange(T, dtype=np.int64)
+        f_route += 2 * D * G * Hkv * int((t // ls).sum())
+        blk = sel[s:s + T].astype(np.int64)
+        keys = np.where(blk >= 0, np.minimum(ls, t[:, None, None] - blk * ls + 1), 0)
+        f_attn += 4 * D * G * int(keys.clip(min=0).sum())
+        s += T
+    return {"route": f_route, "attn": f_attn, "total": f_route + f_attn}
+
+
+def run_block_select_leg(dev, world, steps=10, warmup=3, name="prefill_64k"):
+    """Select-only block attention (own block + n - 1 routed blocks of l'
+    tokens, mean-pooled routing keys) on the geometry and length of `name`:
+    tokens/s and the tensor roofline of the routing and attention kernels."""
+    import torch
+    from sparse_attention_long_06_b200 import nsa
+    cfg = wl.CONFIGS[name]
+    inputs = wl.prefill_inputs(cfg)
+    lens = list(inputs["seqlens"])
+    T = int(inputs["cu_seqlens"][-1])
+    D, Hq, Hkv = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads
+    d = {}
+    for k in ("q", "k", "v", "cu_seqlens"):
+        a = np.ascontiguousarray(inputs[k])
+        d[k] = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+    plan = nsa.Plan.for_config(cfg, max_batch=len(lens), max_seqlen=max(lens), max_total_tokens=T,
+                               out_dtype=nsa.OUT_BF16)
+    out = torch.empty((T, Hq, D), dtype=torch.int16, device=dev)
+    km = torch.empty((max(plan.block_rows(T), 1), Hkv, D), dtype=torch.int16, device=dev)
+    sel = torch.empty((T, Hkv, cfg.top_n), dtype=torch.int32, device=dev)
+    ws = plan.alloc_workspace(nsa.MODE_BLOCK_SELECT, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        plan.block_select_prefill(d["q"], d["k"], d["v"], d["cu_seqlens"], out, km, ws, sel_idx=sel)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if nsa.read_device_status(ws) != nsa.NSA_OK:
+        raise RuntimeError("block select: device status after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ev), world, dev)
+    nsa.profile_enable(True)
+    stage = []
+    for _ in range(3):
+        flush.zero_()
+        step()
+        stage.append(nsa.profile_stage_ms())
+    nsa.profile_enable(False)
+    stage_ms = [statistics.median(x[i] for x in stage) for i in range(len(stage[0]))]
+    flops = block_select_flops(cfg, lens, sel.cpu().numpy())
+    _, _, tc_sust, src = _peaks()
+    roof = {}
+    for kname, key in (("nsa_block_score_kernel", "route"), ("nsa_slc_kernel", "attn")):
+        idx = BLOCK_SELECT_KERNELS.index(kname)
+        ach = flops[key] / (stage_ms[idx] / 1e3) / 1e12
+        roof[kname] = {"achieved": round(ach, 2), "frac": round(ach / tc_sust, 4)}
+    tflops = flops["total"] / (ms / 1e3) / 1e12
+    return {"metric": "select-only block attention tokens/s", "value": round(job_rate(T, world, ms), 1),
+            "unit": "tokens/s", "ms_per_step_median": round(ms, 4), "steps": steps,
+            "sparse_tflops": round(tflops, 2), "frac_of_peak": round(tflops / tc_sust, 4),
+            "peak": tc_sust, "peak_source": f"{src} bf16 sustained",
+            "config": prefill_config(cfg, T, world) | {"mode": "block_select (own block + n - 1 routed)"},
+            "algorithmic_flop_per_step": flops,
+            "stage_ms": dict(zip(BLOCK_SELECT_KERNELS, [round(x, 4) for x in stage_ms])),
             "rooflines": roof}
 
 
@@ -602,6 +692,8 @@ def main():
                     help="run only the decode leg and print its object (profiling)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="sequences in the decode leg (default: the workload's 32)")
+    ap.add_argument("--block-select-only", action="store_true",
+                    help="time only the select-only block attention leg")
     ap.add_argument("--no-legs", action="store_true",
                     help="skip the 8k / varlen prefill lines")
     ap.add_argument("--oracle-sample", default="",
@@ -634,6 +726,9 @@ def main():
         torch.distributed.barrier()
     if args.decode_only:
         res = run_decode_leg(args, torch.device("cuda", torch.cuda.current_device()), world)
+    elif args.block_select_only:
+        res = run_block_select_leg(torch.device("cuda", torch.cuda.current_device()), world,
+                                   steps=max(args.steps, 3), warmup=args.warmup)
     else:
         res = run_ours(args, rank, world)
     if world > 1:

@@ -72,7 +72,11 @@ typedef enum {
 } nsa_status;
 
 typedef enum { NSA_OUT_BF16 = 0, NSA_OUT_F32 = 1 } nsa_out_dtype;
-typedef enum { NSA_MODE_PREFILL = 0, NSA_MODE_DECODE = 1 } nsa_mode;
+typedef enum {
+  NSA_MODE_PREFILL = 0,      /* nsa_prefill, nsa_prefill_noalloc */
+  NSA_MODE_DECODE = 1,       /* nsa_decode */
+  NSA_MODE_BLOCK_SELECT = 2  /* nsa_block_select_prefill */
+} nsa_mode;
 
 typedef struct {
   int head_dim;          /* D = d_k = d_v: 64 or 128 */
@@ -107,7 +111,8 @@ void nsa_plan_destroy(nsa_plan_t plan);
 size_t nsa_workspace_size(nsa_plan_t plan, int mode);
 
 /* Named regions of the prefill workspace, for inspection by tests and
- * debugging.  Valid after a completed nsa_prefill on that workspace. */
+ * debugging.  Valid after a completed nsa_prefill on that workspace (or, for
+ * mode NSA_MODE_BLOCK_SELECT, nsa_block_select_prefill: STATUS, SCORES, SEL). */
 typedef enum {
   NSA_WS_STATUS = 0,  /* int32 status word */
   NSA_WS_O_CMP = 1,   /* fp32 [T_total, Hq, D] compressed-branch output */
@@ -218,6 +223,49 @@ int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* 
                int cache_capacity, const float* gates, const float* w_k, const float* w_v,
                void* out, int* sel_idx, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * Select-only block attention (MoBA style) over a packed batch: causal, each
+ * query attends to its own block of l' tokens and to the n - 1 best-routed
+ * complete blocks before it, with one softmax per head and no other branch.
+ * "NSA vs MoBA" page (gtnt.cn/news/122266), section 1: the sequence is cut
+ * into blocks and a gate routes every query to a few of them, like a mixture
+ * of experts.  Readings of that description (the page gives no formula):
+ *   - the routing key of block j of a sequence is the mean of its l' keys,
+ *     rounded once to bf16 (nearest even);
+ *   - the routing score of block j for token t and KV group g is the sum over
+ *     the group's query heads of q_t,h . key_j (shared by the group);
+ *   - the n - 1 highest scores among the blocks j < t / l' are taken (ties to
+ *     the lower index; all of them when there are at most n - 1), plus t's own
+ *     block t / l', whose keys u <= t are attended;
+ *   - scale as in nsa_prefill (plan softmax_scale, else 1/sqrt(D)).
+ * The plan's sel_block (l'), top_n (n, the own block included), head
+ * geometry, scale and out_dtype are used; cmp_block, cmp_stride and window
+ * are not.
+ *   q          [T_total, Hq, D]  bf16
+ *   k, v       [T_total, Hkv, D] bf16
+ *   cu_seqlens [batch + 1]       int32 device, as in nsa_prefill
+ *   out        [T_total, Hq, D]  bf16 or fp32 (plan out_dtype)
+ *   k_mean     [nsa_block_rows, Hkv, D] bf16, written: the routing keys of
+ *              sequence b's floor(T_b / l') complete blocks follow those of the
+ *              sequences before it; remaining rows are zero-filled
+ *   sel_idx    [T_total, Hkv, top_n] int32 or NULL: attended blocks of each
+ *              token, ascending (the own block last), -1 padded
+ *   workspace  >= nsa_workspace_size(plan, NSA_MODE_BLOCK_SELECT) bytes,
+ *              256-byte aligned (regions NSA_WS_STATUS, NSA_WS_SCORES = fp32
+ *              [T_total, Hkv, max_seqlen / l'] routing scores, entry j of row t
+ *              defined for j < t / l', and NSA_WS_SEL)
+ * Returns the same codes as nsa_prefill; device-side faults land in the
+ * workspace status word (nsa_read_device_status).  Five launches.
+ */
+int nsa_block_select_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,
+                             const int* cu_seqlens, int batch, int total_tokens, void* out,
+                             void* k_mean, int* sel_idx, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Rows of the packed routing-key output of nsa_block_select_prefill over
+ * `total_tokens` tokens: floor(total_tokens / l'). */
+int nsa_block_rows(nsa_plan_t plan, int total_tokens);
+
 /* Synchronises `stream`, returns the device status word of the last call that
  * used `workspace` (NSA_OK or NSA_ERR_DEVICE_*), and clears it.  Meant for
  * tests and debugging; returns NSA_ERR_CUDA if the stream itself failed. */
@@ -231,7 +279,7 @@ int nsa_selftest_timeout(void* workspace, size_t workspace_bytes, long long cycl
                          void* stream);
 
 /* Per-launch timing for benchmarks.  While enabled on the calling thread,
- * nsa_prefill / nsa_decode record a CUDA event on the call's stream before
+ * nsa_prefill / nsa_block_select_prefill / nsa_decode record a CUDA event on the call's stream before
  * each kernel launch and after the last one (the library owns the events).
  * nsa_profile_stage_ms synchronises the last profiled call's events and
  * writes up to `max_stages` per-launch durations in milliseconds, in launch
@@ -244,7 +292,7 @@ int nsa_profile_stage_ms(float* ms, int max_stages);
 const char* nsa_strerror(int status);
 
 /* Number of kernel launches made by the last successful nsa_prefill /
- * nsa_decode call on this thread (for launch accounting in benchmarks). */
+ * nsa_block_select_prefill / nsa_decode call on this thread (for launch accounting in benchmarks). */
 int nsa_last_launch_count(void);
 
 #ifdef __cplusplus

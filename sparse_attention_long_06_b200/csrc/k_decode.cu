@@ -143,7 +143,9 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // in flight before one wait.
 template <int kMaxChunks, typename Op>
 __device__ __forceinline__ void sweep_chunks(uint32_t lane_addr, uint32_t col, int nchunks, Op op) {
-#pragma unroll
+  // not unrolled: a one-shot decode CTA pays for every instruction fetch, and
+  // one group of four chunks is already a long straight run of code
+#pragma unroll 1
   for (int c0 = 0; c0 < kMaxChunks; c0 += 4) {
     if (c0 >= nchunks) break;
     float v[64];
@@ -302,7 +304,7 @@ __global__ void __launch_bounds__(kDecThreads)
   const uint32_t sbase = smem_u32(sm);
   int* status = a.status;
   const int G = a.geo.G, n = a.geo.n;
-  const int b = P.b, g = P.g, t = P.t;
+  const int b = P.b, g = P.g;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -792,12 +794,16 @@ __global__ void __launch_bounds__(kDecThreads)
         if (u2 < ncv)
           vc[u2] = __ldcg(reinterpret_cast<const float4*>(rec.cmp + ((size_t)u2 * G + h) * D + c4));
       // softmax partials (row maximum m, sum, unnormalised O) -> normalised O
-      auto merge = [&](const float* mlv, const float4* v, int units_of, int max_units) {
+      auto merge = [&](const float* mlv, const auto& v, int units_of) {
+        constexpr int kMax = sizeof(v) / sizeof(float4);  // unrolled: v stays in registers
         float M = -INFINITY;
-        for (int s2 = 0; s2 < units_of; ++s2) M = fmaxf(M, mlv[s2 * 32 + h]);
+#pragma unroll
+        for (int s2 = 0; s2 < kMax; ++s2)
+          if (s2 < units_of) M = fmaxf(M, mlv[s2 * 32 + h]);
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
         float ls = 0.f;
-        for (int s2 = 0; s2 < max_units; ++s2) {
+#pragma unroll
+        for (int s2 = 0; s2 < kMax; ++s2) {
           if (s2 >= units_of) break;
           const float ms = mlv[s2 * 32 + h];
           const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : ex2(ms - M);
@@ -810,8 +816,8 @@ __global__ void __launch_bounds__(kDecThreads)
         const float inv = ls > 0.f ? 1.f / ls : 0.f;
         return make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
       };
-      const float4 os = merge(ml, vs, a.nsl, kMaxSlcUnits);
-      const float4 ow = merge(wml, vw, a.nwu, kMaxWinUnits);
+      const float4 os = merge(ml, vs, a.nsl);
+      const float4 ow = merge(wml, vw, a.nwu);
       float4 oc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u2 = 0; u2 < kMaxCmpUnits; ++u2) {

@@ -160,7 +160,9 @@ cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s) {
 // One warp per (token, KV group); the selection itself is warp_topn.  With
 // l == d == l' the candidates' scores are the compressed-block scores; else
 // each selection block's score is first summed from the compressed blocks
-// that overlap it (written to the selection-score table, then ranked).
+// that overlap it (written to the selection-score table, then ranked).  In
+// select-only block attention the scores are routing scores and the query's
+// own block is always taken.
 __global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
@@ -174,8 +176,26 @@ __global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   const int t = tg - __ldg(a.cu + b);
   const float* S = a.scores + ((size_t)tg * H + g) * a.geo.cmp_cap;
   int* out = a.sel + ((size_t)tg * H + g) * n;
-  const int ncmp = num_cmp_blocks(t + 1, a.geo.l, a.geo.d), ncand = t / a.geo.ls + 1;
   auto put = [&](int i, int j) { out[i] = j; };
+  if (a.select_only) {
+    // select-only block attention: the n - 1 best of the complete blocks
+    // before t's own block (routing scores), then the own block, which has
+    // the largest index, last
+    const int cur = t >> a.geo.lg_ls, m = n - 1;
+    if (m > 0) {
+      auto score = [&](int j) { return S[j]; };
+      if (!(cur <= 1024 && m <= 32 && warp_topn_regs(score, cur, cur, m, cand_all[warp], put)))
+        warp_topn(score, cur, cur, m, hist_all[warp], put);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      const int taken = cur < m ? cur : m;
+      out[taken] = cur;
+      for (int i = taken + 1; i < n; ++i) out[i] = -1;
+    }
+    return;
+  }
+  const int ncmp = num_cmp_blocks(t + 1, a.geo.l, a.geo.d), ncand = t / a.geo.ls + 1;
   if (!a.geo.remap) {
     auto score = [&](int j) { return S[j]; };
     if (ncand <= 1024 && n <= 32 && warp_topn_regs(score, ncmp, ncand, n, cand_all[warp], put))

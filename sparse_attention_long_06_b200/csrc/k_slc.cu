@@ -383,18 +383,21 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       }
     };
     // output of job j (thread = channel r < D): g_cmp O_cmp + g_slc O_slc / sum + g_win O_win
+    // (O_slc / sum alone in select-only block attention)
     auto epilogue = [&](int j) {
       const SlcJob jb = slc_job(a, blockIdx.x + (long long)j * gridDim.x);
       const int os = j & 3;
       float oc[16], ow[16], g0[16], g1[16];
+      const bool gated = !a.select_only;  // select-only: out = O_slc
 #pragma unroll
       for (int h = 0; h < 16; ++h) {
         const bool v = r < D && h < G;
+        const bool vg = v && gated;
         const size_t gh = (size_t)jb.row * Hq + jb.g * G + h;
-        oc[h] = v ? a.o_cmp[gh * D + r] : 0.f;
-        ow[h] = v ? a.o_win[gh * D + r] : 0.f;
-        g0[h] = v ? __ldg(a.gates + gh * 3 + 0) : 0.f;
-        g1[h] = v ? __ldg(a.gates + gh * 3 + 1) : 0.f;
+        oc[h] = vg ? a.o_cmp[gh * D + r] : 0.f;
+        ow[h] = vg ? a.o_win[gh * D + r] : 0.f;
+        g0[h] = vg ? __ldg(a.gates + gh * 3 + 0) : 0.f;
+        g1[h] = vg ? __ldg(a.gates + gh * 3 + 1) : (v ? 1.f : 0.f);
       }
       mbar_wait(o_full + os, (j >> 2) & 1, abort_flag, status, kWaitCycles);
       tc_fence_after();
@@ -435,7 +438,7 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       // the epilogue of job j (one job from now) reads its G rows of O_cmp
       // and g_win O_win from HBM: bring them into L2 now, one 128-byte line
       // per thread (G * D * 4 bytes each)
-      if (jb.valid) {
+      if (jb.valid && !a.select_only) {
         const size_t base = ((size_t)jb.row * Hq + jb.g * G) * D;
         const int lines = (G * D * 4) >> 7;
         if (r < lines) {

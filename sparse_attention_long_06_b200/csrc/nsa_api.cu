@@ -71,6 +71,41 @@ PrefillLayout prefill_layout(const nsa_plan_s* pl) {
   return L;
 }
 
+// Select-only block attention: the plan's geometry with blocks of l' tokens
+// as the pooled (routing) blocks; the score table holds max_seqlen / l'
+// routing scores per (token, group).
+Geometry block_select_geometry(const nsa_plan_s* pl) {
+  Geometry g = pl->geo;
+  g.l = g.ls;
+  g.d = g.ls;
+  g.remap = 0;
+  g.cmp_cap = pl->p.max_seqlen / g.ls > 0 ? pl->p.max_seqlen / g.ls : 1;
+  return g;
+}
+
+struct BlockSelectLayout {
+  size_t meta, scores, sel, total;
+};
+
+BlockSelectLayout block_select_layout(const nsa_plan_s* pl) {
+  const nsa_params& p = pl->p;
+  const Geometry g = block_select_geometry(pl);
+  const size_t T = (size_t)p.max_total_tokens;
+  BlockSelectLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  take(kHeaderBytes);
+  L.meta = take(sizeof(Meta) + 2 * sizeof(int) * ((size_t)p.max_batch + 1));
+  L.scores = take(T * g.Hkv * (size_t)g.cmp_cap * sizeof(float));
+  L.sel = take(T * g.Hkv * (size_t)g.n * sizeof(int));
+  L.total = off;
+  return L;
+}
+
 struct DecodeLayout {
   size_t counters, sel, pt, win, cmp, slc, total;
   int ncc_max, ncv_max, nsl, nwu;
@@ -294,11 +329,25 @@ size_t nsa_workspace_size(nsa_plan_t plan, int mode) {
     const int cap = plan->p.max_seqlen / unit * unit;
     return decode_layout(plan, plan->p.max_batch, cap).total;
   }
+  if (mode == NSA_MODE_BLOCK_SELECT) return block_select_layout(plan).total;
   return 0;
 }
 
 int nsa_workspace_region(nsa_plan_t plan, int mode, int region, size_t* offset, size_t* bytes) {
-  if (!plan || !offset || !bytes || mode != NSA_MODE_PREFILL) return NSA_ERR_INVALID_ARG;
+  if (!plan || !offset || !bytes) return NSA_ERR_INVALID_ARG;
+  if (mode == NSA_MODE_BLOCK_SELECT) {
+    const BlockSelectLayout L = block_select_layout(plan);
+    const Geometry g = block_select_geometry(plan);
+    const size_t T = (size_t)plan->p.max_total_tokens;
+    switch (region) {
+      case NSA_WS_STATUS: *offset = 0; *bytes = sizeof(int); break;
+      case NSA_WS_SCORES: *offset = L.scores; *bytes = T * g.Hkv * (size_t)g.cmp_cap * sizeof(float); break;
+      case NSA_WS_SEL: *offset = L.sel; *bytes = T * g.Hkv * (size_t)g.n * sizeof(int); break;
+      default: return NSA_ERR_INVALID_ARG;
+    }
+    return NSA_OK;
+  }
+  if (mode != NSA_MODE_PREFILL) return NSA_ERR_INVALID_ARG;
   const PrefillLayout L = prefill_layout(plan);
   const Geometry& g = plan->geo;
   const size_t T = (size_t)plan->p.max_total_tokens;
@@ -419,6 +468,92 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   prof_mark(s);
   if (e != cudaSuccess) {
     fprintf(stderr, "nsa_prefill: launch failed: %s\n", cudaGetErrorString(e));
+    return NSA_ERR_CUDA;
+  }
+  g_last_launches = launches + 1;
+  return NSA_OK;
+}
+
+int nsa_block_rows(nsa_plan_t plan, int total_tokens) {
+  if (!plan || total_tokens < 0) return -1;
+  return total_tokens / plan->geo.ls;
+}
+
+int nsa_block_select_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,
+                             const int* cu_seqlens, int batch, int total_tokens, void* out,
+                             void* k_mean, int* sel_idx, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  g_last_launches = 0;
+  if (!plan) return NSA_ERR_INVALID_ARG;
+  const nsa_params& p = plan->p;
+  const Geometry geo = block_select_geometry(plan);
+  if (batch <= 0 || batch > p.max_batch || total_tokens < 0 ||
+      total_tokens > p.max_total_tokens)
+    return NSA_ERR_INVALID_ARG;
+  if (!cu_seqlens || !workspace) return workspace ? NSA_ERR_INVALID_ARG : NSA_ERR_WORKSPACE;
+  const BlockSelectLayout L = block_select_layout(plan);
+  if (workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return NSA_ERR_WORKSPACE;
+  const int rows = total_tokens / geo.ls;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !out) return NSA_ERR_INVALID_ARG;
+    if (rows > 0 && !k_mean) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (rows > 0 && !aligned16(k_mean)) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(sel_idx) & 3u))
+      return NSA_ERR_MISALIGNED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  PrefillArgs a{};
+  a.geo = geo;
+  a.batch = batch;
+  a.total_tokens = total_tokens;
+  a.cmp_rows = rows;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.cu = cu_seqlens;
+  a.out = out;
+  a.k_cmp = static_cast<uint16_t*>(k_mean);
+  a.status = reinterpret_cast<int*>(ws);
+  a.meta = reinterpret_cast<Meta*>(ws + L.meta);
+  a.cmp_off = reinterpret_cast<int*>(ws + L.meta + sizeof(Meta));
+  a.tile_off = a.cmp_off + (batch + 1);
+  a.scores = reinterpret_cast<float*>(ws + L.scores);
+  a.sel = sel_idx ? sel_idx : reinterpret_cast<int*>(ws + L.sel);
+  a.select_only = 1;
+
+  if (cudaMemsetAsync(a.status, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
+  if (total_tokens == 0) {
+    if (cudaMemsetAsync(a.meta, 0, sizeof(Meta), s) != cudaSuccess) return NSA_ERR_CUDA;
+    return NSA_OK;
+  }
+  PrefillMaps m;
+  memset(&m, 0, sizeof(m));
+  bool ok = encode3d(&m.q, q, geo.D, geo.Hq, total_tokens, geo.G, geo.tpt) &&
+            encode3d(&m.q_tok, q, geo.D, geo.Hq, total_tokens, geo.Hq < 16 ? geo.Hq : 16, 1) &&
+            encode3d(&m.kc, k_mean, geo.D, geo.Hkv, rows, 1, kChunk) &&
+            encode3d(&m.k_blk, k, geo.D, geo.Hkv, total_tokens, 1, geo.ls) &&
+            encode3d(&m.v_blk, v, geo.D, geo.Hkv, total_tokens, 1, geo.ls);
+  if (!ok) return NSA_ERR_CUDA;
+  a.split_q = geo.Hq >= 16 && encode_split4d(&m.q_split, q, geo.D, geo.Hq, total_tokens, false, 16);
+  a.split_v = geo.ls == 64 && encode_split4d(&m.v_split, v, geo.D, geo.Hkv, total_tokens, true, 64);
+  const int sms = num_sms_current();
+  if (sms <= 0) return NSA_ERR_CUDA;
+
+  int launches = 0;
+  prof_reset();
+  prof_mark(s);
+  cudaError_t e = launch_meta(a, s);
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_block_mean(a, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_block_score(a, m, sms, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_topn(a, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_slc(a, m, sms, s); }
+  prof_mark(s);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "nsa_block_select_prefill: launch failed: %s\n", cudaGetErrorString(e));
     return NSA_ERR_CUDA;
   }
   g_last_launches = launches + 1;

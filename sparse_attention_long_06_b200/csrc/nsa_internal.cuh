@@ -76,6 +76,8 @@ struct PrefillArgs {
   float* scores;  // [T, Hkv, cmp_cap]
   float* sel_scores;  // [T, Hkv, sel_cap] selection-block scores (remap only)
   float* o_win;   // [T, Hq, D] g_win * O_win
+  int select_only;  // select-only block attention: routing scores, the own
+                    // block forced into the selection, output = selected branch
   int split_q;    // PrefillMaps.q_split is valid (Hq >= 16)
   int split_v;    // PrefillMaps.v_split is valid (l' = 64)
 };
@@ -189,6 +191,9 @@ cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int num_
 cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_win(const PrefillArgs& a, const PrefillMaps& m, int num_sms, cudaStream_t s);
 cudaError_t launch_slc(const PrefillArgs& a, const PrefillMaps& m, int num_sms, cudaStream_t s);
+cudaError_t launch_block_mean(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_block_score(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
+                               cudaStream_t s);
 cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s);
 cudaError_t launch_decode_compress(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_a(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);

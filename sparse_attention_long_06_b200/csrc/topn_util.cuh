@@ -4,14 +4,23 @@
 // Candidates are blocks j < ncand; the complete ones (j < ncmp) carry their
 // score, the incomplete block holding the query competes with score 0.  The
 // n largest under (score descending, index ascending) are found by an 8-bit
-// radix select on the score bits (scores are non-negative, so their bit
-// patterns order like the values), followed by taking the lowest-index ties
-// at the threshold.  The result is written in ascending block order, padded
-// with -1.
+// radix select on an order-preserving 32-bit key of each score, followed by
+// taking the lowest-index ties at the threshold.  The result is written in
+// ascending block order, padded with -1.
 #pragma once
 #include <cstdint>
 
 namespace nsa {
+
+// Order-preserving key of an fp32 score: larger score, larger key; -0 and +0
+// share a key (they compare equal); non-negative scores keep their bit
+// pattern with the top bit set, negative ones are bit-inverted.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t b = __float_as_uint(s);
+  b = (b == 0x80000000u) ? 0u : b;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+constexpr uint32_t kZeroScoreKey = 0x80000000u;  // score_key(0.f)
 
 // `score(j)` returns the fp32 score of complete block j; `hist` is 256
 // words of warp-private shared memory; `out(i, j)` stores result i.
@@ -20,7 +29,7 @@ __device__ __forceinline__ void warp_topn(ScoreFn score, int ncmp, int ncand, in
                                           unsigned* hist, OutFn out) {
   const int lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
-  auto bits = [&](int j) -> uint32_t { return j < ncmp ? __float_as_uint(score(j)) : 0u; };
+  auto bits = [&](int j) -> uint32_t { return j < ncmp ? score_key(score(j)) : kZeroScoreKey; };
   if (ncand <= n) {
     for (int j = lane; j < n; j += 32) out(j, j < ncand ? j : -1);
     return;
@@ -100,7 +109,7 @@ __device__ __forceinline__ void warp_topn(ScoreFn score, int ncmp, int ncand, in
 }
 
 // Register path of the same selection for rows with at most 1024 candidates
-// (32 per lane).  Every candidate j gets the 64-bit key (score bits << 32) |
+// (32 per lane).  Every candidate j gets the 64-bit key (score key << 32) |
 // (0xFFFFFFFF - j), so larger keys rank first and equal scores rank by lower
 // index; keys are distinct.  The n-th largest of the 32 per-lane maxima is a
 // lower bound T0 of the n-th largest key (n lanes hold a key >= it); the keys
@@ -124,7 +133,7 @@ __device__ __forceinline__ bool warp_topn_regs(ScoreFn score, int ncmp, int ncan
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int j = lane + 32 * i;
-    const uint32_t b = j < ncmp ? __float_as_uint(score(j)) : 0u;
+    const uint32_t b = j < ncmp ? score_key(score(j)) : kZeroScoreKey;
     key[i] = j < ncand ? (((unsigned long long)b << 32) | (0xFFFFFFFFu - (uint32_t)j)) : 0ull;
     lmax = key[i] > lmax ? key[i] : lmax;
   }
@@ -193,7 +202,7 @@ __device__ __forceinline__ bool warp_topn_reread(ScoreFn score, int ncmp, int nc
     return true;
   }
   auto key = [&](int j) -> unsigned long long {
-    const uint32_t b = j < ncmp ? __float_as_uint(score(j)) : 0u;
+    const uint32_t b = j < ncmp ? score_key(score(j)) : kZeroScoreKey;
     return ((unsigned long long)b << 32) | (0xFFFFFFFFu - (uint32_t)j);
   };
   unsigned long long lmax = 0;

@@ -23,14 +23,15 @@ NSA_ERR_CUDA = 5
 NSA_ERR_DEVICE_TIMEOUT = 6
 NSA_ERR_DEVICE_BAD_INPUT = 7
 OUT_BF16, OUT_F32 = 0, 1
-MODE_PREFILL, MODE_DECODE = 0, 1
+MODE_PREFILL, MODE_DECODE, MODE_BLOCK_SELECT = 0, 1, 2
 WS_STATUS, WS_O_CMP, WS_LSE, WS_SCORES, WS_SEL, WS_WIN, WS_SEL_SCORES = 0, 1, 2, 3, 4, 5, 6
 
 EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_workspace_region",
             "nsa_cmp_rows", "nsa_prefill", "nsa_decode", "nsa_read_device_status",
             "nsa_selftest_timeout", "nsa_strerror", "nsa_last_launch_count",
             "nsa_profile_enable", "nsa_profile_stage_ms", "nsa_prefill_noalloc",
-            "nsa_plan", "nsa_noalloc_read_device_status"]
+            "nsa_plan", "nsa_noalloc_read_device_status", "nsa_block_select_prefill",
+            "nsa_block_rows"]
 
 
 class NsaError(RuntimeError):
@@ -79,6 +80,10 @@ def lib():
             L.nsa_prefill.restype = i
             L.nsa_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp]
             L.nsa_prefill_noalloc.restype = i
+            L.nsa_block_select_prefill.argtypes = [vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, sz, vp]
+            L.nsa_block_select_prefill.restype = i
+            L.nsa_block_rows.argtypes = [vp, i]
+            L.nsa_block_rows.restype = i
             L.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
             L.nsa_decode.restype = i
             L.nsa_read_device_status.argtypes = [vp, vp]
@@ -189,6 +194,23 @@ class Plan:
                                        _ptr(out), _ptr(k_cmp), _ptr(v_cmp), _ptr(sel_idx),
                                        _stream(stream))
         _check(rc, "nsa_prefill_noalloc")
+
+    def block_rows(self, total_tokens: int) -> int:
+        return int(lib().nsa_block_rows(self.handle, total_tokens))
+
+    def block_select_prefill(self, q, k, v, cu_seqlens, out, k_mean, workspace, sel_idx=None,
+                             stream=None):
+        """Select-only block attention over a packed batch (the own block plus
+        the n - 1 best-routed earlier blocks of l' tokens); workspace of
+        workspace_size(MODE_BLOCK_SELECT) bytes."""
+        batch = cu_seqlens.numel() - 1
+        total = q.shape[0]
+        rc = lib().nsa_block_select_prefill(self.handle, _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(cu_seqlens), batch, total, _ptr(out),
+                                            _ptr(k_mean), _ptr(sel_idx), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(stream))
+        _check(rc, "nsa_block_select_prefill")
 
     def decode(self, q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, seqlens, gates, w_k, w_v,
                out, workspace, sel_idx=None, stream=None):

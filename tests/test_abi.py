@@ -162,6 +162,44 @@ def test_decode_rejects_bad_arguments_before_launch(L):
     assert L.nsa_last_launch_count() == 0
 
 
+def test_block_select_sizes_and_bad_arguments(L):
+    p = nsa.Plan(**_params(max_total_tokens=4096, max_seqlen=4096))
+    T, Hkv, n = 4096, 4, 16
+    wsb = p.workspace_size(nsa.MODE_BLOCK_SELECT)
+    # status + metadata, routing scores [T, Hkv, max_seqlen / l'], selection
+    assert wsb >= T * Hkv * (4096 // 64) * 4 + T * Hkv * n * 4
+    assert wsb < p.workspace_size(nsa.MODE_PREFILL)
+    assert p.workspace_region(nsa.WS_SCORES, nsa.MODE_BLOCK_SELECT)[1] == T * Hkv * 64 * 4
+    assert p.workspace_region(nsa.WS_SEL, nsa.MODE_BLOCK_SELECT)[1] == T * Hkv * n * 4
+    with pytest.raises(nsa.NsaError):
+        p.workspace_region(nsa.WS_O_CMP, nsa.MODE_BLOCK_SELECT)
+    assert p.block_rows(4096) == 64 and p.block_rows(100) == 1 and p.block_rows(63) == 0
+    fake = 1 << 20  # an aligned address that is never dereferenced
+    args = dict(q=fake, k=fake, v=fake, cu=fake, batch=1, total=4096, out=fake, km=fake,
+                sel=None, ws=fake, wsb=wsb)
+
+    def call(**over):
+        a = dict(args)
+        a.update(over)
+        return L.nsa_block_select_prefill(p.handle, a["q"], a["k"], a["v"], a["cu"], a["batch"],
+                                          a["total"], a["out"], a["km"], a["sel"], a["ws"],
+                                          a["wsb"], None)
+
+    assert call(q=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(km=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(total=4097) == nsa.NSA_ERR_INVALID_ARG
+    assert call(ws=None) == nsa.NSA_ERR_WORKSPACE
+    assert call(wsb=wsb - 1) == nsa.NSA_ERR_WORKSPACE
+    assert call(ws=fake + 16) == nsa.NSA_ERR_WORKSPACE
+    assert call(v=fake + 2) == nsa.NSA_ERR_MISALIGNED
+    assert call(km=fake + 8) == nsa.NSA_ERR_MISALIGNED
+    assert call(sel=fake + 2) == nsa.NSA_ERR_MISALIGNED
+    assert L.nsa_block_select_prefill(None, fake, fake, fake, fake, 1, 1, fake, fake, None, fake,
+                                      wsb, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_last_launch_count() == 0
+
+
 def test_noalloc_rejects_plans_beyond_its_static_array(L):
     big = nsa.Plan(**_params())  # 64k tokens: several GB of workspace
     assert big.workspace_size() > 32 << 20
