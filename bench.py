@@ -36,12 +36,13 @@ sys.path.insert(0, ROOT)
 from sparse_attention_long_06_b200 import workloads as wl  # noqa: E402
 
 METRIC = "NSA prefill tokens/s"
-KERNEL_NAMES = ["nsa_meta_kernel", "nsa_compress_kernel", "nsa_cmp_attn_kernel",
-                "nsa_topn_kernel", "nsa_win_kernel", "nsa_slc_kernel"]
+KERNEL_NAMES = ["nsa_meta_kernel", "nsa_weight_split_kernel", "nsa_compress_tc_kernel",
+                "nsa_cmp_attn_kernel", "nsa_topn_kernel", "nsa_win_kernel", "nsa_slc_kernel"]
 # tensor-core kernels: (stage index, source file, algorithmic FLOP key)
-TENSOR_KERNELS = {"nsa_cmp_attn_kernel": (2, "k_cmp.cu", "cmp"),
-                  "nsa_win_kernel": (4, "k_win.cu", "win"),
-                  "nsa_slc_kernel": (5, "k_slc.cu", "slc")}
+TENSOR_KERNELS = {"nsa_compress_tc_kernel": (2, "k_compress.cu", "compress"),
+                  "nsa_cmp_attn_kernel": (3, "k_cmp.cu", "cmp"),
+                  "nsa_win_kernel": (5, "k_win.cu", "win"),
+                  "nsa_slc_kernel": (6, "k_slc.cu", "slc")}
 
 
 def _peaks():

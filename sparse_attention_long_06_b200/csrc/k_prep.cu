@@ -1,10 +1,6 @@
-// Small prefill kernels: per-call metadata, block compression (step 1) and
-// top-n block selection (step 4).
+// Small prefill kernels: per-call metadata and top-n block selection
+// (step 4; block compression, step 1, is in k_compress.cu).
 //
-// Compression follows the NSA pages: "DeepSeek NSA config.toml" page,
-// section 3 (compress_block_size) and "DeepSeek NSA in manufacturing" page,
-// section on what dynamic sparsity sparsifies (each block is flattened and
-// mapped by one learned linear layer to a single compressed token).
 // Selection follows the config page, section 3 (select_top_k), and the
 // manufacturing page, same section (the highest-scoring blocks are kept);
 // the selection itself is in topn_util.cuh.
@@ -49,113 +45,6 @@ cudaError_t launch_meta(const PrefillArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ compression
-// Kc[r, h, c] = sum_{p < l, c' < D} W[h, c, p*D + c'] * X[tok0(r) + p, h, c']
-// for every complete block r of every sequence (tok0 = first token of the
-// block: the sequence start plus d times the block's index in it).  A tiled fp32 GEMM: CTA tile 32 blocks x D outputs, k-step 32.
-// Rows in [cmp_total, cmp_rows) are zero-filled so that later tiles reading
-// past the last sequence see finite values.
-template <int D>
-__global__ void __launch_bounds__(256) nsa_compress_kernel(PrefillArgs a) {
-  if (a.meta->bad) return;
-  constexpr int BM = 32, BK = 32, TN = D / 32;
-  const int l = a.geo.l, H = a.geo.Hkv;
-  const int h = blockIdx.y;
-  const bool is_v = blockIdx.z != 0;
-  const uint16_t* X = is_v ? a.v : a.k;
-  const float* W = (is_v ? a.w_v : a.w_k) + (size_t)h * D * l * D;
-  uint16_t* out = is_v ? a.v_cmp : a.k_cmp;
-  const int C = a.meta->cmp_total;
-  const int r0 = blockIdx.x * BM;
-  if (r0 >= a.cmp_rows) return;
-
-  __shared__ int tok0[BM];
-  __shared__ float As[BK][BM + 4];
-  __shared__ float Ws[BK][D + 4];
-  const int tid = threadIdx.x;
-  if (tid < BM) {
-    const int r = r0 + tid;
-    int t0 = -1;
-    if (r < C) {
-      const int b = seq_of_offset(a.cmp_off, a.batch, r);
-      t0 = __ldg(a.cu + b) + (r - a.cmp_off[b]) * a.geo.d;
-    }
-    tok0[tid] = t0;
-  }
-  __syncthreads();
-
-  const int ty = tid / 32, tx = tid % 32;  // rows ty*4..+4, cols tx*TN..+TN
-  float acc[4][TN];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
-
-  const int K = l * D;
-  for (int k0 = 0; k0 < K; k0 += BK) {
-    const int p = k0 / D, c0 = k0 % D;
-    {  // A tile: 32 rows x 32 k, 4 consecutive k per thread
-      const int row = tid / 8, kk = (tid % 8) * 4;
-      const int t0 = tok0[row];
-      float v4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (t0 >= 0) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(X + ((size_t)(t0 + p) * H + h) * D + c0 + kk);
-        v4[0] = __uint_as_float(raw.x << 16);
-        v4[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-        v4[2] = __uint_as_float(raw.y << 16);
-        v4[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) As[kk + j][row] = v4[j];
-    }
-#pragma unroll
-    for (int it = 0; it < D * BK / 4 / 256; ++it) {  // W tile: D rows x 32 k
-      const int idx = it * 256 + tid;
-      const int c = idx / 8, kq = (idx % 8) * 4;
-      const float4 w4 = __ldg(reinterpret_cast<const float4*>(W + (size_t)c * K + k0 + kq));
-      Ws[kq + 0][c] = w4.x;
-      Ws[kq + 1][c] = w4.y;
-      Ws[kq + 2][c] = w4.z;
-      Ws[kq + 3][c] = w4.w;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < BK; ++kk) {
-      float av[4], bv[TN];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < TN; ++j) bv[j] = Ws[kk][tx * TN + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = r0 + ty * 4 + i;
-    if (r >= a.cmp_rows) continue;
-    const bool live = r < C;
-#pragma unroll
-    for (int j = 0; j < TN; ++j) {
-      const __nv_bfloat16 bv = __float2bfloat16_rn(live ? acc[i][j] : 0.f);
-      out[((size_t)r * H + h) * D + tx * TN + j] = *reinterpret_cast<const uint16_t*>(&bv);
-    }
-  }
-}
-
-cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s) {
-  if (a.cmp_rows <= 0) return cudaSuccess;
-  dim3 grid((a.cmp_rows + 31) / 32, a.geo.Hkv, 2);
-  if (a.geo.D == 128)
-    nsa_compress_kernel<128><<<grid, 256, 0, s>>>(a);
-  else
-    nsa_compress_kernel<64><<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
 // ------------------------------------------------------------------ top-n
 // One warp per (token, KV group); the selection itself is warp_topn.  With
 // l == d == l' the candidates' scores are the compressed-block scores; else
@@ -163,7 +52,7 @@ cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s) {
 // that overlap it (written to the selection-score table, then ranked).  In
 // select-only block attention the scores are routing scores and the query's
 // own block is always taken.
-__global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(256, 3) nsa_topn_kernel(PrefillArgs a) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
   __shared__ unsigned long long cand_all[8][kTopnCand];

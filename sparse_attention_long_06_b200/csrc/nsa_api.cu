@@ -45,8 +45,13 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 bool is_pow2_le16(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
 
 struct PrefillLayout {
-  size_t meta, o_cmp, lse, scores, sel_scores, sel, o_win, total;
+  size_t meta, o_cmp, lse, scores, sel_scores, sel, o_win, wplanes, total;
 };
+
+// bf16 terms of the compressor weights: [tensor][term][Hkv][D][l D]
+size_t weight_plane_bytes(const Geometry& g) {
+  return (size_t)2 * 3 * g.Hkv * g.D * (size_t)g.l * g.D * 2;
+}
 
 PrefillLayout prefill_layout(const nsa_plan_s* pl) {
   const nsa_params& p = pl->p;
@@ -67,6 +72,7 @@ PrefillLayout prefill_layout(const nsa_plan_s* pl) {
   L.sel_scores = take(g.remap ? T * g.Hkv * (size_t)g.sel_cap * sizeof(float) : 0);
   L.sel = take(T * g.Hkv * (size_t)g.n * sizeof(int));
   L.o_win = take(T * g.Hq * g.D * sizeof(float));
+  L.wplanes = take(weight_plane_bytes(g));
   L.total = off;
   return L;
 }
@@ -215,6 +221,20 @@ bool encode_split4d(CUtensorMap* m, const void* base, int D, int heads, long lon
   cuuint32_t box[4] = {64, (cuuint32_t)box_inner, (cuuint32_t)(D / 64), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor (inner `cols`, outer `rows`), 128-byte swizzled box (64, box_rows).
+bool encode2d(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows) {
+  memset(m, 0, sizeof(*m));
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -441,7 +461,8 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
             encode3d(&m.k_blk, k, geo.D, geo.Hkv, total_tokens, 1, geo.ls) &&
             encode3d(&m.v_blk, v, geo.D, geo.Hkv, total_tokens, 1, geo.ls) &&
             encode3d(&m.k_win, k, geo.D, geo.Hkv, total_tokens, 1, kChunk) &&
-            encode3d(&m.v_win, v, geo.D, geo.Hkv, total_tokens, 1, kChunk);
+            encode3d(&m.v_win, v, geo.D, geo.Hkv, total_tokens, 1, kChunk) &&
+            encode2d(&m.wpl, ws + L.wplanes, (long long)geo.l * geo.D, 6LL * geo.Hkv * geo.D, 64);
   if (!ok) return NSA_ERR_CUDA;
   // one-copy query rows (16 heads) and one-copy V blocks (64 keys), when the
   // driver accepts the channel-split maps
@@ -460,7 +481,12 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   prof_reset();
   prof_mark(s);
   cudaError_t e = launch_meta(a, s);
-  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_compress(a, s); }
+  if (e == cudaSuccess) {
+    ++launches;
+    prof_mark(s);
+    e = launch_weight_split(a, reinterpret_cast<uint16_t*>(ws + L.wplanes), s);
+  }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_compress_tc(a, m, sms, s); }
   if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_cmp_attn(a, m, sms, s); }
   if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_topn(a, s); }
   if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_win(a, m, sms, s); }

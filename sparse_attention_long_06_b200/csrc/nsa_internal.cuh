@@ -93,6 +93,7 @@ struct PrefillMaps {
   CUtensorMap v_blk;
   CUtensorMap k_win;  // (D, Hkv, T) box (64, 1, 128)
   CUtensorMap v_win;
+  CUtensorMap wpl;    // (l D, 2 x 3 x Hkv x D) box (64, 64): the bf16 weight terms
 };
 
 struct DecodeArgs {
@@ -185,7 +186,9 @@ __device__ __forceinline__ int seq_of_offset(const int* off, int B, int x) {
 
 // ---------------------------------------------------------------- launchers
 cudaError_t launch_meta(const PrefillArgs& a, cudaStream_t s);
-cudaError_t launch_compress(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_weight_split(const PrefillArgs& a, uint16_t* planes, cudaStream_t s);
+cudaError_t launch_compress_tc(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
+                               cudaStream_t s);
 cudaError_t launch_cmp_attn(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
                             cudaStream_t s);
 cudaError_t launch_topn(const PrefillArgs& a, cudaStream_t s);

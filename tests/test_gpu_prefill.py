@@ -43,6 +43,8 @@ def _assert_report(rep, res=None, e2e=True, name="prefill"):
     assert rep["kc_bound_fail"] == 0
     assert rep["kc_total"] == 0 or rep["kc_diff"] / rep["kc_total"] < 0.01
     assert rep["idx_bad_stageB"] == 0
+    # only rows with an exempt near-tie group are left out of the output check
+    assert rep.get("out_rows_skipped", 0) <= rep["idx_exempt"]
     assert rep["max_abs"] <= 1e-2
     if res is not None and "out_bf16" in res:
         assert res["status_bf16"] == nsa.NSA_OK
@@ -64,7 +66,7 @@ def test_tiny_config_all_rows():
     inputs = wl.prefill_inputs(cfg)
     res = gu.run_prefill(cfg, inputs, both_dtypes=True)
     assert res["status"] == nsa.NSA_OK
-    assert res["launches"] == 6
+    assert res["launches"] == 7
     rep = gu.check_prefill(cfg, inputs, res, [np.arange(1024, dtype=np.int32)])
     _assert_report(rep, res, name="tiny")
 
