@@ -729,7 +729,8 @@ def main():
         res = run_decode_leg(args, torch.device("cuda", torch.cuda.current_device()), world)
     elif args.block_select_only:
         res = run_block_select_leg(torch.device("cuda", torch.cuda.current_device()), world,
-                                   steps=max(args.steps, 3), warmup=args.warmup)
+                                   steps=max(args.steps, 3), warmup=args.warmup,
+                                   name=args.workload)
     else:
         res = run_ours(args, rank, world)
     if world > 1:

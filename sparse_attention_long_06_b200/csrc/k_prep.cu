@@ -52,7 +52,7 @@ cudaError_t launch_meta(const PrefillArgs& a, cudaStream_t s) {
 // that overlap it (written to the selection-score table, then ranked).  In
 // select-only block attention the scores are routing scores and the query's
 // own block is always taken.
-__global__ void __launch_bounds__(256, 3) nsa_topn_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(256) nsa_topn_kernel(PrefillArgs a) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
   __shared__ unsigned long long cand_all[8][kTopnCand];
