@@ -345,6 +345,16 @@ def run_ours(args, rank, world):
                            "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a repeated step)"}
     dominant = max(TENSOR_KERNELS, key=lambda k: stage_ms[TENSOR_KERNELS[k][0]])
     roofline = rooflines[dominant]
+    # the selected kernel's other bound: every (token, group) gathers its
+    # selected blocks' K and V (l' keys x D x 2 B each) from L2 into shared memory
+    nblk = int((sel_h >= 0).sum())
+    gather_bytes = nblk * cfg.sel_block * cfg.head_dim * 2 * 2
+    slc_ms = stage_ms[TENSOR_KERNELS["nsa_slc_kernel"][0]]
+    l2_gather = {"kernel": "nsa_slc_kernel", "bound": "l2", "bytes_per_call": gather_bytes,
+                 "achieved": round(gather_bytes / (slc_ms / 1e3) / 1e12, 2), "unit": "TB/s",
+                 "peak": None,
+                 "note": "selected K/V blocks moved L2 -> shared memory per call; no measured "
+                         "L2 peak on this pool"}
 
     # end to end through the public API with host buffers: every step uploads
     # its inputs from pinned host memory and downloads its output; steps are
@@ -372,6 +382,7 @@ def run_ours(args, rank, world):
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_ms_max, 3),
                 "steps": e2e_steps, "schedule": "pipelined: upload, kernels, download on 3 streams, "
                                                 "2 device buffer sets"},
+        "l2_gather": l2_gather,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
     }

@@ -245,7 +245,8 @@ struct DecALayout {
   static constexpr int kSel = kRed + 2 * 64 * 4;                 // int [64]
   static constexpr int kHist = kSel + 64 * 4;                    // unsigned [256]
   static constexpr int kCand = kHist + 256 * 4;                  // u64 [kTopnCand]
-  static constexpr int kBars = kCand + kTopnCand * 8;
+  static constexpr int kMax = kCand + kTopnCand * 8;             // u64 [128] + [2]
+  static constexpr int kBars = kMax + 130 * 8;
   static constexpr int kEnd = kBars + 24 * 8;
   static constexpr int kSmem = kEnd + 1024;  // manual 1024-byte alignment
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -270,6 +271,7 @@ __global__ void __launch_bounds__(kDecThreads)
   float* red = reinterpret_cast<float*>(sm + L::kRed);
   unsigned* hist = reinterpret_cast<unsigned*>(sm + L::kHist);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(sm + L::kCand);
+  unsigned long long* smax = reinterpret_cast<unsigned long long*>(sm + L::kMax);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int pair = blockIdx.x;
@@ -418,25 +420,26 @@ __global__ void __launch_bounds__(kDecThreads)
         if (on) scores[j] = s;
       });
       named_bar_128<1>();
-      // top-n (one warp): the workspace copy feeds the selected units
-      if (warp == 2) {
-        int* gsel = a.sel ? a.sel + ((size_t)b * a.geo.Hkv + g) * n : nullptr;
-        auto put = [&](int i, int j) {
-          if (live) rec.sel[i] = j;
-          if (gsel && live) gsel[i] = j;
-        };
-        // the bound-and-rank selection over the shared-memory scores, else
-        // (when too many keys tie at its bound) the radix select
-        if (!a.geo.remap) {
-          auto score = [&](int j) { return scores[j]; };
-          if (!warp_topn_reread(score, P.C, P.ncand, n, cand, put))
-            warp_topn(score, P.C, P.ncand, n, hist, put);
-        } else {
-          const int C = P.C;
-          auto score = [&](int j) { return remap_score(a.geo, [&](int i) { return scores[i]; }, C, j); };
-          if (!warp_topn_reread(score, P.ncand, P.ncand, n, cand, put))
-            warp_topn(score, P.ncand, P.ncand, n, hist, put);
-        }
+      // top-n (the four softmax warps; the workspace copy feeds the selected
+      // units): the bound-and-rank selection over the shared-memory scores,
+      // else (when too many keys tie at its bound) the radix select on one warp
+      int* gsel = a.sel ? a.sel + ((size_t)b * a.geo.Hkv + g) * n : nullptr;
+      auto put = [&](int i, int j) {
+        if (live) rec.sel[i] = j;
+        if (gsel && live) gsel[i] = j;
+      };
+      auto sync = [&]() { named_bar_128<1>(); };
+      const int C = P.C;
+      auto remapped = [&](int j) { return remap_score(a.geo, [&](int i) { return scores[i]; }, C, j); };
+      auto plain = [&](int j) { return scores[j]; };
+      const bool done = a.geo.remap
+                            ? group_topn_128(remapped, P.ncand, P.ncand, n, r, smax, cand, smax + 128, sync, put)
+                            : group_topn_128(plain, C, P.ncand, n, r, smax, cand, smax + 128, sync, put);
+      if (!done && warp == 2) {
+        if (a.geo.remap)
+          warp_topn(remapped, P.ncand, P.ncand, n, hist, put);
+        else
+          warp_topn(plain, C, P.ncand, n, hist, put);
       }
     }
   }

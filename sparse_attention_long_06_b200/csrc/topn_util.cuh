@@ -256,4 +256,76 @@ __device__ __forceinline__ bool warp_topn_reread(ScoreFn score, int ncmp, int nc
   return true;
 }
 
+
+// The same selection by the 128 threads of a warpgroup (t = 0..127; `sync`
+// is a barrier over exactly those threads) for rows whose scores `score(j)`
+// are cheap to re-read: thread t takes the largest key of candidates t,
+// t + 128, ...; T0 = the n-th largest of the 128 thread maxima (at least n
+// keys reach it); the keys >= T0 are gathered into `cand` and ranked
+// exactly, and each of the n largest writes itself at its position in
+// ascending block order.  Scratch: `smax` 128 words, `cand` kTopnCand words,
+// `ctl` 2 words, all shared.  Returns false (uniformly), having written
+// nothing, when more than kTopnCand keys reach T0.
+template <typename ScoreFn, typename OutFn, typename SyncFn>
+__device__ __forceinline__ bool group_topn_128(ScoreFn score, int ncmp, int ncand, int n, int t,
+                                               unsigned long long* smax,
+                                               unsigned long long* cand,
+                                               unsigned long long* ctl, SyncFn sync, OutFn out) {
+  if (ncand <= n) {
+    for (int j = t; j < n; j += 128) out(j, j < ncand ? j : -1);
+    return true;
+  }
+  auto key = [&](int j) -> unsigned long long {
+    const uint32_t b = j < ncmp ? score_key(score(j)) : kZeroScoreKey;
+    return ((unsigned long long)b << 32) | (0xFFFFFFFFu - (uint32_t)j);
+  };
+  unsigned long long lmax = 0;
+  for (int j = t; j < ncand; j += 128) {
+    const unsigned long long k = key(j);
+    lmax = k > lmax ? k : lmax;
+  }
+  smax[t] = lmax;
+  if (t == 0) ctl[1] = 0;
+  sync();
+  // T0: the thread maxima are distinct keys (or 0 for a thread without
+  // candidates); more than n threads hold one because ncand > n
+  int rank = 0;
+  for (int u = 0; u < 128; ++u) rank += smax[u] > lmax;
+  if (lmax != 0ull && rank == n - 1) ctl[0] = lmax;
+  sync();
+  const unsigned long long t0 = ctl[0];
+  for (int j = t; j < ncand; j += 128) {
+    const unsigned long long k = key(j);
+    if (k >= t0) {
+      const unsigned long long pos = atomicAdd(ctl + 1, 1ull);
+      if (pos < (unsigned long long)kTopnCand) cand[pos] = k;
+    }
+  }
+  sync();
+  const int count = (int)ctl[1];
+  if (count > kTopnCand) return false;
+  // the n-th largest gathered key
+  unsigned long long mine = 0;
+  if (t < count) {
+    mine = cand[t];
+    int r = 0;
+    for (int e = 0; e < count; ++e) r += cand[e] > mine;
+    if (r == n - 1) ctl[0] = mine;
+  }
+  sync();
+  const unsigned long long kth = ctl[0];
+  if (t < count && mine >= kth) {
+    // position among the selected keys in ascending block order (a larger
+    // key field below the score means a smaller block index)
+    const uint32_t jm = 0xFFFFFFFFu - (uint32_t)(mine & 0xFFFFFFFFull);
+    int pos = 0;
+    for (int e = 0; e < count; ++e) {
+      const unsigned long long o = cand[e];
+      pos += (o >= kth) && ((0xFFFFFFFFu - (uint32_t)(o & 0xFFFFFFFFull)) < jm);
+    }
+    out(pos, (int)jm);
+  }
+  return true;
+}
+
 }  // namespace nsa
