@@ -397,6 +397,8 @@ def run_ours(args, rank, world):
                           if name != args.workload}
         torch.cuda.empty_cache()
         result["legs"]["block_select_64k"] = run_block_select_leg(dev, world)
+        torch.cuda.empty_cache()
+        result["legs"]["block_select_decode_64k"] = run_block_select_decode_leg(dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(cfg, inputs)
         result["cpu_baseline_1core"] = oracle_single_core()
@@ -559,6 +561,66 @@ def run_block_select_leg(dev, world, steps=10, warmup=3, name="prefill_64k"):
             "rooflines": roof}
 
 
+def run_block_select_decode_leg(dev, world=1, steps=20, warmup=3):
+    """Select-only decode step (own block + n - 1 routed blocks) on the decode
+    workload (32 sequences x 65 537 cached tokens): tokens/s and the time of
+    each launch.  The routing-key cache holds the generator's synthetic cache
+    state (the amount of work does not depend on its values)."""
+    import torch
+    from sparse_attention_long_06_b200 import nsa
+    cfg = wl.CONFIGS["decode_64k"]
+    inp = wl.decode_inputs(cfg)
+    B, cap = cfg.decode_batch, int(inp["capacity"])
+    d = {}
+    for k in ("q", "k", "v", "seqlens"):
+        a = np.ascontiguousarray(inp[k])
+        d[k] = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+    km = np.ascontiguousarray(inp["kc"][:, :cap // cfg.sel_block])
+    d["km"] = torch.from_numpy(km.view(np.int16)).to(dev)
+    del inp
+    plan = nsa.Plan.for_config(cfg, max_batch=B, max_seqlen=cap, out_dtype=nsa.OUT_BF16)
+    out = torch.empty((B, cfg.num_q_heads, cfg.head_dim), dtype=torch.int16, device=dev)
+    sel = torch.empty((B, cfg.num_kv_heads, cfg.top_n), dtype=torch.int32, device=dev)
+    ws = plan.alloc_workspace(nsa.MODE_BLOCK_SELECT_DECODE, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        plan.block_select_decode(d["q"], d["k"], d["v"], d["km"], d["seqlens"], out, ws,
+                                 sel_idx=sel)
+
+    for _ in range(max(3, warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if nsa.read_device_status(ws) != nsa.NSA_OK:
+        raise RuntimeError("select-only decode: device status after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ev), world, dev)
+    nsa.profile_enable(True)
+    flush.zero_()
+    step()
+    stage = nsa.profile_stage_ms()
+    nsa.profile_enable(False)
+    return {"metric": "select-only block attention decode tokens/s",
+            "value": round(job_rate(B, world, ms), 1), "unit": "tokens/s",
+            "ms_per_step_median": round(ms, 5), "steps": steps,
+            "config": {"workload": cfg.name, "batch": B, "context": int(cfg.decode_len),
+                       "l_sel": cfg.sel_block, "top_n": cfg.top_n,
+                       "mode": "block_select (own block + n - 1 routed)",
+                       "routing_key_cache": "synthetic random state",
+                       "l2": "flushed before every timed step"},
+            "stage_ms": {"nsa_decode_block_mean_kernel": round(stage[0], 5),
+                         "nsa_decode_a_kernel": round(stage[1], 5),
+                         "nsa_decode_b_kernel": round(stage[2], 5)}}
+
+
 def oracle_single_core(names=("tiny", "prefill_8k"), nrows=64):
     """The oracle's tokens/s on one host core for small configurations, in a
     child process with OMP_NUM_THREADS=1 (bounded: `nrows` sampled rows)."""
@@ -704,6 +766,8 @@ def main():
                     help="run only the decode leg and print its object (profiling)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="sequences in the decode leg (default: the workload's 32)")
+    ap.add_argument("--block-select-decode-only", action="store_true",
+                    help="time only the select-only decode leg")
     ap.add_argument("--block-select-only", action="store_true",
                     help="time only the select-only block attention leg")
     ap.add_argument("--no-legs", action="store_true",
@@ -738,6 +802,9 @@ def main():
         torch.distributed.barrier()
     if args.decode_only:
         res = run_decode_leg(args, torch.device("cuda", torch.cuda.current_device()), world)
+    elif args.block_select_decode_only:
+        res = run_block_select_decode_leg(torch.device("cuda", torch.cuda.current_device()), world,
+                                          steps=max(args.steps, 20), warmup=args.warmup)
     elif args.block_select_only:
         res = run_block_select_leg(torch.device("cuda", torch.cuda.current_device()), world,
                                    steps=max(args.steps, 3), warmup=args.warmup,

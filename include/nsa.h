@@ -75,7 +75,8 @@ typedef enum { NSA_OUT_BF16 = 0, NSA_OUT_F32 = 1 } nsa_out_dtype;
 typedef enum {
   NSA_MODE_PREFILL = 0,      /* nsa_prefill, nsa_prefill_noalloc */
   NSA_MODE_DECODE = 1,       /* nsa_decode */
-  NSA_MODE_BLOCK_SELECT = 2  /* nsa_block_select_prefill */
+  NSA_MODE_BLOCK_SELECT = 2,        /* nsa_block_select_prefill */
+  NSA_MODE_BLOCK_SELECT_DECODE = 3  /* nsa_block_select_decode */
 } nsa_mode;
 
 typedef struct {
@@ -261,6 +262,31 @@ int nsa_block_select_prefill(nsa_plan_t plan, const void* q, const void* k, cons
                              const int* cu_seqlens, int batch, int total_tokens, void* out,
                              void* k_mean, int* sel_idx, void* workspace, size_t workspace_bytes,
                              void* stream);
+
+/*
+ * One decode step of select-only block attention for a batch of sequences:
+ * the newest token of each sequence (already written into the caches)
+ * attends to its own block and to the n - 1 best-routed complete blocks
+ * before it, with the readings of nsa_block_select_prefill.
+ *   q            [batch, Hq, D]             bf16, query of the newest token
+ *   k_cache, v_cache [batch, cache_capacity, Hkv, D] bf16
+ *   k_mean_cache [batch, cache_capacity / l', Hkv, D] bf16: the routing keys
+ *                of every complete block before the newest token; when the
+ *                newest token completes its block (len % l' == 0) that
+ *                block's routing key is computed here and written back (it is
+ *                routed from the next step on)
+ *   seqlens      [batch] int32 device, 1 <= len <= cache_capacity
+ *   cache_capacity  multiple of l', <= plan max_seqlen, at most 4096 blocks
+ *   out          [batch, Hq, D] bf16 or fp32 (plan out_dtype)
+ *   sel_idx      [batch, Hkv, top_n] int32 or NULL (ascending, own block last)
+ *   workspace    >= nsa_workspace_size(plan, NSA_MODE_BLOCK_SELECT_DECODE)
+ * Three launches: the routing key of a completed block, the routing and
+ * top-n kernel, and the selected-block kernel with the merge.
+ */
+int nsa_block_select_decode(nsa_plan_t plan, const void* q, const void* k_cache,
+                            const void* v_cache, void* k_mean_cache, const int* seqlens, int batch,
+                            int cache_capacity, void* out, int* sel_idx, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /* Rows of the packed routing-key output of nsa_block_select_prefill over
  * `total_tokens` tokens: floor(total_tokens / l'). */

@@ -90,6 +90,9 @@ def _load():
             lib.oracle_block_select_rows.argtypes = [P, ctypes.c_int, vp, vp, vp, vp, vp,
                                                      ctypes.c_int, vp, vp, ctypes.c_int, vp, vp]
             lib.oracle_block_select_rows.restype = ctypes.c_int
+            lib.oracle_block_select_query.argtypes = [P, ctypes.c_int, vp, vp, vp, vp, vp, vp,
+                                                      ctypes.c_int, vp, vp]
+            lib.oracle_block_select_query.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -298,3 +301,36 @@ def block_select_reference(p: OracleParams, inputs: dict, rows_per_seq=None,
         r.update(rows=rows, kbar64=kb64, kbar16=kb16)
         out.append(r)
     return out
+
+
+def block_select_query(p: OracleParams, t: int, q_row, k, v, kbar, cmax: int) -> dict:
+    """Select-only block attention for a single query at position t (decode):
+    q_row [Hq,D], k/v [>=t+1,Hkv,D], kbar [>=max(1, t // l'),Hkv,D]."""
+    q_row, k, v, kbar = _c(q_row, np.uint16), _c(k, np.uint16), _c(v, np.uint16), _c(kbar, np.uint16)
+    Hq, Hkv, D, n = p.num_q_heads, p.num_kv_heads, p.head_dim, p.top_n
+    res = {"out": np.zeros((Hq, D)), "scores": np.zeros((Hkv, cmax)),
+           "sel": np.zeros((Hkv, n), dtype=np.int32), "gap": np.zeros(Hkv)}
+    rc = _load().oracle_block_select_query(ctypes.byref(p.c()), int(t), _ptr(q_row), _ptr(k),
+                                           _ptr(v), _ptr(kbar), _ptr(res["out"]),
+                                           _ptr(res["scores"]), cmax, _ptr(res["sel"]),
+                                           _ptr(res["gap"]))
+    if rc != 0:
+        raise ValueError("oracle rejected the geometry")
+    return res
+
+
+def block_select_decode_reference(p: OracleParams, q_row, k_seq, v_seq, kmean, L: int) -> dict:
+    """Select-only decode of the newest token (t = L - 1) of one sequence:
+    k_seq/v_seq [>=L,Hkv,D] the caches, kmean [>=1,Hkv,D] the routing keys of
+    the complete blocks before the newest token.  The routing key of the block
+    the newest token completes (L % l' == 0) is computed here ("written")."""
+    ls = p.sel_block
+    t = L - 1
+    written = None
+    if L % ls == 0:
+        _, written = block_means(p, k_seq[L - ls:L])
+        written = written[0]
+    kb = kmean if kmean.shape[0] else np.zeros((1, p.num_kv_heads, p.head_dim), np.uint16)
+    r = block_select_query(p, t, q_row, k_seq, v_seq, kb, cmax=max(1, kb.shape[0]))
+    r.update(t=t, written=written)
+    return r

@@ -70,6 +70,46 @@ cudaError_t launch_block_mean(const PrefillArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Decode: when the newest token completes its block (len % l' == 0), that
+// block's mean key (fp64 sum in token order, rounded once) goes into the
+// mean-key cache [B, cap / l', Hkv, D] for the steps that follow.  One CTA
+// per (sequence, KV head), one thread per 8 channels.
+__global__ void nsa_decode_block_mean_kernel(DecodeArgs a) {
+  const int b = blockIdx.x, h = blockIdx.y, D = a.geo.D, H = a.geo.Hkv, L = a.geo.ls;
+  const int c0 = threadIdx.x * 8;
+  if (c0 >= D) return;
+  const int len = __ldg(a.seqlens + b);
+  if (len < L || len > a.cap || len % L != 0) return;
+  const int j = len / L - 1;
+  const uint16_t* src = a.k_cache + (((size_t)b * a.cap + (size_t)j * L) * H + h) * D + c0;
+  double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+  for (int p = 0; p < L; ++p) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + (size_t)p * H * D));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += (double)__uint_as_float(w[e] << 16);
+      acc[2 * e + 1] += (double)__uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  }
+  const double inv = 1.0 / (double)L;
+  uint32_t o[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat16 lo = __double2bfloat16(acc[2 * e] * inv);
+    const __nv_bfloat16 hi = __double2bfloat16(acc[2 * e + 1] * inv);
+    o[e] = (uint32_t)*reinterpret_cast<const uint16_t*>(&lo) |
+           ((uint32_t)*reinterpret_cast<const uint16_t*>(&hi) << 16);
+  }
+  uint16_t* dst = a.k_cmp + (((size_t)b * a.ccap + j) * H + h) * D + c0;
+  *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+cudaError_t launch_decode_block_mean(const DecodeArgs& a, cudaStream_t s) {
+  nsa_decode_block_mean_kernel<<<dim3(a.batch, a.geo.Hkv), a.geo.D / 8, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ routing scores
 // S[t, g, j] = sum over the G heads h of group g of q[t, h] . Kbar[j, g] for
 // the blocks j < t / l' (the complete blocks before t's own block).

@@ -111,13 +111,21 @@ __device__ __forceinline__ DecPair dec_pair(const DecodeArgs& a, int pair) {
   p.ok = p.L >= 1 && p.L <= a.cap;
   if (!p.ok) return p;
   p.t = p.L - 1;
-  p.C = num_cmp_blocks(p.L, a.geo.l, a.geo.d);
-  p.ncc = (p.C + kChunk - 1) / kChunk;
-  const int wn = min(a.geo.w, p.L);
-  p.nwc = (wn + kChunk - 1) / kChunk;
   const int bpc = kChunk >> a.geo.lg_ls;
   p.nsc = (a.geo.n + bpc - 1) / bpc;
-  p.ncand = p.t / a.geo.ls + 1;
+  if (a.select_only) {
+    // routing candidates: the complete blocks before the own block t / l'
+    p.C = p.t >> a.geo.lg_ls;
+    p.ncc = (p.C + kChunk - 1) / kChunk;
+    p.nwc = 0;
+    p.ncand = p.C;
+  } else {
+    p.C = num_cmp_blocks(p.L, a.geo.l, a.geo.d);
+    p.ncc = (p.C + kChunk - 1) / kChunk;
+    const int wn = min(a.geo.w, p.L);
+    p.nwc = (wn + kChunk - 1) / kChunk;
+    p.ncand = p.t / a.geo.ls + 1;
+  }
   p.cmp_row0 = p.C - kChunk * p.ncc;      // compressed chunks end at the last block
   p.win_row0 = p.t - kChunk * p.nwc + 1;  // window chunks end at t
   return p;
@@ -376,6 +384,36 @@ __global__ void __launch_bounds__(kDecThreads)
     for (int c = 0; c < nchunks; ++c) kok |= (P.cmp_row0 + c * kChunk + r >= 0) ? (1u << c) : 0u;
     mbar_wait(s_full, 0, abort_flag, status, kWaitCycles);
     tc_fence_after();
+    if (a.select_only) {
+      // routing scores: the sum over the group's heads of q . mean key (one
+      // sweep, no softmax), then the n - 1 best earlier blocks and the own one
+      float* scores = reinterpret_cast<float*>(sm + L::kU);
+      const bool live = !*abort_flag;
+      sweep_chunks<32>(lane_addr, 0, nchunks, [&](int c, const float(&v)[16]) {
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < 16; ++h) s += ((colmask >> h) & 1u) ? v[h] : 0.f;
+        if ((kok >> c) & 1u) scores[P.cmp_row0 + c * kChunk + r] = s;
+      });
+      named_bar_128<1>();
+      int* gsel = a.sel ? a.sel + ((size_t)b * a.geo.Hkv + g) * n : nullptr;
+      auto put = [&](int i, int j) {
+        if (live) rec.sel[i] = j;
+        if (gsel && live) gsel[i] = j;
+      };
+      auto sync = [&]() { named_bar_128<1>(); };
+      auto plain = [&](int j) { return scores[j]; };
+      const int C = P.C, m = n - 1;
+      bool done = true;
+      if (m > 0) done = group_topn_128(plain, C, C, m, r, smax, cand, smax + 128, sync, put);
+      if (!done && warp == 2) warp_topn(plain, C, C, m, hist, put);
+      sync();
+      if (r == 0) {
+        const int taken = C < m ? C : m;
+        put(taken, P.t >> a.geo.lg_ls);
+        for (int i = taken + 1; i < n; ++i) put(i, -1);
+      }
+    } else {
     // sweep 1: per-head maximum (log2 units)
     float mx[16];
 #pragma unroll
@@ -441,6 +479,7 @@ __global__ void __launch_bounds__(kDecThreads)
         else
           warp_topn(plain, C, P.ncand, n, hist, put);
       }
+    }
     }
   }
   tc_fence_before();
@@ -778,9 +817,10 @@ __global__ void __launch_bounds__(kDecThreads)
     for (int i = threadIdx.x; i < a.nwu * 32; i += blockDim.x)
       wml[i] = __ldcg(rec.win + (size_t)(i >> 5) * PF + G * D + (i & 31));
     for (int i = threadIdx.x; i < G * 3; i += blockDim.x)
-      gt[i] = __ldg(a.gates + ((size_t)b * Hq + g * G) * 3 + i);
+      gt[i] = a.select_only ? ((i % 3) == 1 ? 1.f : 0.f)  // the selected branch alone
+                            : __ldg(a.gates + ((size_t)b * Hq + g * G) * 3 + i);
     __syncthreads();
-    const int ncv = (P.ncc + kUnitChunks - 1) / kUnitChunks;
+    const int ncv = a.select_only ? 0 : (P.ncc + kUnitChunks - 1) / kUnitChunks;
     for (int item = threadIdx.x; item < G * (D / 4); item += blockDim.x) {
       const int h = item / (D / 4), c4 = (item - h * (D / 4)) * 4;
       float4 vs[kMaxSlcUnits], vw[kMaxWinUnits], vc[kMaxCmpUnits];

@@ -120,17 +120,18 @@ struct DecodeLayout {
 // Decode workspace for `batch` sequences in a cache of `cap` tokens:
 // status header, per-pair unit counters, selection, compressed P^T and the
 // fp32 partial records of the second decode kernel.
-DecodeLayout decode_layout(const nsa_plan_s* pl, int batch, int cap) {
+DecodeLayout decode_layout(const nsa_plan_s* pl, int batch, int cap, bool select_only = false) {
   const Geometry& g = pl->geo;
   DecodeLayout L{};
   const size_t pairs = (size_t)batch * g.Hkv;
-  const int ccap = cap / g.d;
+  const int ccap = cap / (select_only ? g.ls : g.d);
   L.ncc_max = (ccap + kChunk - 1) / kChunk;
-  L.ncv_max = (L.ncc_max + kUnitChunks - 1) / kUnitChunks;
   const int nsc = (g.n + (kChunk >> g.lg_ls) - 1) / (kChunk >> g.lg_ls);
   L.nsl = (nsc + kUnitChunks - 1) / kUnitChunks;
   const int wmax = g.w < cap ? g.w : cap;
-  L.nwu = ((wmax + kChunk - 1) / kChunk + kUnitChunks - 1) / kUnitChunks;
+  // select-only: selected units only (no compressed values, no window, no P^T)
+  L.ncv_max = select_only ? 0 : (L.ncc_max + kUnitChunks - 1) / kUnitChunks;
+  L.nwu = select_only ? 0 : ((wmax + kChunk - 1) / kChunk + kUnitChunks - 1) / kUnitChunks;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -140,7 +141,7 @@ DecodeLayout decode_layout(const nsa_plan_s* pl, int batch, int cap) {
   take(kHeaderBytes);
   L.counters = take(pairs * sizeof(int));
   L.sel = take(pairs * g.n * sizeof(int));
-  L.pt = take(pairs * (size_t)L.ncc_max * 4096);
+  L.pt = take(select_only ? 0 : pairs * (size_t)L.ncc_max * 4096);
   L.win = take(pairs * (size_t)L.nwu * (g.G * g.D + 32) * sizeof(float));
   L.cmp = take(pairs * (size_t)L.ncv_max * g.G * g.D * sizeof(float));
   L.slc = take(pairs * (size_t)L.nsl * (g.G * g.D + 32) * sizeof(float));
@@ -350,6 +351,10 @@ size_t nsa_workspace_size(nsa_plan_t plan, int mode) {
     return decode_layout(plan, plan->p.max_batch, cap).total;
   }
   if (mode == NSA_MODE_BLOCK_SELECT) return block_select_layout(plan).total;
+  if (mode == NSA_MODE_BLOCK_SELECT_DECODE) {
+    const int cap = plan->p.max_seqlen / plan->geo.ls * plan->geo.ls;
+    return decode_layout(plan, plan->p.max_batch, cap, true).total;
+  }
   return 0;
 }
 
@@ -669,6 +674,83 @@ int nsa_decode(nsa_plan_t plan, const void* q, const void* k_cache, const void* 
   prof_mark(s);
   if (e != cudaSuccess) {
     fprintf(stderr, "nsa_decode: launch failed: %s\n", cudaGetErrorString(e));
+    return NSA_ERR_CUDA;
+  }
+  g_last_launches = 3;
+  return NSA_OK;
+}
+
+int nsa_block_select_decode(nsa_plan_t plan, const void* q, const void* k_cache,
+                            const void* v_cache, void* k_mean_cache, const int* seqlens, int batch,
+                            int cache_capacity, void* out, int* sel_idx, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  g_last_launches = 0;
+  if (!plan) return NSA_ERR_INVALID_ARG;
+  const nsa_params& p = plan->p;
+  const Geometry& geo = plan->geo;
+  if (batch <= 0 || batch > p.max_batch || cache_capacity <= 0 ||
+      cache_capacity > p.max_seqlen || cache_capacity % geo.ls != 0)
+    return NSA_ERR_INVALID_ARG;
+  // all of one query's routing scores stay on chip: at most 4096 blocks
+  if (cache_capacity / geo.ls > kDecodeMaxCmp) return NSA_ERR_UNSUPPORTED;
+  if (!workspace) return NSA_ERR_WORKSPACE;
+  const DecodeLayout DL = decode_layout(plan, batch, cache_capacity, true);
+  if (workspace_bytes < DL.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return NSA_ERR_WORKSPACE;
+  if (!q || !k_cache || !v_cache || !k_mean_cache || !seqlens || !out) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_mean_cache) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sel_idx) & 3u))
+    return NSA_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a{};
+  a.geo = geo;
+  a.batch = batch;
+  a.cap = cache_capacity;
+  a.ccap = cache_capacity / geo.ls;
+  a.q = static_cast<const uint16_t*>(q);
+  a.k_cache = static_cast<const uint16_t*>(k_cache);
+  a.v_cache = static_cast<const uint16_t*>(v_cache);
+  a.k_cmp = static_cast<uint16_t*>(k_mean_cache);
+  a.seqlens = seqlens;
+  a.out = out;
+  a.sel = sel_idx;
+  a.select_only = 1;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.status = reinterpret_cast<int*>(ws);
+  a.ncc_max = DL.ncc_max;
+  a.ncv_max = DL.ncv_max;
+  a.nsl = DL.nsl;
+  a.nwu = DL.nwu;
+  a.counters = reinterpret_cast<int*>(ws + DL.counters);
+  a.ws_sel = reinterpret_cast<int*>(ws + DL.sel);
+  a.ws_pt = ws + DL.pt;
+  a.ws_win = reinterpret_cast<float*>(ws + DL.win);
+  a.ws_cmp = reinterpret_cast<float*>(ws + DL.cmp);
+  a.ws_slc = reinterpret_cast<float*>(ws + DL.slc);
+  DecodeMaps m;
+  memset(&m, 0, sizeof(m));
+  bool ok = encode3d(&m.q, q, geo.D, geo.Hq, batch, geo.Hq < 16 ? geo.Hq : 16, 1) &&
+            encode4d(&m.kc, k_mean_cache, geo.D, geo.Hkv, a.ccap, batch, kChunk) &&
+            encode4d(&m.k_blk, k_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.ls) &&
+            encode4d(&m.v_blk, v_cache, geo.D, geo.Hkv, cache_capacity, batch, geo.ls);
+  if (!ok) return NSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, DL.counters + (size_t)batch * geo.Hkv * sizeof(int), s) != cudaSuccess)
+    return NSA_ERR_CUDA;
+  prof_reset();
+  prof_mark(s);
+  cudaError_t e = launch_decode_block_mean(a, s);
+  if (e == cudaSuccess) {
+    prof_mark(s);
+    e = launch_decode_a(a, m, s);
+  }
+  if (e == cudaSuccess) {
+    prof_mark(s);
+    e = launch_decode_b(a, m, s);
+  }
+  prof_mark(s);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "nsa_block_select_decode: launch failed: %s\n", cudaGetErrorString(e));
     return NSA_ERR_CUDA;
   }
   g_last_launches = 3;

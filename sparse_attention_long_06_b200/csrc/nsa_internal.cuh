@@ -113,6 +113,9 @@ struct DecodeArgs {
   void* out;                // [B, Hq, D]
   int* sel;                 // [B, Hkv, n] or null
   int* status;
+  int select_only;          // select-only block attention: k_cmp is the mean-key cache
+                            // [B, cap / l', Hkv, D]; routing scores, the own block
+                            // forced in, output = selected branch (no gates)
   // units of the second decode kernel and its workspace records (per
   // (sequence, group) pair: see nsa_decode_b_kernel)
   int ncc_max;              // ceil(ccap / 128): compressed chunks of the longest sequence
@@ -199,6 +202,7 @@ cudaError_t launch_block_score(const PrefillArgs& a, const PrefillMaps& m, int n
                                cudaStream_t s);
 cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s);
 cudaError_t launch_decode_compress(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_block_mean(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_a(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);
 cudaError_t launch_decode_b(const DecodeArgs& a, const DecodeMaps& m, cudaStream_t s);
 

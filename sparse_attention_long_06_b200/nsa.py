@@ -23,7 +23,7 @@ NSA_ERR_CUDA = 5
 NSA_ERR_DEVICE_TIMEOUT = 6
 NSA_ERR_DEVICE_BAD_INPUT = 7
 OUT_BF16, OUT_F32 = 0, 1
-MODE_PREFILL, MODE_DECODE, MODE_BLOCK_SELECT = 0, 1, 2
+MODE_PREFILL, MODE_DECODE, MODE_BLOCK_SELECT, MODE_BLOCK_SELECT_DECODE = 0, 1, 2, 3
 WS_STATUS, WS_O_CMP, WS_LSE, WS_SCORES, WS_SEL, WS_WIN, WS_SEL_SCORES = 0, 1, 2, 3, 4, 5, 6
 
 EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_workspace_region",
@@ -31,7 +31,7 @@ EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_wo
             "nsa_selftest_timeout", "nsa_strerror", "nsa_last_launch_count",
             "nsa_profile_enable", "nsa_profile_stage_ms", "nsa_prefill_noalloc",
             "nsa_plan", "nsa_noalloc_read_device_status", "nsa_block_select_prefill",
-            "nsa_block_rows"]
+            "nsa_block_rows", "nsa_block_select_decode"]
 
 
 class NsaError(RuntimeError):
@@ -82,6 +82,8 @@ def lib():
             L.nsa_prefill_noalloc.restype = i
             L.nsa_block_select_prefill.argtypes = [vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, sz, vp]
             L.nsa_block_select_prefill.restype = i
+            L.nsa_block_select_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp]
+            L.nsa_block_select_decode.restype = i
             L.nsa_block_rows.argtypes = [vp, i]
             L.nsa_block_rows.restype = i
             L.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -211,6 +213,19 @@ class Plan:
                                             workspace.numel() * workspace.element_size(),
                                             _stream(stream))
         _check(rc, "nsa_block_select_prefill")
+
+    def block_select_decode(self, q, k_cache, v_cache, k_mean_cache, seqlens, out, workspace,
+                            sel_idx=None, stream=None):
+        """One select-only decode step (caches include the newest token);
+        workspace of workspace_size(MODE_BLOCK_SELECT_DECODE) bytes."""
+        batch = q.shape[0]
+        cap = k_cache.shape[1]
+        rc = lib().nsa_block_select_decode(self.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                           _ptr(k_mean_cache), _ptr(seqlens), batch, cap,
+                                           _ptr(out), _ptr(sel_idx), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream))
+        _check(rc, "nsa_block_select_decode")
 
     def decode(self, q, k_cache, v_cache, k_cmp_cache, v_cmp_cache, seqlens, gates, w_k, w_v,
                out, workspace, sel_idx=None, stream=None):

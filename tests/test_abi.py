@@ -200,6 +200,36 @@ def test_block_select_sizes_and_bad_arguments(L):
     assert L.nsa_last_launch_count() == 0
 
 
+def test_block_select_decode_rejects_bad_arguments_before_launch(L):
+    p = nsa.Plan(**_params(max_batch=4, max_seqlen=65536))
+    fake = 1 << 20  # an aligned address that is never dereferenced
+    wsb = p.workspace_size(nsa.MODE_BLOCK_SELECT_DECODE)
+    assert 256 < wsb < p.workspace_size(nsa.MODE_DECODE)  # selected units only
+    args = dict(q=fake, k=fake, v=fake, km=fake, lens=fake, batch=2, cap=4096, out=fake, sel=None,
+                ws=fake, wsb=wsb)
+
+    def call(**over):
+        a = dict(args)
+        a.update(over)
+        return L.nsa_block_select_decode(p.handle, a["q"], a["k"], a["v"], a["km"], a["lens"],
+                                         a["batch"], a["cap"], a["out"], a["sel"], a["ws"],
+                                         a["wsb"], None)
+
+    assert call(batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(batch=5) == nsa.NSA_ERR_INVALID_ARG
+    assert call(cap=4000) == nsa.NSA_ERR_INVALID_ARG            # not a multiple of l'
+    assert call(cap=65536 + 64) == nsa.NSA_ERR_INVALID_ARG      # above the plan's max_seqlen
+    assert call(ws=None) == nsa.NSA_ERR_WORKSPACE
+    assert call(wsb=255) == nsa.NSA_ERR_WORKSPACE
+    assert call(km=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(km=fake + 8) == nsa.NSA_ERR_MISALIGNED
+    assert call(lens=fake + 2) == nsa.NSA_ERR_MISALIGNED
+    big = nsa.Plan(**_params(max_batch=1, max_seqlen=4097 * 64))
+    assert L.nsa_block_select_decode(big.handle, fake, fake, fake, fake, fake, 1, 4097 * 64, fake,
+                                     None, fake, 1 << 30, None) == nsa.NSA_ERR_UNSUPPORTED
+    assert L.nsa_last_launch_count() == 0
+
+
 def test_noalloc_rejects_plans_beyond_its_static_array(L):
     big = nsa.Plan(**_params())  # 64k tokens: several GB of workspace
     assert big.workspace_size() > 32 << 20

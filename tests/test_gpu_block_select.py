@@ -213,3 +213,121 @@ def test_block_select_rejects_inconsistent_seqlens_on_device():
     bad["cu_seqlens"] = np.array([0, 120, 150], dtype=np.int32)  # 120 > max_seqlen 100
     res = run_block_select(cfg, bad, max_seqlen=100)
     assert res["status"] == nsa.NSA_ERR_DEVICE_BAD_INPUT
+
+
+# ---------------------------------------------------------------- decode
+def _mean_cache(p, inp, cap):
+    """Routing keys of the blocks complete before each sequence's newest
+    token (the state earlier steps leave), from the oracle; other rows hold a
+    sentinel."""
+    B = len(inp["seqlens"])
+    ls = p.sel_block
+    km = np.full((B, cap // ls, p.num_kv_heads, p.head_dim), 0x7F7F, dtype=np.uint16)
+    for b, L in enumerate(inp["seqlens"]):
+        nb = (int(L) - 1) // ls
+        if nb:
+            _, kb = oracle.block_means(p, inp["k"][b][:nb * ls])
+            km[b, :nb] = kb
+    return km
+
+
+def run_block_select_decode(cfg, inp, km, out_dtype=nsa.OUT_F32):
+    import torch
+    B = len(inp["seqlens"])
+    cap = int(inp["capacity"])
+    plan = nsa.Plan.for_config(cfg, max_batch=B, max_seqlen=cap, out_dtype=out_dtype)
+    d = {k: gu.to_dev(inp[k]) for k in ("q", "k", "v", "seqlens")}
+    kmd = gu.to_dev(km)
+    out = torch.empty((B, cfg.num_q_heads, cfg.head_dim),
+                      dtype=torch.float32 if out_dtype == nsa.OUT_F32 else torch.int16, device="cuda")
+    sel = torch.full((B, cfg.num_kv_heads, cfg.top_n), -7, dtype=torch.int32, device="cuda")
+    ws = plan.alloc_workspace(nsa.MODE_BLOCK_SELECT_DECODE)
+    plan.block_select_decode(d["q"], d["k"], d["v"], kmd, d["seqlens"], out, ws, sel_idx=sel)
+    res = {"status": nsa.read_device_status(ws), "launches": nsa.last_launch_count(),
+           "sel": sel.cpu().numpy(), "km": gu.bits(kmd)}
+    res["out"] = (out.cpu().numpy().astype(np.float64) if out_dtype == nsa.OUT_F32
+                  else wl.bf16_to_f32(gu.bits(out)).astype(np.float64))
+    return res
+
+
+def check_block_select_decode(cfg, inp, km_in, res, seqs):
+    p = OracleParams.of(cfg)
+    ls = cfg.sel_block
+    rep = {"seqs": 0, "idx_mismatch": 0, "idx_near_tie": 0, "max_abs": 0.0}
+    num = den = 0.0
+    assert res["status"] == nsa.NSA_OK
+    for b in seqs:
+        L = int(inp["seqlens"][b])
+        nb = (L - 1) // ls
+        r = oracle.block_select_decode_reference(p, inp["q"][b], inp["k"][b], inp["v"][b],
+                                                 km_in[b, :nb], L)
+        # the routing key of a block the newest token completes, bit for bit;
+        # every other row of the cache untouched
+        exp = km_in[b].copy()
+        if r["written"] is not None:
+            exp[L // ls - 1] = r["written"]
+        np.testing.assert_array_equal(res["km"][b], exp)
+        same = np.all(r["sel"] == res["sel"][b], axis=1)
+        near = r["gap"] < 2 * SCORE_TOL
+        rep["idx_mismatch"] += int(np.count_nonzero(~same & ~near))
+        rep["idx_near_tie"] += int(np.count_nonzero(~same & near))
+        if np.all(same):
+            diff = np.abs(res["out"][b] - r["out"])
+            rep["max_abs"] = max(rep["max_abs"], float(diff.max()))
+            num += float(np.sum(diff ** 2))
+            den += float(np.sum(r["out"] ** 2))
+        rep["seqs"] += 1
+    rep["rel_l2"] = (num / den) ** 0.5 if den > 0 else 0.0
+    gu.log_report(f"block_select_decode:{cfg.name}", rep)
+    assert rep["idx_mismatch"] == 0, rep
+    assert rep["max_abs"] <= 1e-2 and rep["rel_l2"] <= 5e-3, rep
+    return rep
+
+
+@pytest.mark.parametrize("geom", [
+    # D, Hq, Hkv, l', n, lengths, capacity
+    (64, 4, 1, 32, 4, [1, 31, 32, 33, 100, 640, 1000], 1024),
+    (128, 64, 4, 64, 16, [700, 4096, 5000, 63, 64, 9000], 9024),
+    (64, 16, 2, 32, 1, [200, 32, 1], 256),
+    (128, 32, 4, 32, 12, [2048, 2047, 40000], 40000),
+])
+def test_block_select_decode_geometries(geom):
+    D, Hq, Hkv, ls, n, lens, cap = geom
+    cfg = wl.NsaConfig("bsd", 51, D, Hq, Hkv, ls, ls, ls, n, 1, decode_batch=len(lens))
+    inp = wl.decode_inputs(cfg, lengths=lens, capacity=cap)
+    km = _mean_cache(OracleParams.of(cfg), inp, int(inp["capacity"]))
+    res = run_block_select_decode(cfg, inp, km)
+    assert res["launches"] == 3
+    check_block_select_decode(cfg, inp, km, res, range(len(lens)))
+
+
+def test_block_select_decode_64k_batch_and_bf16_output():
+    cfg = wl.CONFIGS["decode_64k"]
+    inp = wl.decode_inputs(cfg)
+    km = _mean_cache(OracleParams.of(cfg), inp, int(inp["capacity"]))
+    res = run_block_select_decode(cfg, inp, km)
+    check_block_select_decode(cfg, inp, km, res, [0, 13, 31])
+    rb = run_block_select_decode(cfg, inp, km, out_dtype=nsa.OUT_BF16)
+    assert rb["status"] == nsa.NSA_OK
+    np.testing.assert_array_equal(rb["sel"], res["sel"])
+    np.testing.assert_array_equal(wl.bf16_bits(res["out"].astype(np.float32)),
+                                  wl.bf16_bits(rb["out"].astype(np.float32)))
+
+
+def test_block_select_decode_exact_ties_go_to_the_lower_block():
+    # keys repeating every three blocks: equal routing keys, equal scores
+    cfg = wl.NsaConfig("bsd_ties", 52, 128, 64, 4, 32, 32, 32, 8, 1, decode_batch=2)
+    inp = wl.decode_inputs(cfg, lengths=[3000, 1500], capacity=3008)
+    for b, L in enumerate(inp["seqlens"]):
+        idx = np.arange(int(L)) % 96
+        inp["k"][b][:L] = inp["k"][b][idx]
+    km = _mean_cache(OracleParams.of(cfg), inp, int(inp["capacity"]))
+    res = run_block_select_decode(cfg, inp, km)
+    rep = check_block_select_decode(cfg, inp, km, res, [0, 1])
+    assert rep["idx_near_tie"] == 0
+    for b, L in enumerate(inp["seqlens"]):
+        own = (int(L) - 1) // 32
+        for g in range(4):
+            picked = [int(j) for j in res["sel"][b, g] if j >= 0 and j != own]
+            assert len(picked) == 7 and picked[0] < 3
+            assert picked == list(range(picked[0], picked[0] + 21, 3))

@@ -187,3 +187,21 @@ def test_future_tokens_do_not_change_a_row():
     r2, _ = _run(p, q2, k2, v2)
     np.testing.assert_array_equal(r["out"][:t + 1], r2["out"][:t + 1])
     np.testing.assert_array_equal(r["sel"][:t + 1], r2["sel"][:t + 1])
+
+
+@pytest.mark.parametrize("L", [1, 31, 32, 33, 96, 130])
+def test_decode_step_equals_the_last_prefill_row(L):
+    D, Hq, Hkv, lsel, n = 64, 4, 2, 32, 3
+    p = _params(D, Hq, Hkv, lsel, n)
+    q, k, v = _inputs(40 + L, L, Hq, Hkv, D)
+    r, kb = _run(p, q, k, v)
+    # the routing keys of the blocks complete before the newest token
+    before = (L - 1) // lsel
+    _, kb_before = oracle.block_means(p, k[:before * lsel])
+    d = oracle.block_select_decode_reference(p, q[L - 1], k, v, kb_before, L)
+    np.testing.assert_array_equal(d["sel"], r["sel"][L - 1])
+    np.testing.assert_array_equal(d["out"], r["out"][L - 1])
+    if L % lsel == 0:
+        np.testing.assert_array_equal(d["written"], kb[L // lsel - 1])
+    else:
+        assert d["written"] is None
