@@ -485,3 +485,105 @@ int oracle_block_select_rows(const nsa_oracle_params* P, int T, const uint16_t* 
   }
   return bad ? -1 : 0;
 }
+
+/* ------------------------------------------------------------ token-level selection (DSA style) */
+/*
+ * Sparse attention with a token-level top-k chosen by a light indexer, in the
+ * style of DSA ("DeepSeek V3.2-Exp sparse attention" page
+ * (bjdmk.com.cn/news/5181035), sections 1 and 3: an indexer with 8 or 16
+ * heads and a ReLU activation scores every earlier token, the top_k = 2048
+ * tokens per query take part in the main attention).  The page gives no
+ * formula; the readings (listed in the repository's design notes) are:
+ *  - index score I[t, s] = sum over indexer heads j of w[t, j] *
+ *    ReLU(qi[t, j] . ki[s]) for s <= t (qi [T, Hi, Di], ki [T, Di] bf16, the
+ *    per-token head weights w [T, Hi] fp32; the page's fp8 indexer is a
+ *    precision choice this statement does not make);
+ *  - the top_k tokens by I (ties to the lower index; all of them when there
+ *    are at most top_k) are shared by every query head;
+ *  - each head attends (one softmax, scale as in the NSA branches) to the
+ *    keys and values of its KV group at the chosen tokens.
+ */
+typedef struct {
+  int Hi;   /* indexer heads */
+  int Di;   /* indexer head dim */
+  int top_k;
+} dsa_oracle_params;
+
+/* One query at position t: q [Hq, D], k, v [>= t+1, Hkv, D] bf16 (main
+ * attention), qi [Hi, Di] bf16 and w [Hi] fp32 of query t, ki [>= t+1, Di]
+ * bf16.  Outputs (any may be NULL): out [Hq, D], index [t + 1] (I[t, s]),
+ * sel [top_k] (ascending, -1 padded), gap (top_k-th minus (top_k+1)-th score). */
+int oracle_dsa_query(const nsa_oracle_params* P, const dsa_oracle_params* X, int t,
+                     const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     const uint16_t* qi, const float* w, const uint16_t* ki, double* out,
+                     double* index, int* sel, double* gap) {
+  const int D = P->D, Hq = P->Hq, Hkv = P->Hkv, G = Hq / Hkv;
+  if (Hq % Hkv != 0 || X->top_k < 1 || X->Hi < 1 || X->Di < 1) return -1;
+  const int ncand = t + 1;
+  double* I = (double*)malloc(sizeof(double) * (size_t)ncand);
+  int* chosen = (int*)malloc(sizeof(int) * (size_t)X->top_k);
+  int* rows = (int*)malloc(sizeof(int) * (size_t)X->top_k);
+  double* scratch = (double*)malloc(sizeof(double) * (size_t)X->top_k);
+  double* qh = (double*)malloc(sizeof(double) * (size_t)D);
+  double* o = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int s = 0; s < ncand; ++s) {
+    double acc = 0.0;
+    for (int j = 0; j < X->Hi; ++j) {
+      double dot = 0.0;
+      for (int c = 0; c < X->Di; ++c)
+        dot += oracle_bf16_to_f64(qi[(size_t)j * X->Di + c]) *
+               oracle_bf16_to_f64(ki[(size_t)s * X->Di + c]);
+      acc += (double)w[j] * (dot > 0.0 ? dot : 0.0);
+    }
+    I[s] = acc;
+  }
+  if (index)
+    for (int s = 0; s < ncand; ++s) index[s] = I[s];
+  const double gp = oracle_select(I, ncand, X->top_k, chosen);
+  if (gap) *gap = gp;
+  if (sel) memcpy(sel, chosen, sizeof(int) * (size_t)X->top_k);
+  int nk = 0;
+  for (int i = 0; i < X->top_k; ++i)
+    if (chosen[i] >= 0) rows[nk++] = chosen[i];
+  for (int g = 0; g < Hkv; ++g)
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      for (int c = 0; c < D; ++c) qh[c] = oracle_bf16_to_f64(q[(size_t)h * D + c]);
+      attend(P, qh, k, v, g, rows, nk, o, NULL, scratch);
+      if (out)
+        for (int c = 0; c < D; ++c) out[(size_t)h * D + c] = o[c];
+    }
+  free(I);
+  free(chosen);
+  free(rows);
+  free(scratch);
+  free(qh);
+  free(o);
+  return 0;
+}
+
+/* oracle_dsa_query for a list of rows of one sequence: q [T, Hq, D], k, v
+ * [T, Hkv, D], qi [T, Hi, Di], w [T, Hi], ki [T, Di]; outputs by position in
+ * `rows` (index rows of length T). */
+int oracle_dsa_rows(const nsa_oracle_params* P, const dsa_oracle_params* X, int T,
+                    const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* qi,
+                    const float* w, const uint16_t* ki, const int* rows, int nrows, double* out,
+                    double* index, int* sel, double* gap) {
+  const int D = P->D, Hq = P->Hq;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int r = 0; r < nrows; ++r) {
+    const int t = rows[r];
+    if (t < 0 || t >= T) {
+      bad |= 1;
+      continue;
+    }
+    const size_t hd = (size_t)Hq * D;
+    int rc = oracle_dsa_query(P, X, t, q + (size_t)t * hd, k, v, qi + (size_t)t * X->Hi * X->Di,
+                              w + (size_t)t * X->Hi, ki, out ? out + r * hd : NULL,
+                              index ? index + (size_t)r * T : NULL,
+                              sel ? sel + (size_t)r * X->top_k : NULL, gap ? gap + r : NULL);
+    bad |= (rc != 0);
+  }
+  return bad ? -1 : 0;
+}

@@ -39,6 +39,10 @@ class _Params(ctypes.Structure):
                 ("n", ctypes.c_int), ("w", ctypes.c_int), ("scale", ctypes.c_double)]
 
 
+class _DsaParams(ctypes.Structure):
+    _fields_ = [("Hi", ctypes.c_int), ("Di", ctypes.c_int), ("top_k", ctypes.c_int)]
+
+
 @dataclasses.dataclass(frozen=True)
 class OracleParams:
     head_dim: int
@@ -93,6 +97,9 @@ def _load():
             lib.oracle_block_select_query.argtypes = [P, ctypes.c_int, vp, vp, vp, vp, vp, vp,
                                                       ctypes.c_int, vp, vp]
             lib.oracle_block_select_query.restype = ctypes.c_int
+            lib.oracle_dsa_rows.argtypes = [P, ctypes.POINTER(_DsaParams), ctypes.c_int, vp, vp, vp,
+                                            vp, vp, vp, vp, ctypes.c_int, vp, vp, vp, vp]
+            lib.oracle_dsa_rows.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -334,3 +341,29 @@ def block_select_decode_reference(p: OracleParams, q_row, k_seq, v_seq, kmean, L
     r = block_select_query(p, t, q_row, k_seq, v_seq, kb, cmax=max(1, kb.shape[0]))
     r.update(t=t, written=written)
     return r
+
+
+# ---------------------------------------------------------------- token-level selection (DSA style)
+def dsa_rows(p: OracleParams, top_k: int, q, k, v, qi, w, ki, rows, with_index: bool = False) -> dict:
+    """Token-level top-k attention for the query rows `rows` of one sequence:
+    q [T,Hq,D], k/v [T,Hkv,D], qi [T,Hi,Di], ki [T,Di] (bf16 bits), w [T,Hi]
+    fp32.  Returns fp64 out [R,Hq,D], sel [R,top_k] (int32), gap [R] and,
+    with_index, the index scores [R,T] (entries > t are 0)."""
+    q, k, v = _c(q, np.uint16), _c(k, np.uint16), _c(v, np.uint16)
+    qi, ki, w = _c(qi, np.uint16), _c(ki, np.uint16), _c(w, np.float32)
+    rows = _c(rows, np.int32)
+    T, Hi, Di = qi.shape
+    R, Hq, D = len(rows), p.num_q_heads, p.head_dim
+    x = _DsaParams(Hi, Di, int(top_k))
+    res = {"out": np.zeros((R, Hq, D)), "sel": np.zeros((R, top_k), dtype=np.int32),
+           "gap": np.zeros(R)}
+    idx = np.zeros((R, T)) if with_index else None
+    rc = _load().oracle_dsa_rows(ctypes.byref(p.c()), ctypes.byref(x), T, _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(qi), _ptr(w), _ptr(ki), _ptr(rows), R, _ptr(res["out"]),
+                                 _ptr(idx) if with_index else None, _ptr(res["sel"]),
+                                 _ptr(res["gap"]))
+    if rc != 0:
+        raise ValueError("oracle rejected the geometry or a row index")
+    if with_index:
+        res["index"] = idx
+    return res
