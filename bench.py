@@ -399,6 +399,8 @@ def run_ours(args, rank, world):
         result["legs"]["block_select_64k"] = run_block_select_leg(dev, world)
         torch.cuda.empty_cache()
         result["legs"]["block_select_decode_64k"] = run_block_select_decode_leg(dev, world)
+        torch.cuda.empty_cache()
+        result["legs"]["token_select_8k"] = run_token_select_leg(dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = oracle_sample(cfg, inputs)
         result["cpu_baseline_1core"] = oracle_single_core()
@@ -621,6 +623,91 @@ def run_block_select_decode_leg(dev, world=1, steps=20, warmup=3):
                          "nsa_decode_b_kernel": round(stage[2], 5)}}
 
 
+TOKEN_SELECT_KERNELS = ["nsa_meta_kernel", "nsa_block_score_kernel", "nsa_token_topk_kernel",
+                        "nsa_token_attn_kernel"]
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA per clock x 2 FLOP x 1.965 GHz
+ALU_FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_token_select_leg(dev, world, steps=5, warmup=3, name="prefill_8k", index_heads=16,
+                         index_dim=128, top_k=2048):
+    """Token-level top-k attention (DSA style: indexer of `index_heads` x
+    `index_dim`, top_k tokens per query) on the geometry and length of
+    `name`: tokens/s, the index scores against the tensor peak and the
+    attention over the chosen tokens against the CUDA cores' fp32 peak."""
+    import torch
+    from sparse_attention_long_06_b200 import nsa
+    cfg = wl.CONFIGS[name]
+    inputs = wl.prefill_inputs(cfg)
+    lens = list(inputs["seqlens"])
+    T = int(inputs["cu_seqlens"][-1])
+    idx = wl.indexer_inputs(lens, index_heads, index_dim, seed=cfg.seed)
+    D, Hq = cfg.head_dim, cfg.num_q_heads
+    d = {}
+    for k in ("q", "k", "v", "cu_seqlens"):
+        a = np.ascontiguousarray(inputs[k])
+        d[k] = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+    for k in ("q_index", "w_index", "k_index"):
+        a = np.ascontiguousarray(idx[k])
+        d[k] = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(dev)
+    plan = nsa.Plan.for_config(cfg, max_batch=len(lens), max_seqlen=max(lens), max_total_tokens=T,
+                               out_dtype=nsa.OUT_BF16)
+    out = torch.empty((T, Hq, D), dtype=torch.int16, device=dev)
+    sel = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+    ws = torch.empty(plan.token_select_workspace_size(top_k), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        plan.token_select_prefill(d["q"], d["k"], d["v"], d["q_index"], d["w_index"], d["k_index"],
+                                  top_k, d["cu_seqlens"], out, ws, sel_idx=sel)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if nsa.read_device_status(ws) != nsa.NSA_OK:
+        raise RuntimeError("token select: device status after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in ev), world, dev)
+    nsa.profile_enable(True)
+    flush.zero_()
+    step()
+    stage = nsa.profile_stage_ms()
+    nsa.profile_enable(False)
+    # algorithmic work: index 2 Di per (query, indexer head, visible token);
+    # attention 4 D per (query, head, chosen token)
+    f_index = f_attn = 0
+    for Tb in lens:
+        t = np.arange(Tb, dtype=np.int64)
+        f_index += 2 * index_dim * index_heads * int((t + 1).sum())
+        f_attn += 4 * D * Hq * int(np.minimum(t + 1, top_k).sum())
+    _, _, tc_sust, src = _peaks()
+    ach_i = f_index / (stage[1] / 1e3) / 1e12
+    ach_a = f_attn / (stage[3] / 1e3) / 1e12
+    return {"metric": "token-level top-k attention tokens/s", "value": round(job_rate(T, world, ms), 1),
+            "unit": "tokens/s", "ms_per_step_median": round(ms, 4), "steps": steps,
+            "config": prefill_config(cfg, T, world) | {
+                "mode": f"token select (indexer {index_heads} x {index_dim}, top_k {top_k})"},
+            "algorithmic_flop_per_step": {"index": f_index, "attn": f_attn},
+            "stage_ms": dict(zip(TOKEN_SELECT_KERNELS, [round(x, 4) for x in stage])),
+            "rooflines": {
+                "nsa_block_score_kernel": {"bound": "tensor", "achieved": round(ach_i, 2),
+                                           "peak": tc_sust, "unit": "TFLOP/s",
+                                           "frac": round(ach_i / tc_sust, 4),
+                                           "peak_source": f"{src} bf16 sustained"},
+                "nsa_token_attn_kernel": {"bound": "alu", "achieved": round(ach_a, 2),
+                                          "peak": round(ALU_FP32_PEAK_TFLOPS, 1), "unit": "TFLOP/s",
+                                          "frac": round(ach_a / ALU_FP32_PEAK_TFLOPS, 4),
+                                          "peak_source": "fp32 FMA units x SM count x max SM clock"}}}
+
+
 def oracle_single_core(names=("tiny", "prefill_8k"), nrows=64):
     """The oracle's tokens/s on one host core for small configurations, in a
     child process with OMP_NUM_THREADS=1 (bounded: `nrows` sampled rows)."""
@@ -766,6 +853,8 @@ def main():
                     help="run only the decode leg and print its object (profiling)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="sequences in the decode leg (default: the workload's 32)")
+    ap.add_argument("--token-select-only", action="store_true",
+                    help="time only the token-level top-k leg (on --workload)")
     ap.add_argument("--block-select-decode-only", action="store_true",
                     help="time only the select-only decode leg")
     ap.add_argument("--block-select-only", action="store_true",
@@ -802,6 +891,9 @@ def main():
         torch.distributed.barrier()
     if args.decode_only:
         res = run_decode_leg(args, torch.device("cuda", torch.cuda.current_device()), world)
+    elif args.token_select_only:
+        res = run_token_select_leg(torch.device("cuda", torch.cuda.current_device()), world,
+                                   steps=max(args.steps, 3), warmup=args.warmup, name=args.workload)
     elif args.block_select_decode_only:
         res = run_block_select_decode_leg(torch.device("cuda", torch.cuda.current_device()), world,
                                           steps=max(args.steps, 20), warmup=args.warmup)

@@ -288,6 +288,43 @@ int nsa_block_select_decode(nsa_plan_t plan, const void* q, const void* k_cache,
                             int cache_capacity, void* out, int* sel_idx, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/*
+ * Token-level top-k attention (DSA style) over a packed batch.  "DeepSeek
+ * V3.2-Exp sparse attention" page (bjdmk.com.cn/news/5181035), sections 1 and
+ * 3: a light indexer with a ReLU scores every earlier token of a query and
+ * the top_k of them take part in the main attention.  Readings (the page
+ * gives no formula): the index score of token s <= t for query t is
+ * sum_j w_index[t, j] * ReLU(q_index[t, j] . k_index[s]); the top_k tokens
+ * by that score (ties to the lower index; all of them when t + 1 <= top_k)
+ * are shared by every query head; each head attends (one softmax, the plan's
+ * scale) to the keys and values of its KV group at those tokens.  The page's
+ * fp8 indexer is a precision choice not made here: the indexer runs on bf16
+ * inputs with fp32 accumulation.
+ *   q, k, v     as in nsa_prefill (the plan's heads and head dim; Hq <= 64,
+ *               Hkv <= 4 at D = 128, Hkv <= 8 at D = 64)
+ *   q_index     [T_total, index_heads, index_dim] bf16 (index_heads 1, 2, 4,
+ *               8 or 16; index_dim 64 or 128)
+ *   w_index     [T_total, index_heads] fp32 per-token head weights
+ *   k_index     [T_total, index_dim] bf16
+ *   top_k       1 <= top_k <= plan max_seqlen
+ *   out         [T_total, Hq, D] bf16 or fp32 (plan out_dtype)
+ *   sel_idx     [T_total, top_k] int32 or NULL: chosen tokens (positions in
+ *               the sequence), ascending, -1 padded
+ *   workspace   >= nsa_token_select_workspace_size(plan, top_k) bytes,
+ *               256-byte aligned: the index scores fp32 [T_total, max_seqlen]
+ *               (entry s of row t defined for s <= t) and the selection
+ * Four launches: metadata, index scores (tcgen05), top-k, attention over the
+ * chosen tokens (CUDA cores).  Plan cmp_block, cmp_stride, sel_block, top_n
+ * and window are not used.
+ */
+int nsa_token_select_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,
+                             const void* q_index, const float* w_index, const void* k_index,
+                             int index_heads, int index_dim, int top_k, const int* cu_seqlens,
+                             int batch, int total_tokens, void* out, int* sel_idx,
+                             void* workspace, size_t workspace_bytes, void* stream);
+/* Workspace bytes of nsa_token_select_prefill for `top_k` (0 when invalid). */
+size_t nsa_token_select_workspace_size(nsa_plan_t plan, int top_k);
+
 /* Rows of the packed routing-key output of nsa_block_select_prefill over
  * `total_tokens` tokens: floor(total_tokens / l'). */
 int nsa_block_rows(nsa_plan_t plan, int total_tokens);

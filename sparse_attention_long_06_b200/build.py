@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnsa_b200.so")
 SOURCES = ["nsa_api.cu", "nsa_noalloc.cu", "k_prep.cu", "k_cmp.cu", "k_win.cu", "k_slc.cu",
-           "k_decode.cu", "k_bsel.cu", "k_compress.cu"]
+           "k_decode.cu", "k_bsel.cu", "k_compress.cu", "k_dsa.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]
 

@@ -161,8 +161,9 @@ __device__ __forceinline__ BsItem bs_item(const PrefillArgs& a, int k) {
   it.T = __ldg(a.cu + b + 1) - c0;
   it.row0 = c0 + it.t0;
   it.ntok = min(a.geo.tpt, it.T - it.t0);
-  // blocks before the own block of the tile's last token
-  const int nb = (it.t0 + it.ntok - 1) >> a.geo.lg_ls;
+  // blocks before the own block of the tile's last token (token-level
+  // selection: every token up to and including it)
+  const int nb = a.token_select ? it.t0 + it.ntok : (it.t0 + it.ntok - 1) >> a.geo.lg_ls;
   it.nc = (nb + kChunk - 1) / kChunk;
   it.blk0 = a.cmp_off[b];
   return it;
@@ -170,10 +171,14 @@ __device__ __forceinline__ BsItem bs_item(const PrefillArgs& a, int k) {
 
 // One chunk's epilogue for the thread owning key `key` (TMEM lane): the G
 // columns of each token summed, stored where the key is a candidate of the
-// token (key < t / l').
+// token (key < t / l').  With token-level selection (`wts` non-null) the G
+// columns of a token are indexer heads: the score is the sum of the token's
+// head weights times ReLU(column), and keys up to and including the token
+// take part.
 template <int G>
 __device__ __forceinline__ void bs_rows(uint32_t taddr, float* srow, size_t tok_stride, int key,
-                                        int t0, int ntok, int lg_ls, bool live) {
+                                        int t0, int ntok, int lg_ls, bool live,
+                                        const float* wts) {
 #pragma unroll 2
   for (int grp = 0; grp < kTileRows / 16; ++grp) {
     float v[16];
@@ -181,11 +186,18 @@ __device__ __forceinline__ void bs_rows(uint32_t taddr, float* srow, size_t tok_
     tmem_ld_wait();
 #pragma unroll
     for (int kt = 0; kt < 16 / G; ++kt) {
-      float s = 0.f;
-#pragma unroll
-      for (int j = 0; j < G; ++j) s += v[kt * G + j];
       const int tok = (grp * 16 + kt * G) / G;
-      if (live && tok < ntok && key < ((t0 + tok) >> lg_ls)) srow[(size_t)tok * tok_stride] = s;
+      float s = 0.f;
+      if (wts) {
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+          s += (tok < ntok ? __ldg(wts + (size_t)tok * G + j) : 0.f) * fmaxf(v[kt * G + j], 0.f);
+      } else {
+#pragma unroll
+        for (int j = 0; j < G; ++j) s += v[kt * G + j];
+      }
+      const bool vis = wts ? key <= t0 + tok : key < ((t0 + tok) >> lg_ls);
+      if (live && tok < ntok && vis) srow[(size_t)tok * tok_stride] = s;
     }
   }
 }
@@ -346,12 +358,14 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         float* srow = a.scores + ((size_t)it.row0 * Hkv + it.g) * cap + key;
         const bool live = !*abort_flag;
         const uint32_t taddr = lane_addr + buf * 128;
+        // per-token indexer head weights of the tile (token-level selection)
+        const float* wts = a.token_select ? a.gates + (size_t)it.row0 * a.geo.G : nullptr;
         switch (lgG) {
-          case 0: bs_rows<1>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live); break;
-          case 1: bs_rows<2>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live); break;
-          case 2: bs_rows<4>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live); break;
-          case 3: bs_rows<8>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live); break;
-          default: bs_rows<16>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live); break;
+          case 0: bs_rows<1>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live, wts); break;
+          case 1: bs_rows<2>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live, wts); break;
+          case 2: bs_rows<4>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live, wts); break;
+          case 3: bs_rows<8>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live, wts); break;
+          default: bs_rows<16>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live, wts); break;
         }
         tc_fence_before();
         __syncwarp();

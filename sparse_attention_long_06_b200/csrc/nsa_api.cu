@@ -505,6 +505,129 @@ int nsa_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v, co
   return NSA_OK;
 }
 
+namespace {
+struct TokenSelectLayout {
+  size_t meta, scores, sel, total;
+};
+
+TokenSelectLayout token_select_layout(const nsa_plan_s* pl, int top_k) {
+  const nsa_params& p = pl->p;
+  const size_t T = (size_t)p.max_total_tokens;
+  TokenSelectLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  take(kHeaderBytes);
+  L.meta = take(sizeof(Meta) + 2 * sizeof(int) * ((size_t)p.max_batch + 1));
+  L.scores = take(T * (size_t)p.max_seqlen * sizeof(float));
+  L.sel = take(T * (size_t)top_k * sizeof(int));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+size_t nsa_token_select_workspace_size(nsa_plan_t plan, int top_k) {
+  if (!plan || top_k < 1) return 0;
+  return token_select_layout(plan, top_k).total;
+}
+
+int nsa_token_select_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,
+                             const void* q_index, const float* w_index, const void* k_index,
+                             int index_heads, int index_dim, int top_k, const int* cu_seqlens,
+                             int batch, int total_tokens, void* out, int* sel_idx,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_launches = 0;
+  if (!plan) return NSA_ERR_INVALID_ARG;
+  const nsa_params& p = plan->p;
+  const Geometry& geo = plan->geo;
+  if (batch <= 0 || batch > p.max_batch || total_tokens < 0 ||
+      total_tokens > p.max_total_tokens || top_k < 1 || top_k > p.max_seqlen || index_heads < 1 ||
+      index_dim < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (!is_pow2_le16(index_heads) || (index_dim != 64 && index_dim != 128) || geo.Hq > 64 ||
+      geo.Hkv > (geo.D == 128 ? 4 : 8))
+    return NSA_ERR_UNSUPPORTED;
+  if (!cu_seqlens || !workspace) return workspace ? NSA_ERR_INVALID_ARG : NSA_ERR_WORKSPACE;
+  const TokenSelectLayout L = token_select_layout(plan, top_k);
+  if (workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return NSA_ERR_WORKSPACE;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !q_index || !w_index || !k_index || !out) return NSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_index) ||
+        !aligned16(k_index) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w_index) & 3u) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(sel_idx) & 3u))
+      return NSA_ERR_MISALIGNED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  // the indexer's geometry: its heads are the columns of a token, one key head
+  Geometry gi = geo;
+  gi.D = index_dim;
+  gi.Hq = index_heads;
+  gi.Hkv = 1;
+  gi.G = index_heads;
+  gi.lg_G = __builtin_ctz(index_heads);
+  gi.tpt = kTileRows / index_heads;
+  gi.l = gi.d = gi.ls = 1;
+  gi.lg_ls = 0;
+  gi.remap = 0;
+  gi.cmp_cap = p.max_seqlen;  // row stride of the index-score table
+  PrefillArgs ai{};
+  ai.geo = gi;
+  ai.batch = batch;
+  ai.total_tokens = total_tokens;
+  ai.cmp_rows = total_tokens;
+  ai.q = static_cast<const uint16_t*>(q_index);
+  ai.k_cmp = static_cast<uint16_t*>(const_cast<void*>(k_index));
+  ai.gates = w_index;
+  ai.cu = cu_seqlens;
+  ai.status = reinterpret_cast<int*>(ws);
+  ai.meta = reinterpret_cast<Meta*>(ws + L.meta);
+  ai.cmp_off = reinterpret_cast<int*>(ws + L.meta + sizeof(Meta));
+  ai.tile_off = ai.cmp_off + (batch + 1);
+  ai.scores = reinterpret_cast<float*>(ws + L.scores);
+  ai.sel = sel_idx ? sel_idx : reinterpret_cast<int*>(ws + L.sel);
+  ai.token_select = 1;
+  PrefillArgs am = ai;  // the main attention: the plan's geometry
+  am.geo = geo;
+  am.q = static_cast<const uint16_t*>(q);
+  am.k = static_cast<const uint16_t*>(k);
+  am.v = static_cast<const uint16_t*>(v);
+  am.out = out;
+  am.token_select = 0;
+
+  if (cudaMemsetAsync(ai.status, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
+  if (total_tokens == 0) {
+    if (cudaMemsetAsync(ai.meta, 0, sizeof(Meta), s) != cudaSuccess) return NSA_ERR_CUDA;
+    return NSA_OK;
+  }
+  PrefillMaps m;
+  memset(&m, 0, sizeof(m));
+  bool ok = encode3d(&m.q, q_index, index_dim, index_heads, total_tokens, index_heads, gi.tpt) &&
+            encode3d(&m.kc, k_index, index_dim, 1, total_tokens, 1, kChunk);
+  if (!ok) return NSA_ERR_CUDA;
+  const int sms = num_sms_current();
+  if (sms <= 0) return NSA_ERR_CUDA;
+  int launches = 0;
+  prof_reset();
+  prof_mark(s);
+  cudaError_t e = launch_meta(ai, s);
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_block_score(ai, m, sms, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_token_topk(ai, top_k, s); }
+  if (e == cudaSuccess) { ++launches; prof_mark(s); e = launch_token_attn(am, top_k, s); }
+  prof_mark(s);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "nsa_token_select_prefill: launch failed: %s\n", cudaGetErrorString(e));
+    return NSA_ERR_CUDA;
+  }
+  g_last_launches = launches + 1;
+  return NSA_OK;
+}
+
 int nsa_block_rows(nsa_plan_t plan, int total_tokens) {
   if (!plan || total_tokens < 0) return -1;
   return total_tokens / plan->geo.ls;

@@ -78,6 +78,9 @@ struct PrefillArgs {
   float* o_win;   // [T, Hq, D] g_win * O_win
   int select_only;  // select-only block attention: routing scores, the own
                     // block forced into the selection, output = selected branch
+  int token_select; // token-level top-k (index scores into `scores`, geometry of
+                    // the indexer: G = indexer heads, Hkv = 1, D = indexer dim;
+                    // `gates` holds the per-token head weights [T, G])
   int split_q;    // PrefillMaps.q_split is valid (Hq >= 16)
   int split_v;    // PrefillMaps.v_split is valid (l' = 64)
 };
@@ -200,6 +203,8 @@ cudaError_t launch_slc(const PrefillArgs& a, const PrefillMaps& m, int num_sms, 
 cudaError_t launch_block_mean(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_block_score(const PrefillArgs& a, const PrefillMaps& m, int num_sms,
                                cudaStream_t s);
+cudaError_t launch_token_topk(const PrefillArgs& a, int top_k, cudaStream_t s);
+cudaError_t launch_token_attn(const PrefillArgs& a, int top_k, cudaStream_t s);
 cudaError_t launch_timeout_selftest(int* status, long long cycles, cudaStream_t s);
 cudaError_t launch_decode_compress(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_block_mean(const DecodeArgs& a, cudaStream_t s);

@@ -31,7 +31,8 @@ EXPORTED = ["nsa_plan_create", "nsa_plan_destroy", "nsa_workspace_size", "nsa_wo
             "nsa_selftest_timeout", "nsa_strerror", "nsa_last_launch_count",
             "nsa_profile_enable", "nsa_profile_stage_ms", "nsa_prefill_noalloc",
             "nsa_plan", "nsa_noalloc_read_device_status", "nsa_block_select_prefill",
-            "nsa_block_rows", "nsa_block_select_decode"]
+            "nsa_block_rows", "nsa_block_select_decode", "nsa_token_select_prefill",
+            "nsa_token_select_workspace_size"]
 
 
 class NsaError(RuntimeError):
@@ -84,6 +85,11 @@ def lib():
             L.nsa_block_select_prefill.restype = i
             L.nsa_block_select_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp]
             L.nsa_block_select_decode.restype = i
+            L.nsa_token_select_prefill.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, vp, i, i,
+                                                    vp, vp, vp, sz, vp]
+            L.nsa_token_select_prefill.restype = i
+            L.nsa_token_select_workspace_size.argtypes = [vp, i]
+            L.nsa_token_select_workspace_size.restype = sz
             L.nsa_block_rows.argtypes = [vp, i]
             L.nsa_block_rows.restype = i
             L.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -213,6 +219,25 @@ class Plan:
                                             workspace.numel() * workspace.element_size(),
                                             _stream(stream))
         _check(rc, "nsa_block_select_prefill")
+
+    def token_select_workspace_size(self, top_k: int) -> int:
+        return int(lib().nsa_token_select_workspace_size(self.handle, int(top_k)))
+
+    def token_select_prefill(self, q, k, v, q_index, w_index, k_index, top_k, cu_seqlens, out,
+                             workspace, sel_idx=None, stream=None):
+        """Token-level top-k attention over a packed batch: an indexer
+        (q_index [T, Hi, Di], w_index [T, Hi], k_index [T, Di]) picks each
+        query's top_k earlier tokens, every query head attends to them."""
+        batch = cu_seqlens.numel() - 1
+        total = q.shape[0]
+        rc = lib().nsa_token_select_prefill(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(q_index),
+                                            _ptr(w_index), _ptr(k_index), q_index.shape[1],
+                                            q_index.shape[2], int(top_k), _ptr(cu_seqlens),
+                                            batch, total, _ptr(out), _ptr(sel_idx),
+                                            _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(stream))
+        _check(rc, "nsa_token_select_prefill")
 
     def block_select_decode(self, q, k_cache, v_cache, k_mean_cache, seqlens, out, workspace,
                             sel_idx=None, stream=None):

@@ -243,3 +243,14 @@ def decode_inputs(cfg: NsaConfig, lengths: list[int] | None = None, capacity: in
     out = {key: np.stack([s[key] for s in seqs]) for key in ("q", "k", "v", "kc", "vc", "gates")}
     out.update(w_k=wk, w_v=wv, seqlens=np.asarray(lens, dtype=np.int32), capacity=cap)
     return out
+
+
+def indexer_inputs(seqlens: list[int], heads: int, dim: int, seed: int) -> dict:
+    """Indexer tensors of a packed batch for token-level selection: queries
+    q_index [T, heads, dim] and keys k_index [T, dim] N(0,1) rounded to bf16,
+    per-token head weights w_index [T, heads] ~ U(0,1)."""
+    T = int(sum(seqlens))
+    rng = np.random.default_rng([seed, 97])
+    return {"q_index": bf16_bits(rng.standard_normal((T, heads, dim), dtype=np.float32)),
+            "k_index": bf16_bits(rng.standard_normal((T, dim), dtype=np.float32)),
+            "w_index": rng.random((T, heads), dtype=np.float32)}

@@ -230,6 +230,40 @@ def test_block_select_decode_rejects_bad_arguments_before_launch(L):
     assert L.nsa_last_launch_count() == 0
 
 
+def test_token_select_sizes_and_bad_arguments(L):
+    p = nsa.Plan(**_params(max_total_tokens=4096, max_seqlen=4096))
+    wsb = p.token_select_workspace_size(2048)
+    assert wsb >= 4096 * 4096 * 4 + 4096 * 2048 * 4  # index scores + selection
+    assert p.token_select_workspace_size(0) == 0
+    fake = 1 << 20  # an aligned address that is never dereferenced
+    args = dict(q=fake, k=fake, v=fake, qi=fake, wi=fake, ki=fake, hi=16, di=128, top_k=2048,
+                cu=fake, batch=1, total=4096, out=fake, sel=None, ws=fake, wsb=wsb)
+
+    def call(**over):
+        a = dict(args)
+        a.update(over)
+        return L.nsa_token_select_prefill(p.handle, a["q"], a["k"], a["v"], a["qi"], a["wi"],
+                                          a["ki"], a["hi"], a["di"], a["top_k"], a["cu"],
+                                          a["batch"], a["total"], a["out"], a["sel"], a["ws"],
+                                          a["wsb"], None)
+
+    assert call(top_k=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(top_k=4097) == nsa.NSA_ERR_INVALID_ARG       # above max_seqlen
+    assert call(hi=3) == nsa.NSA_ERR_UNSUPPORTED
+    assert call(di=96) == nsa.NSA_ERR_UNSUPPORTED
+    assert call(qi=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(batch=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(ws=None) == nsa.NSA_ERR_WORKSPACE
+    assert call(wsb=wsb - 1) == nsa.NSA_ERR_WORKSPACE
+    assert call(ki=fake + 8) == nsa.NSA_ERR_MISALIGNED
+    assert call(wi=fake + 2) == nsa.NSA_ERR_MISALIGNED
+    wide = nsa.Plan(**_params(num_q_heads=128, num_kv_heads=8))
+    assert L.nsa_token_select_prefill(wide.handle, fake, fake, fake, fake, fake, fake, 16, 128, 16,
+                                      fake, 1, 16, fake, None, fake, 1 << 40,
+                                      None) == nsa.NSA_ERR_UNSUPPORTED  # Hq > 64
+    assert L.nsa_last_launch_count() == 0
+
+
 def test_noalloc_rejects_plans_beyond_its_static_array(L):
     big = nsa.Plan(**_params())  # 64k tokens: several GB of workspace
     assert big.workspace_size() > 32 << 20
