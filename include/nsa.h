@@ -311,10 +311,12 @@ int nsa_block_select_decode(nsa_plan_t plan, const void* q, const void* k_cache,
  *   sel_idx     [T_total, top_k] int32 or NULL: chosen tokens (positions in
  *               the sequence), ascending, -1 padded
  *   workspace   >= nsa_token_select_workspace_size(plan, top_k) bytes,
- *               256-byte aligned: the index scores fp32 [T_total, max_seqlen]
- *               (entry s of row t defined for s <= t) and the selection
- * Four launches: metadata, index scores (tcgen05), top-k, attention over the
- * chosen tokens (CUDA cores).  Plan cmp_block, cmp_stride, sel_block, top_n
+ *               256-byte aligned: the index scores fp32 [T_total, S] with
+ *               S = max_seqlen rounded up to a multiple of 4 (entry s of row
+ *               t defined for s <= t) and the selection
+ * Four launches: metadata, index scores (tcgen05), top-k (a radix select,
+ * one CTA per row), attention over the chosen tokens (mma.sync tensor
+ * cores).  Plan cmp_block, cmp_stride, sel_block, top_n
  * and window are not used.
  */
 int nsa_token_select_prefill(nsa_plan_t plan, const void* q, const void* k, const void* v,

@@ -18,10 +18,13 @@ namespace nsa {
 using namespace sm100;
 
 // ------------------------------------------------------------------ selection
-// One warp per query token t: the top_k of its t + 1 index scores, ascending,
-// -1 padded (the register path for rows of at most 1024 candidates and
-// top_k <= 32, else the radix select).
-__global__ void __launch_bounds__(256) nsa_token_topk_kernel(PrefillArgs a, int top_k) {
+// Each query token t selects the top_k of its t + 1 index scores (score
+// descending, ties to the lower token), written in ascending token order and
+// padded with -1 when t + 1 < top_k.
+//
+// Short rows (at most 1024 candidates, top_k <= 32): one warp per row, the
+// register path of the block selection.
+__global__ void __launch_bounds__(256) nsa_token_topk_short_kernel(PrefillArgs a, int top_k) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
   __shared__ unsigned long long cand_all[8][kTopnCand];
@@ -35,9 +38,175 @@ __global__ void __launch_bounds__(256) nsa_token_topk_kernel(PrefillArgs a, int 
   auto put = [&](int i, int j) { out[i] = j; };
   auto score = [&](int j) { return S[j]; };
   const int ncand = t + 1;
-  if (ncand <= 1024 && top_k <= 32 && warp_topn_regs(score, ncand, ncand, top_k, cand_all[warp], put))
-    return;
+  if (warp_topn_regs(score, ncand, ncand, top_k, cand_all[warp], put)) return;
   warp_topn(score, ncand, ncand, top_k, hist_all[warp], put);
+}
+
+// Rows of any length: one CTA per row, rows taken from the last token back
+// so that the longest rows of a sequence start first.  The row (16-byte
+// aligned: the table's row stride is a multiple of four) is read as float4.
+// A radix select on the 32-bit order-preserving score key with digits of
+// 11, 11 and 10 bits finds the key of the top_k-th largest score: each pass
+// histograms, in shared memory, the digit of the keys that share the prefix
+// found so far (the lanes of a warp holding the same digit add their count
+// with one atomic), and a block scan over the bins picks the digit holding
+// the remaining rank.  The passes stop early once every key of that digit is
+// taken.  A last pass compacts the row in token order: a key above the
+// threshold is taken, a key equal to it while fewer than the remaining rank
+// of equal keys have been taken before it; one block scan per tile gives
+// each taken token its output position.
+namespace {
+
+constexpr int kTkThreads = 512;
+constexpr int kTkWarps = kTkThreads / 32;
+constexpr int kTkBins = 2048;
+constexpr int kTkBinsPerThread = kTkBins / kTkThreads;
+
+// Exclusive prefix of v over the CTA's threads in thread order; `total`
+// receives the sum over all threads.
+__device__ __forceinline__ unsigned tk_excl_scan(unsigned v, unsigned* wsum, unsigned& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  unsigned before = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kTkWarps; ++w) {
+    const unsigned x = wsum[w];
+    before += w < warp ? x : 0u;
+    tot += x;
+  }
+  __syncthreads();
+  total = tot;
+  return before + inc - v;
+}
+
+__device__ __forceinline__ float4 tk_load(const float* S, int q, int nq) {
+  return q < nq ? __ldg(reinterpret_cast<const float4*>(S) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kTkThreads) nsa_token_topk_kernel(PrefillArgs a, int top_k) {
+  if (a.meta->bad) return;
+  __shared__ unsigned hist[kTkBins];
+  __shared__ unsigned wsum[kTkWarps];
+  __shared__ unsigned ctl[2];
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int tg = a.total_tokens - 1 - (int)blockIdx.x;
+  const int b = seq_of_token(a.cu, a.batch, tg);
+  const int ncand = tg - __ldg(a.cu + b) + 1;
+  const float* S = a.scores + (size_t)tg * a.geo.cmp_cap;
+  int* out = a.sel + (size_t)tg * top_k;
+  if (ncand <= top_k) {
+    for (int j = tid; j < top_k; j += kTkThreads) out[j] = j < ncand ? j : -1;
+    return;
+  }
+  const int nq = (ncand + 3) >> 2;  // float4 words of the row
+  uint32_t prefix = 0, pmask = 0;
+  unsigned k = (unsigned)top_k;  // rank still to be found inside the prefix class
+  int shift = 21;
+  for (int pass = 0; pass < 3; ++pass) {
+    shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+    for (int i = tid; i < kTkBins; i += kTkThreads) hist[i] = 0;
+    __syncthreads();
+    for (int base = 0; base < nq; base += 4 * kTkThreads) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = tk_load(S, base + u * kTkThreads + tid, nq);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j0 = 4 * (base + u * kTkThreads + tid);
+        const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t x = score_key(f[e]);
+          const bool in = j0 + e < ncand && (x & pmask) == prefix;
+          if (__any_sync(0xffffffffu, in)) {
+            const uint32_t digit = in ? (x >> shift) & dmask : 0xFFFFFFFFu;
+            const unsigned peers = __match_any_sync(0xffffffffu, digit);
+            if (in && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], (unsigned)__popc(peers));
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // thread i owns bins [i * 4, i * 4 + 4); higher threads hold higher digits
+    unsigned c[kTkBinsPerThread], mine = 0;
+#pragma unroll
+    for (int e = 0; e < kTkBinsPerThread; ++e) {
+      c[e] = hist[tid * kTkBinsPerThread + e];
+      mine += c[e];
+    }
+    unsigned total;
+    const unsigned excl = tk_excl_scan(mine, wsum, total);
+    const unsigned above = total - excl - mine;  // keys in the class with a higher digit
+    if (above < k && k <= above + mine) {
+      unsigned acc = above;
+      int d = tid * kTkBinsPerThread;
+#pragma unroll
+      for (int e = kTkBinsPerThread - 1; e >= 0; --e) {
+        if (acc + c[e] >= k) {
+          d = tid * kTkBinsPerThread + e;
+          break;
+        }
+        acc += c[e];
+      }
+      ctl[0] = (unsigned)d;
+      ctl[1] = acc;
+    }
+    __syncthreads();
+    const uint32_t digit = ctl[0];
+    k -= ctl[1];
+    prefix |= digit << shift;
+    pmask |= dmask << shift;
+    const bool all_taken = hist[digit] == k;
+    __syncthreads();
+    if (all_taken) break;
+  }
+  // keys compared on their bits from `shift` up: above thr taken, the first
+  // `krem` equal to it taken
+  const uint32_t thr = prefix >> shift;
+  const unsigned krem = k;
+  unsigned written = 0, ties = 0;
+  float4 nxt = tk_load(S, tid, nq);
+  for (int base = 0; base < nq && written < (unsigned)top_k; base += kTkThreads) {
+    const float4 cur = nxt;
+    nxt = tk_load(S, base + kTkThreads + tid, nq);
+    const int j0 = 4 * (base + tid);
+    const float f[4] = {cur.x, cur.y, cur.z, cur.w};
+    unsigned gtm = 0, eqm = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t xt = score_key(f[e]) >> shift;
+      const bool valid = j0 + e < ncand;
+      gtm |= (valid && xt > thr) ? 1u << e : 0u;
+      eqm |= (valid && xt == thr) ? 1u << e : 0u;
+    }
+    unsigned tot;
+    const unsigned excl = tk_excl_scan(((unsigned)__popc(eqm) << 16) | (unsigned)__popc(gtm), wsum, tot);
+    const unsigned rem = krem > ties ? krem - ties : 0u;  // equal keys still to take
+    unsigned eqb = excl >> 16;
+    unsigned pos = written + (excl & 0xFFFFu) + min(eqb, rem);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      bool take = (gtm >> e) & 1u;
+      if ((eqm >> e) & 1u) take = eqb++ < rem;
+      if (take) {
+        if (pos < (unsigned)top_k) out[pos] = j0 + e;
+        ++pos;
+      }
+    }
+    written += (tot & 0xFFFFu) + min(tot >> 16, rem);
+    ties += tot >> 16;
+  }
+  for (unsigned j = written + tid; j < (unsigned)top_k; j += kTkThreads) out[j] = -1;
 }
 
 // ------------------------------------------------------------------ attention
@@ -274,7 +443,10 @@ cudaError_t launch_token_attn_t(const PrefillArgs& a, int top_k, cudaStream_t s)
 
 cudaError_t launch_token_topk(const PrefillArgs& a, int top_k, cudaStream_t s) {
   if (a.total_tokens <= 0) return cudaSuccess;
-  nsa_token_topk_kernel<<<(unsigned)((a.total_tokens + 7) / 8), 256, 0, s>>>(a, top_k);
+  if (a.geo.cmp_cap <= 1024 && top_k <= 32)
+    nsa_token_topk_short_kernel<<<(unsigned)((a.total_tokens + 7) / 8), 256, 0, s>>>(a, top_k);
+  else
+    nsa_token_topk_kernel<<<(unsigned)a.total_tokens, kTkThreads, 0, s>>>(a, top_k);
   return cudaGetLastError();
 }
 

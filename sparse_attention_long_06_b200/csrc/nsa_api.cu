@@ -510,6 +510,9 @@ struct TokenSelectLayout {
   size_t meta, scores, sel, total;
 };
 
+// row stride (floats) of the index-score table: rows start on 16 bytes
+int token_score_stride(int max_seqlen) { return (max_seqlen + 3) & ~3; }
+
 TokenSelectLayout token_select_layout(const nsa_plan_s* pl, int top_k) {
   const nsa_params& p = pl->p;
   const size_t T = (size_t)p.max_total_tokens;
@@ -522,7 +525,7 @@ TokenSelectLayout token_select_layout(const nsa_plan_s* pl, int top_k) {
   };
   take(kHeaderBytes);
   L.meta = take(sizeof(Meta) + 2 * sizeof(int) * ((size_t)p.max_batch + 1));
-  L.scores = take(T * (size_t)p.max_seqlen * sizeof(float));
+  L.scores = take(T * (size_t)token_score_stride(p.max_seqlen) * sizeof(float));
   L.sel = take(T * (size_t)top_k * sizeof(int));
   L.total = off;
   return L;
@@ -575,7 +578,7 @@ int nsa_token_select_prefill(nsa_plan_t plan, const void* q, const void* k, cons
   gi.l = gi.d = gi.ls = 1;
   gi.lg_ls = 0;
   gi.remap = 0;
-  gi.cmp_cap = p.max_seqlen;  // row stride of the index-score table
+  gi.cmp_cap = token_score_stride(p.max_seqlen);  // row stride of the index-score table
   PrefillArgs ai{};
   ai.geo = gi;
   ai.batch = batch;

@@ -51,7 +51,8 @@ def run_token_select(cfg, inputs, idx, top_k, out_dtype=nsa.OUT_F32):
     # index scores: the workspace region after the header and the metadata
     wsn = ws.cpu().numpy()
     meta = 256 + ((16 + 8 * (len(lens) + 1) + 255) // 256) * 256
-    res["index"] = wsn[meta:meta + total * max_seqlen * 4].view(np.float32).reshape(total, max_seqlen).copy()
+    stride = (max_seqlen + 3) // 4 * 4  # row stride of the index-score table
+    res["index"] = wsn[meta:meta + total * stride * 4].view(np.float32).reshape(total, stride).copy()
     return res
 
 
@@ -138,7 +139,8 @@ def test_token_select_8k_top2048_and_bf16_output():
                                   wl.bf16_bits(rb["out"].astype(np.float32)))
 
 
-def test_token_select_relu_floor_ties_go_to_the_lowest_tokens():
+@pytest.mark.parametrize("top_k", [24, 40])  # warp path (top_k <= 32), CTA path
+def test_token_select_relu_floor_ties_go_to_the_lowest_tokens(top_k):
     # every indexer product negative: all scores are exactly 0 and the
     # lowest top_k tokens are chosen
     cfg = _cfg("ts_floor", 64, 4, 1)
@@ -147,11 +149,36 @@ def test_token_select_relu_floor_ties_go_to_the_lowest_tokens():
     idx = wl.indexer_inputs(lens, 4, 64, seed=9)
     idx["q_index"] = wl.bf16_bits(np.abs(wl.bf16_to_f32(idx["q_index"])))
     idx["k_index"] = wl.bf16_bits(-np.abs(wl.bf16_to_f32(idx["k_index"])) - 0.01)
-    res = run_token_select(cfg, inp, idx, 24)
-    rep = check_token_select(cfg, inp, idx, res, 24, [np.arange(500)])
+    res = run_token_select(cfg, inp, idx, top_k)
+    rep = check_token_select(cfg, inp, idx, res, top_k, [np.arange(500)])
     assert rep["idx_near_tie"] == 0
     assert np.all(res["index"][np.arange(500)[:, None] >= np.arange(500)[None, :]] == 0.0)
-    assert (res["sel"][24:] == np.arange(24)[None, :]).all()
+    assert (res["sel"][top_k:] == np.arange(top_k)[None, :]).all()
+
+
+def test_token_select_partial_ties_at_the_threshold():
+    # index scores on a coarse grid (many equal values around every row's
+    # threshold): the top-k takes the lowest tokens among the equal ones
+    cfg = _cfg("ts_grid", 64, 4, 1)
+    lens = [1500, 301]
+    inp = wl.prefill_inputs(cfg, seqlens=lens)
+    idx = wl.indexer_inputs(lens, 1, 64, seed=11)
+    rng = np.random.default_rng(12)
+    T = sum(lens)
+    # one indexer head of weight 1, a query with one unit coordinate and keys
+    # of 0..7 on that coordinate: the score of token s is exactly k_s[0]
+    qi = np.zeros((T, 1, 64), dtype=np.float32)
+    qi[:, 0, 0] = 1.0
+    ki = np.zeros((T, 64), dtype=np.float32)
+    ki[:, 0] = rng.integers(0, 8, size=T).astype(np.float32)
+    idx["q_index"] = wl.bf16_bits(qi)
+    idx["k_index"] = wl.bf16_bits(ki)
+    idx["w_index"] = np.ones((T, 1), dtype=np.float32)
+    for top_k in (33, 200):
+        res = run_token_select(cfg, inp, idx, top_k)
+        rows = [np.arange(T_b) for T_b in lens]
+        rep = check_token_select(cfg, inp, idx, res, top_k, rows)
+        assert rep["idx_near_tie"] == 0 and rep["idx_mismatch"] == 0
 
 
 def test_token_select_rejects_inconsistent_seqlens_on_device():
