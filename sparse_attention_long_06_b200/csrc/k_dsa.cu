@@ -214,9 +214,9 @@ __global__ void __launch_bounds__(kTkThreads) nsa_token_topk_kernel(PrefillArgs 
 // are the 16 rows of mma.sync m16n8k16 bf16 products with fp32 accumulators
 // (rows past G are zero queries whose results are dropped).  The selected
 // tokens are taken 32 at a time; their keys and values for every group are
-// copied (16-byte cp.async, double buffered) into shared memory rows padded
-// to D + 8 elements, so that the eight rows an operand fragment spans fall
-// in different banks.  Per step and warp: S = Q K^T (queries as A fragments
+// copied (16-byte cp.async, a ring of three steps: two in flight while one is
+// computed) into shared memory rows padded to D + 8 elements, so that the
+// eight rows an operand fragment spans fall in different banks.  Per step and warp: S = Q K^T (queries as A fragments
 // kept in registers, keys read as B fragments), an online softmax on the
 // accumulator fragments (row statistics over the four threads of a quad),
 // then O += P V with P re-packed from the S fragments as A fragments and V
@@ -247,17 +247,30 @@ __device__ __forceinline__ void ldmatrix_x2_trans(uint32_t& r0, uint32_t& r1, ui
 }
 
 template <int D, int HKV>
+struct TokenAttnCfg {
+  static constexpr int RS = D + 8;                          // padded row, elements
+  static constexpr int kThreads = HKV * 32;
+  static constexpr int kRows = HKV * kDsaKeys;              // rows of one step
+  static constexpr int kBufBytes = kRows * RS * 2;          // keys (or values) of one step
+  static constexpr int kStages = 3;                         // ring depth
+  static constexpr int kSmem = 2 * kStages * kBufBytes;
+  static constexpr int CPR = D / 8;                         // 16-byte chunks of a row
+  static constexpr int RPI = kThreads / CPR;                // rows copied per pass
+  static constexpr int JK = kDsaKeys / RPI;                 // distinct keys per thread
+  static_assert(kThreads % CPR == 0 && kDsaKeys % RPI == 0, "copy mapping");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+};
+
+template <int D, int HKV>
 __global__ void __launch_bounds__(HKV * 32) nsa_token_attn_kernel(PrefillArgs a, int top_k) {
   if (a.meta->bad) return;
-  constexpr int RS = D + 8;                         // padded row, elements
-  constexpr int kRows = HKV * kDsaKeys;             // rows of one step
-  constexpr int kBufBytes = kRows * RS * 2;         // keys (or values) of one step
+  using C = TokenAttnCfg<D, HKV>;
+  constexpr int RS = C::RS, NST = C::kStages, kBufBytes = C::kBufBytes;
   constexpr int KS = D / 16;                        // k-steps of q . k
   constexpr int NT = D / 8;                         // n-tiles of O
   extern __shared__ __align__(16) uint8_t sm[];
-  uint8_t* kbuf = sm;                               // [2][HKV][keys][RS]
-  uint8_t* vbuf = sm + 2 * kBufBytes;               // [2][HKV][keys][RS]
-  int* idx = reinterpret_cast<int*>(sm + 4 * kBufBytes);  // [2][keys]
+  uint8_t* kbuf = sm;                               // [NST][HKV][keys][RS]
+  uint8_t* vbuf = sm + NST * kBufBytes;             // [NST][HKV][keys][RS]
   const int Hq = a.geo.Hq, G = Hq / HKV;
   const int tg = blockIdx.x;
   if (tg >= a.total_tokens) return;
@@ -286,24 +299,35 @@ __global__ void __launch_bounds__(HKV * 32) nsa_token_attn_kernel(PrefillArgs a,
     }
   }
   const int nsteps = (nsel + kDsaKeys - 1) / kDsaKeys;
-  auto issue = [&](int step) {
-    const int buf = step & 1;
-    if (threadIdx.x < kDsaKeys) {
-      const int i = step * kDsaKeys + threadIdx.x;
-      idx[buf * kDsaKeys + threadIdx.x] = i < nsel ? __ldg(sel + i) : -1;
+  // thread i copies chunk i % CPR of rows i / CPR + RPI * j: keys
+  // i / CPR + RPI * jk of every group
+  const int c8 = threadIdx.x % C::CPR, r0 = threadIdx.x / C::CPR;
+  // the selected positions of a step, loaded one step before its copies
+  // are issued so that the load's latency is hidden behind a step's math
+  auto load_sel = [&](int step, int (&sv)[C::JK]) {
+#pragma unroll
+    for (int jk = 0; jk < C::JK; ++jk) {
+      const int i = step * kDsaKeys + r0 + C::RPI * jk;
+      sv[jk] = i < nsel ? __ldg(sel + i) : -1;
     }
-    const uint32_t kb = smem_u32(kbuf + buf * kBufBytes), vb = smem_u32(vbuf + buf * kBufBytes);
-    for (int e = threadIdx.x; e < kRows * (D / 8); e += HKV * 32) {
-      const int c8 = e % (D / 8), row = e / (D / 8);  // row = group * keys + key
-      const int key = row % kDsaKeys, gg = row / kDsaKeys;
-      const int i = step * kDsaKeys + key;
-      const int s = i < nsel ? __ldg(sel + i) : -1;
-      const bool ok = s >= 0;
-      const size_t src = ((size_t)(cu0 + (ok ? s : 0)) * HKV + gg) * D + c8 * 8;
-      cp_async16(kb + (row * RS + c8 * 8) * 2, a.k + src, ok);
-      cp_async16(vb + (row * RS + c8 * 8) * 2, a.v + src, ok);
+  };
+  auto issue = [&](int step, const int (&sv)[C::JK]) {
+    if (step < nsteps) {
+      const int buf = step % NST;
+      const uint32_t kb = smem_u32(kbuf + buf * kBufBytes), vb = smem_u32(vbuf + buf * kBufBytes);
+#pragma unroll
+      for (int gg = 0; gg < HKV; ++gg) {
+#pragma unroll
+        for (int jk = 0; jk < C::JK; ++jk) {
+          const int row = gg * kDsaKeys + r0 + C::RPI * jk;
+          const bool ok = sv[jk] >= 0;
+          const size_t src = ((size_t)(cu0 + (ok ? sv[jk] : 0)) * HKV + gg) * D + c8 * 8;
+          cp_async16(kb + (row * RS + c8 * 8) * 2, a.k + src, ok);
+          cp_async16(vb + (row * RS + c8 * 8) * 2, a.v + src, ok);
+        }
+      }
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");  // empty past the last step
   };
 
   float o[NT][4];
@@ -313,16 +337,20 @@ __global__ void __launch_bounds__(HKV * 32) nsa_token_attn_kernel(PrefillArgs a,
     for (int c = 0; c < 4; ++c) o[n][c] = 0.f;
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};  // rows gid, gid + 8
   const float sl2 = a.geo.scale_log2;
-  if (nsteps > 0) issue(0);
+  int sv[C::JK];
+#pragma unroll
+  for (int st = 0; st < NST - 1; ++st) {
+    load_sel(st, sv);
+    issue(st, sv);
+  }
+  load_sel(NST - 1, sv);
   for (int step = 0; step < nsteps; ++step) {
-    const int buf = step & 1;
-    if (step + 1 < nsteps) {
-      issue(step + 1);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-    }
-    __syncthreads();
+    const int buf = step % NST;
+    // one group committed per step: the NST - 2 after this step's may pend
+    asm volatile("cp.async.wait_group %0;" ::"n"(NST - 2) : "memory");
+    __syncthreads();  // this step's rows visible; step - 1's buffer free
+    issue(step + NST - 1, sv);
+    load_sel(step + NST, sv);
     const uint16_t* kr = reinterpret_cast<const uint16_t*>(kbuf + buf * kBufBytes) + (size_t)g * kDsaKeys * RS;
     const uint32_t vaddr = smem_u32(vbuf + buf * kBufBytes) + (uint32_t)(g * kDsaKeys * RS * 2);
     // S = Q K^T: four n-tiles of 8 keys
@@ -346,7 +374,7 @@ __global__ void __launch_bounds__(HKV * 32) nsa_token_attn_kernel(PrefillArgs a,
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int key = nt * 8 + tig * 2 + (c & 1);
-        const bool on = idx[buf * kDsaKeys + key] >= 0;
+        const bool on = step * kDsaKeys + key < nsel;
         sacc[nt][c] = on ? sacc[nt][c] * sl2 : -INFINITY;
         mloc[c >> 1] = fmaxf(mloc[c >> 1], sacc[nt][c]);
       }
@@ -400,8 +428,8 @@ __global__ void __launch_bounds__(HKV * 32) nsa_token_attn_kernel(PrefillArgs a,
         mma_bf16_16816(o[n], pa[kk], b0, b1);
       }
     }
-    __syncthreads();  // the buffer is refilled two steps on
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   // rows gid and gid + 8 of the group: heads g * G + row
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -424,8 +452,7 @@ __global__ void __launch_bounds__(HKV * 32) nsa_token_attn_kernel(PrefillArgs a,
 
 template <int D, int HKV>
 cudaError_t launch_token_attn_t(const PrefillArgs& a, int top_k, cudaStream_t s) {
-  constexpr int RS = D + 8;
-  const size_t smem = 4 * (size_t)HKV * kDsaKeys * RS * 2 + 2 * kDsaKeys * 4;
+  const size_t smem = TokenAttnCfg<D, HKV>::kSmem;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -458,8 +485,7 @@ cudaError_t launch_token_attn(const PrefillArgs& a, int top_k, cudaStream_t s) {
     switch (H) {
       case 1: return launch_token_attn_t<128, 1>(a, top_k, s);
       case 2: return launch_token_attn_t<128, 2>(a, top_k, s);
-      case 4: return launch_token_attn_t<128, 4>(a, top_k, s);
-      default: return launch_token_attn_t<128, 8>(a, top_k, s);
+      default: return launch_token_attn_t<128, 4>(a, top_k, s);  // Hkv <= 4 at D = 128
     }
   }
   switch (H) {
