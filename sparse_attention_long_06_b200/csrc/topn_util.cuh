@@ -108,8 +108,9 @@ __device__ __forceinline__ void warp_topn(ScoreFn score, int ncmp, int ncand, in
   for (int j = written + lane; j < n; j += 32) out(j, -1);
 }
 
-// Register path of the same selection for rows with at most 1024 candidates
-// (32 per lane).  Every candidate j gets the 64-bit key (score key << 32) |
+// Register path of the same selection for rows with at most 32 NI candidates
+// (NI per lane; warp_topn_regs below picks the smallest NI that holds the
+// row, so short rows cost proportionally less).  Every candidate j gets the 64-bit key (score key << 32) |
 // (0xFFFFFFFF - j), so larger keys rank first and equal scores rank by lower
 // index; keys are distinct.  The n-th largest of the 32 per-lane maxima is a
 // lower bound T0 of the n-th largest key (n lanes hold a key >= it); the keys
@@ -119,19 +120,19 @@ __device__ __forceinline__ void warp_topn(ScoreFn score, int ncmp, int ncand, in
 // when more than kCand keys reach T0; the caller then uses warp_topn.
 constexpr int kTopnCand = 64;
 
-template <typename ScoreFn, typename OutFn>
-__device__ __forceinline__ bool warp_topn_regs(ScoreFn score, int ncmp, int ncand, int n,
-                                               unsigned long long* cand, OutFn out) {
+template <int NI, typename ScoreFn, typename OutFn>
+__device__ __forceinline__ bool warp_topn_regs_n(ScoreFn score, int ncmp, int ncand, int n,
+                                                 unsigned long long* cand, OutFn out) {
   const int lane = threadIdx.x & 31;
   const unsigned lt_mask = (1u << lane) - 1u;
   if (ncand <= n) {
     for (int j = lane; j < n; j += 32) out(j, j < ncand ? j : -1);
     return true;
   }
-  unsigned long long key[32];
+  unsigned long long key[NI];
   unsigned long long lmax = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NI; ++i) {
     const int j = lane + 32 * i;
     const uint32_t b = j < ncmp ? score_key(score(j)) : kZeroScoreKey;
     key[i] = j < ncand ? (((unsigned long long)b << 32) | (0xFFFFFFFFu - (uint32_t)j)) : 0ull;
@@ -149,7 +150,7 @@ __device__ __forceinline__ bool warp_topn_regs(ScoreFn score, int ncmp, int ncan
   // gather the keys >= T0
   int count = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NI; ++i) {
     const bool p = key[i] >= t0 && key[i] != 0ull;
     const unsigned m = __ballot_sync(0xffffffffu, p);
     const int pos = count + __popc(m & lt_mask);
@@ -176,13 +177,23 @@ __device__ __forceinline__ bool warp_topn_regs(ScoreFn score, int ncmp, int ncan
   // every key >= K, in ascending block order
   int written = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < NI; ++i) {
     const bool take = key[i] >= kth && key[i] != 0ull;
     const unsigned m = __ballot_sync(0xffffffffu, take);
     if (take) out(written + __popc(m & lt_mask), lane + 32 * i);
     written += __popc(m);
   }
   return true;
+}
+
+// Rows of at most 1024 candidates: the register path sized to the row.
+template <typename ScoreFn, typename OutFn>
+__device__ __forceinline__ bool warp_topn_regs(ScoreFn score, int ncmp, int ncand, int n,
+                                               unsigned long long* cand, OutFn out) {
+  if (ncand <= 128) return warp_topn_regs_n<4>(score, ncmp, ncand, n, cand, out);
+  if (ncand <= 256) return warp_topn_regs_n<8>(score, ncmp, ncand, n, cand, out);
+  if (ncand <= 512) return warp_topn_regs_n<16>(score, ncmp, ncand, n, cand, out);
+  return warp_topn_regs_n<32>(score, ncmp, ncand, n, cand, out);
 }
 
 // The same selection as warp_topn_regs for any number of candidates whose
