@@ -136,7 +136,8 @@ struct BsLayout {
   static constexpr int kQ = 0;                              // 2 buffers
   static constexpr int kRing = kQ + 2 * kQBytes;            // kStages
   static constexpr int kBars = kRing + kStages * kChunkBytes;
-  static constexpr int kEnd = kBars + 32 * 8;
+  static constexpr int kW = kBars + 32 * 8;                 // per epilogue warpgroup: a tile's
+  static constexpr int kEnd = kW + 2 * kTileRows * 4;       // head weights [token][G] (fp32)
   // at least 116 KB so that one CTA owns an SM (it allocates all 512 TMEM columns)
   static constexpr int kSmem = kEnd > 118 * 1024 ? kEnd : 118 * 1024;
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -171,30 +172,37 @@ __device__ __forceinline__ BsItem bs_item(const PrefillArgs& a, int k) {
 
 // One chunk's epilogue for the thread owning key `key` (TMEM lane): the G
 // columns of each token summed, stored where the key is a candidate of the
-// token (key < t / l').  With token-level selection (`wts` non-null) the G
-// columns of a token are indexer heads: the score is the sum of the token's
-// head weights times ReLU(column), and keys up to and including the token
-// take part.
+// token (key < t / l').  With token-level selection (`wts` non-null: the
+// tile's head weights [token][G] in shared memory, zero past its tokens) the
+// G columns of a token are indexer heads: the score is the sum of the
+// token's head weights times ReLU(column), and keys up to and including the
+// token take part.  The TMEM loads of 64 columns are issued before one wait.
 template <int G>
 __device__ __forceinline__ void bs_rows(uint32_t taddr, float* srow, size_t tok_stride, int key,
                                         int t0, int ntok, int lg_ls, bool live,
                                         const float* wts) {
-#pragma unroll 2
-  for (int grp = 0; grp < kTileRows / 16; ++grp) {
-    float v[16];
-    tmem_ld16(taddr + grp * 16, v);
+#pragma unroll 1
+  for (int g4 = 0; g4 < kTileRows / 64; ++g4) {
+    float v[4][16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld16(taddr + g4 * 64 + q * 16, v[q]);
     tmem_ld_wait();
 #pragma unroll
-    for (int kt = 0; kt < 16 / G; ++kt) {
-      const int tok = (grp * 16 + kt * G) / G;
+    for (int kt = 0; kt < 64 / G; ++kt) {
+      const int tok = (g4 * 64 + kt * G) / G;
       float s = 0.f;
       if (wts) {
 #pragma unroll
-        for (int j = 0; j < G; ++j)
-          s += (tok < ntok ? __ldg(wts + (size_t)tok * G + j) : 0.f) * fmaxf(v[kt * G + j], 0.f);
+        for (int j = 0; j < G; ++j) {
+          const int c = kt * G + j;
+          s += wts[tok * G + j] * fmaxf(v[c >> 4][c & 15], 0.f);
+        }
       } else {
 #pragma unroll
-        for (int j = 0; j < G; ++j) s += v[kt * G + j];
+        for (int j = 0; j < G; ++j) {
+          const int c = kt * G + j;
+          s += v[c >> 4][c & 15];
+        }
       }
       const bool vis = wts ? key <= t0 + tok : key < ((t0 + tok) >> lg_ls);
       if (live && tok < ntok && vis) srow[(size_t)tok * tok_stride] = s;
@@ -345,12 +353,22 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int Hkv = a.geo.Hkv, cap = a.geo.cmp_cap, lgG = a.geo.lg_G, lg_ls = a.geo.lg_ls;
     const size_t tok_stride = (size_t)Hkv * cap;
-    int cc = 0;
+    float* wsm = reinterpret_cast<float*>(sm + L::kW) + w * kTileRows;
+    int cc = 0, w_item = -1;
     for (int k = blockIdx.x;; k += gridDim.x) {
       const BsItem it = bs_item(a, k);
       if (!it.valid) break;
       for (int c = 0; c < it.nc; ++c, ++cc) {
         if ((cc & 1) != w) continue;
+        if (a.token_select && w_item != k) {
+          // the tile's head weights, once per tile and warpgroup (named
+          // barrier 1 + w over its 128 threads: the previous tile's reads are
+          // done before the copy, the copy before the reads)
+          asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+          wsm[r] = r < it.ntok * G ? __ldg(a.gates + (size_t)it.row0 * G + r) : 0.f;
+          asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+          w_item = k;
+        }
         const int buf = cc & 3, ub = cc >> 2;
         mbar_wait(s_full + buf, ub & 1, abort_flag, status, kWaitCycles);
         tc_fence_after();
@@ -359,7 +377,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         const bool live = !*abort_flag;
         const uint32_t taddr = lane_addr + buf * 128;
         // per-token indexer head weights of the tile (token-level selection)
-        const float* wts = a.token_select ? a.gates + (size_t)it.row0 * a.geo.G : nullptr;
+        const float* wts = a.token_select ? wsm : nullptr;
         switch (lgG) {
           case 0: bs_rows<1>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live, wts); break;
           case 1: bs_rows<2>(taddr, srow, tok_stride, key, it.t0, it.ntok, lg_ls, live, wts); break;
