@@ -627,6 +627,19 @@ TOKEN_SELECT_KERNELS = ["nsa_meta_kernel", "nsa_block_score_kernel", "nsa_token_
                         "nsa_token_attn_kernel"]
 
 
+def token_select_work(lens, D, Hq, Hkv, index_heads, index_dim, top_k):
+    """Algorithmic work of token-level top-k attention on a packed batch:
+    index scores 2 Di per (query, indexer head, visible token), attention
+    4 D per (query, head, chosen token), and the bytes of the chosen tokens'
+    key and value rows gathered per (query, KV group)."""
+    f_index = chosen = 0
+    for Tb in lens:
+        t = np.arange(Tb, dtype=np.int64)
+        f_index += 2 * index_dim * index_heads * int((t + 1).sum())
+        chosen += int(np.minimum(t + 1, top_k).sum())
+    return {"index": f_index, "attn": 4 * D * Hq * chosen, "gather_bytes": chosen * Hkv * D * 2 * 2}
+
+
 def run_token_select_leg(dev, world, steps=5, warmup=3, name="prefill_8k", index_heads=16,
                          index_dim=128, top_k=2048):
     """Token-level top-k attention (DSA style: indexer of `index_heads` x
@@ -679,20 +692,11 @@ def run_token_select_leg(dev, world, steps=5, warmup=3, name="prefill_8k", index
     step()
     stage = nsa.profile_stage_ms()
     nsa.profile_enable(False)
-    # algorithmic work: index 2 Di per (query, indexer head, visible token);
-    # attention 4 D per (query, head, chosen token)
-    f_index = f_attn = 0
-    for Tb in lens:
-        t = np.arange(Tb, dtype=np.int64)
-        f_index += 2 * index_dim * index_heads * int((t + 1).sum())
-        f_attn += 4 * D * Hq * int(np.minimum(t + 1, top_k).sum())
+    work = token_select_work(lens, D, Hq, cfg.num_kv_heads, index_heads, index_dim, top_k)
+    f_index, f_attn, gather_bytes = work["index"], work["attn"], work["gather_bytes"]
     _, _, tc_sust, src = _peaks()
     ach_i = f_index / (stage[1] / 1e3) / 1e12
     ach_a = f_attn / (stage[3] / 1e3) / 1e12
-    # the chosen tokens' keys and values, gathered per (query, KV group)
-    Hkv = cfg.num_kv_heads
-    gather = sum(int(np.minimum(np.arange(Tb, dtype=np.int64) + 1, top_k).sum()) for Tb in lens)
-    gather_bytes = gather * Hkv * D * 2 * 2
     return {"metric": "token-level top-k attention tokens/s", "value": round(job_rate(T, world, ms), 1),
             "unit": "tokens/s", "ms_per_step_median": round(ms, 4), "steps": steps,
             "config": prefill_config(cfg, T, world) | {

@@ -1,7 +1,8 @@
 """The work counts behind the bench's roofline fractions (CPU): the
-algorithmic FLOPs are checked against a per-(token, head) count of the keys
-each branch attends to, taken from the oracle's own selection, and the decode
-byte count against a closed form when the selection covers every block."""
+algorithmic FLOPs of NSA, select-only and token-level attention are checked
+against per-(token, head) counts of the keys each branch attends to, taken
+from the oracle's own selections, and the decode byte count against a closed
+form when the selection covers every block."""
 import os
 import sys
 
@@ -55,3 +56,48 @@ def test_decode_bytes_closed_form_when_every_block_is_selected():
         # complete compressed blocks, per group; q, gates and out per sequence
         want += Hkv * ((L // l) * D * 2 * 2 + L * D * 2 * 2) + Hq * D * 2 + Hq * 3 * 4 + Hq * D * 2
     assert got == want
+
+
+def test_block_select_flops_match_a_key_count():
+    cfg = wl.NsaConfig("bscount", 33, 64, 4, 2, 32, 32, 32, 3, 40, seqlens=(150, 77))
+    inp = wl.prefill_inputs(cfg)
+    D, G, ls, Hkv = cfg.head_dim, cfg.group, cfg.sel_block, cfg.num_kv_heads
+    p = OracleParams.of(cfg)
+    res = oracle.block_select_reference(p, inp)
+    route = keys = 0
+    for r, T in zip(res, cfg.seqlens):
+        for t in range(T):
+            route += G * Hkv * (t // ls)  # complete blocks before t's own block
+            for g in range(Hkv):
+                for blk in r["sel"][t, g]:
+                    if blk >= 0:
+                        keys += G * sum(1 for u in range(blk * ls, blk * ls + ls) if u <= t)
+    sel = np.concatenate([r["sel"] for r in res])
+    f = bench.block_select_flops(cfg, list(cfg.seqlens), sel)
+    assert f["route"] == 2 * D * route
+    assert f["attn"] == 4 * D * keys
+    assert f["total"] == f["route"] + f["attn"]
+
+
+def test_token_select_work_matches_a_key_count():
+    cfg = wl.NsaConfig("tscount", 34, 64, 4, 2, 32, 32, 32, 3, 40, seqlens=(90, 41))
+    lens = list(cfg.seqlens)
+    inp = wl.prefill_inputs(cfg)
+    Hi, Di, top_k = 2, 64, 20
+    idx = wl.indexer_inputs(lens, Hi, Di, seed=5)
+    p = OracleParams.of(cfg)
+    D, Hq, Hkv = cfg.head_dim, cfg.num_q_heads, cfg.num_kv_heads
+    cu = inp["cu_seqlens"]
+    index = chosen = 0
+    for b, T in enumerate(lens):
+        s, e = int(cu[b]), int(cu[b + 1])
+        r = oracle.dsa_rows(p, top_k, inp["q"][s:e], inp["k"][s:e], inp["v"][s:e],
+                            idx["q_index"][s:e], idx["w_index"][s:e], idx["k_index"][s:e],
+                            np.arange(T, dtype=np.int32))
+        for t in range(T):
+            index += Hi * (t + 1)  # every token up to and including t is scored
+            chosen += int(np.count_nonzero(r["sel"][t] >= 0))
+    w = bench.token_select_work(lens, D, Hq, Hkv, Hi, Di, top_k)
+    assert w["index"] == 2 * Di * index
+    assert w["attn"] == 4 * D * Hq * chosen
+    assert w["gather_bytes"] == chosen * Hkv * D * 2 * 2
