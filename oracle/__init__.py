@@ -8,7 +8,9 @@ package never imports the product package.  Inputs arrive as numpy arrays
 
 Every function follows the definition written out in ``nsa_oracle.c``; the
 header of that file cites the pages and lists the readings taken where the
-pages are silent.
+pages are silent.  ``backward.py`` (``from oracle import backward``) holds the
+fp64 gradients of that forward with the block selection held fixed, in plain
+numpy; its header states the readings it takes.
 """
 from .oracle import (OracleParams, build, compress, nsa_rows, nsa_query, select_f32,
                      num_cmp_blocks, prefill_reference, decode_reference, bf16_round_f64,
