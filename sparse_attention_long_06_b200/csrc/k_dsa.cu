@@ -23,7 +23,8 @@ using namespace sm100;
 // padded with -1 when t + 1 < top_k.
 //
 // Short rows (at most 1024 candidates, top_k <= 32): one warp per row, the
-// register path of the block selection.
+// register path of the block selection (its 8-bit radix select when more
+// keys than the register path ranks reach its bound).
 __global__ void __launch_bounds__(256) nsa_token_topk_short_kernel(PrefillArgs a, int top_k) {
   if (a.meta->bad) return;
   __shared__ unsigned hist_all[8][256];
@@ -212,12 +213,16 @@ __global__ void __launch_bounds__(kTkThreads) nsa_token_topk_kernel(PrefillArgs 
 // (rows past G are zero queries whose results are dropped).  The selected
 // tokens are taken 32 at a time; their keys and values for every group are
 // copied (16-byte cp.async, a ring of three steps: two in flight while one is
-// computed) into shared memory rows padded to D + 8 elements, so that the
-// eight rows an operand fragment spans fall in different banks.  Per step and warp: S = Q K^T (queries as A fragments
-// kept in registers, keys read as B fragments), an online softmax on the
-// accumulator fragments (row statistics over the four threads of a quad),
-// then O += P V with P re-packed from the S fragments as A fragments and V
-// read by ldmatrix.trans.
+// computed; each step's positions are loaded one step before its copies are
+// issued) into shared memory rows padded to D + 8 elements, so that the
+// eight rows an operand fragment spans fall in different banks.  Per step
+// and warp: S = Q K^T (queries as A fragments kept in registers, keys read
+// as B fragments), an online softmax on the accumulator fragments (row
+// statistics over the four threads of a quad), then O += P V with P
+// re-packed from the S fragments as A fragments and V read by
+// ldmatrix.trans.  The chosen rows are single 256-byte rows at random
+// positions; 16-byte cp.async moved them faster than bulk copies or TMA
+// row gathers (tile::gather4).
 namespace {
 
 constexpr int kDsaKeys = 32;  // selected tokens per step
