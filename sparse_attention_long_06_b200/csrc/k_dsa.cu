@@ -92,6 +92,45 @@ __device__ __forceinline__ float4 tk_load(const float* S, int q, int nq) {
   return q < nq ? __ldg(reinterpret_cast<const float4*>(S) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// The order-preserving key of score_key in fewer operations: the sign bit
+// spread over the word flips every bit of a negative score and only the top
+// bit of a non-negative one; -0 takes the key of +0.
+__device__ __forceinline__ uint32_t tk_key(float s) {
+  const uint32_t b = __float_as_uint(s);
+  const uint32_t k = b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+  return b == 0x80000000u ? 0x80000000u : k;
+}
+
+// One histogram pass of the radix select over the row's candidates: the
+// digit (x >> SHIFT) & DMASK of every key x that shares `prefix` (under
+// `pmask`; the first pass has no prefix).  `vmask(q)` gives the candidate
+// scores of float4 word q (bits 0..3).
+template <int SHIFT, uint32_t DMASK, bool FIRST, typename VMask>
+__device__ __forceinline__ void tk_hist_pass(const float* S, int nq, VMask vmask, uint32_t prefix,
+                                             uint32_t pmask, unsigned* hist) {
+  const int tid = threadIdx.x;
+  for (int base = 0; base < nq; base += 4 * kTkThreads) {
+    float4 v[4];
+    uint32_t vm[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int q = base + u * kTkThreads + tid;
+      v[u] = tk_load(S, q, nq);
+      vm[u] = vmask(q);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t x = tk_key(f[e]);
+        const bool in = ((vm[u] >> e) & 1u) && (FIRST || (x & pmask) == prefix);
+        if (in) atomicAdd(&hist[(x >> SHIFT) & DMASK], 1u);
+      }
+    }
+  }
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kTkThreads) nsa_token_topk_kernel(PrefillArgs a, int top_k) {
@@ -110,6 +149,11 @@ __global__ void __launch_bounds__(kTkThreads) nsa_token_topk_kernel(PrefillArgs 
     return;
   }
   const int nq = (ncand + 3) >> 2;  // float4 words of the row
+  // candidate scores of word q: all four below ncand / 4, the low ncand % 4
+  // of the word holding the row's end, none past it
+  const int nfull = ncand >> 2;
+  const uint32_t tail = (1u << (ncand & 3)) - 1u;
+  auto vmask = [=](int q) -> uint32_t { return q < nfull ? 0xFu : (q == nfull ? tail : 0u); };
   uint32_t prefix = 0, pmask = 0;
   unsigned k = (unsigned)top_k;  // rank still to be found inside the prefix class
   int shift = 21;
@@ -118,22 +162,9 @@ __global__ void __launch_bounds__(kTkThreads) nsa_token_topk_kernel(PrefillArgs 
     const uint32_t dmask = pass == 2 ? 1023u : 2047u;
     for (int i = tid; i < kTkBins; i += kTkThreads) hist[i] = 0;
     __syncthreads();
-    for (int base = 0; base < nq; base += 4 * kTkThreads) {
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = tk_load(S, base + u * kTkThreads + tid, nq);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j0 = 4 * (base + u * kTkThreads + tid);
-        const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t x = score_key(f[e]);
-          const bool in = j0 + e < ncand && (x & pmask) == prefix;
-          if (in) atomicAdd(&hist[(x >> shift) & dmask], 1u);
-        }
-      }
-    }
+    if (pass == 0) tk_hist_pass<21, 2047u, true>(S, nq, vmask, prefix, pmask, hist);
+    else if (pass == 1) tk_hist_pass<10, 2047u, false>(S, nq, vmask, prefix, pmask, hist);
+    else tk_hist_pass<0, 1023u, false>(S, nq, vmask, prefix, pmask, hist);
     __syncthreads();
     // thread i owns bins [i * 4, i * 4 + 4); higher threads hold higher digits
     unsigned c[kTkBinsPerThread], mine = 0;
@@ -179,11 +210,12 @@ __global__ void __launch_bounds__(kTkThreads) nsa_token_topk_kernel(PrefillArgs 
     nxt = tk_load(S, base + kTkThreads + tid, nq);
     const int j0 = 4 * (base + tid);
     const float f[4] = {cur.x, cur.y, cur.z, cur.w};
+    const uint32_t vm = vmask(base + tid);
     unsigned gtm = 0, eqm = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const uint32_t xt = score_key(f[e]) >> shift;
-      const bool valid = j0 + e < ncand;
+      const uint32_t xt = tk_key(f[e]) >> shift;
+      const bool valid = (vm >> e) & 1u;
       gtm |= (valid && xt > thr) ? 1u << e : 0u;
       eqm |= (valid && xt == thr) ? 1u << e : 0u;
     }
