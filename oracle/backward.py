@@ -117,11 +117,37 @@ def _branch_backward(qv, keys, vals, dob, scale):
     return scale * (dz @ keys), scale * np.outer(dz, qv), np.outer(pr, dob)
 
 
-def backward(p, q, k, v, gates, w_k, w_v, sel, dout, kc=None, vc=None) -> dict:
+def rows_touching_keys(p, sel, T: int, key_lo: int, key_hi: int) -> np.ndarray:
+    """Query rows t (ascending) of a sequence of T tokens whose forward reads
+    any key or value token in [key_lo, key_hi) through any branch and any KV
+    group: the window, a chosen block, or a visible compressed block whose
+    tokens overlap the range.  The gradients reaching those tokens come from
+    these rows only."""
+    _, _, Hkv, _, _, _, _, _ = _geometry(p)
+    C = num_blocks(p, T)
+    l, d = p.cmp_block, p.cmp_stride
+    out = []
+    for t in range(T):
+        hit = False
+        for g in range(Hkv):
+            cmp, slc, win = _key_sets(p, t, sel[t, g], C)
+            if (any(key_lo <= u < key_hi for u in slc) or any(key_lo <= u < key_hi for u in win)
+                    or any(i * d < key_hi and key_lo < i * d + l for i in cmp)):
+                hit = True
+                break
+        if hit:
+            out.append(t)
+    return np.asarray(out, dtype=np.int64)
+
+
+def backward(p, q, k, v, gates, w_k, w_v, sel, dout, kc=None, vc=None, rows=None) -> dict:
     """Gradients of sum(dout * out) for the forward of ``forward_fixed`` (same
     arguments).  Returns dq [T,Hq,D], dk, dv [T,Hkv,D], dgates [T,Hq,3],
     dw_k, dw_v [Hkv,D,l*D] and dkc, dvc [C,Hkv,D] (the gradients reaching the
-    compressed keys and values)."""
+    compressed keys and values).  rows: the query rows whose terms are
+    summed (default all): dq and dgates are exact on those rows, and dk, dv
+    are exact on every token that only those rows read (see
+    ``rows_touching_keys``); everything else holds partial sums."""
     D, Hq, Hkv, l, d, _, _, scale = _geometry(p)
     T = q.shape[0]
     G = Hq // Hkv
@@ -134,7 +160,7 @@ def backward(p, q, k, v, gates, w_k, w_v, sel, dout, kc=None, vc=None) -> dict:
     dkc = np.zeros(kc.shape)
     dvc = np.zeros(vc.shape)
     dgates = np.zeros(gates.shape)
-    for t in range(T):
+    for t in (range(T) if rows is None else rows):
         for h in range(Hq):
             g = h // G
             cmp, slc, win = _key_sets(p, t, sel[t, g], C)

@@ -10,7 +10,10 @@
     the selected and the window branch are dense causal attention: their
     gradients equal torch's fp64 autograd of scaled_dot_product_attention;
   - with l = d = 1 and identity compressors the compressed branch is dense
-    causal attention too: same check.
+    causal attention too: same check;
+  - restricted to the query rows that read a key range (the form sampled
+    parity at full sizes uses), dk and dv on that range and dq on those rows
+    equal the full backward's.
 """
 import numpy as np
 import pytest
@@ -137,3 +140,22 @@ def test_identity_compressor_gradients_equal_causal_attention_autograd():
     np.testing.assert_allclose(g["dq"], dq, rtol=0, atol=1e-12)
     np.testing.assert_allclose(g["dk"], dk, rtol=0, atol=1e-12)
     np.testing.assert_allclose(g["dv"], dv, rtol=0, atol=1e-12)
+
+
+def test_rows_touching_a_key_range_give_its_exact_gradients():
+    D, Hq, Hkv, l, d, ls, n, w, T = 4, 4, 2, 4, 2, 4, 2, 5, 30
+    p = OracleParams(D, Hq, Hkv, l, d, ls, n, w)
+    c = _random_case(p, T, seed=91)
+    args = (p, c["q"], c["k"], c["v"], c["gates"], c["w_k"], c["w_v"], c["sel"], c["dout"])
+    full = bw.backward(*args)
+    for lo, hi in ((8, 12), (0, 4), (26, 30)):
+        rows = bw.rows_touching_keys(p, c["sel"], T, lo, hi)
+        assert len(rows) > 0 and rows.min() >= lo  # causal: no earlier row reads the range
+        part = bw.backward(*args, rows=rows)
+        np.testing.assert_allclose(part["dk"][lo:hi], full["dk"][lo:hi], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(part["dv"][lo:hi], full["dv"][lo:hi], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(part["dq"][rows], full["dq"][rows], rtol=0, atol=1e-13)
+        # leaving out one row of the set changes the range's gradients (dv:
+        # a row attending one key alone has p = 1 and adds nothing to dk)
+        fewer = bw.backward(*args, rows=rows[1:])
+        assert not np.allclose(fewer["dv"][lo:hi], full["dv"][lo:hi], rtol=0, atol=1e-13)
