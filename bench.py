@@ -835,7 +835,7 @@ def run_reference(args):
         descs.append(r["sample"])
     wall = time.perf_counter() - t0
     v = statistics.median(vals)
-    cb = {"value": v, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+    cb = {"value": round(v, 3), "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
           "sample": "per step: " + descs[-1]}
     return {"impl": "reference", "metric": METRIC, "value": round(v, 3), "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
