@@ -15,9 +15,9 @@ numpy; its header states the readings it takes.
 from .oracle import (OracleParams, build, compress, nsa_rows, nsa_query, select_f32,
                      num_cmp_blocks, prefill_reference, decode_reference, bf16_round_f64,
                      block_means, block_select_rows, block_select_reference,
-                     block_select_query, block_select_decode_reference, dsa_rows)
+                     block_select_query, block_select_decode_reference, dsa_rows, backward_c)
 
 __all__ = ["OracleParams", "build", "compress", "nsa_rows", "nsa_query", "select_f32",
            "num_cmp_blocks", "prefill_reference", "decode_reference", "bf16_round_f64",
            "block_means", "block_select_rows", "block_select_reference",
-           "block_select_query", "block_select_decode_reference", "dsa_rows"]
+           "block_select_query", "block_select_decode_reference", "dsa_rows", "backward_c"]

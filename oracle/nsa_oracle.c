@@ -42,6 +42,7 @@
  *    applied as given.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -586,4 +587,224 @@ int oracle_dsa_rows(const nsa_oracle_params* P, const dsa_oracle_params* X, int 
     bad |= (rc != 0);
   }
   return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Backward of the forward above with the block selection held fixed, in
+ * fp64 on fp64 inputs: the same definition as oracle/backward.py, whose
+ * header states the readings (fixed selection, the compressed tensor's
+ * rounding taken as the identity, an empty branch passes no gradient).
+ * OpenMP over query rows; the key-side gradients accumulate atomically.
+ * ------------------------------------------------------------------------ */
+
+/* One branch of query row q (D values) over `m` key rows keys[] of K and V
+ * (row r at K + r * rs): forward softmax(scale q . k) and O = sum p v into
+ * o_out; with upstream gradient dob: dq += scale sum dz k, dK[r] += scale dz
+ * q, dV[r] += p dob, where dz = p (v . dob - sum p (v . dob)). */
+static void bw_branch(int D, double scale, const double* qv, const double* K, const double* V,
+                      size_t rs, const int* keys, int m, const double* dob, double* dq,
+                      double* dK, double* dV, double* o_out, double* p, double* dp, int shared) {
+  for (int c = 0; c < D; ++c) o_out[c] = 0.0;
+  if (m == 0) return;
+  double zmax = -INFINITY;
+  for (int a = 0; a < m; ++a) {
+    const double* kr = K + (size_t)keys[a] * rs;
+    double z = 0.0;
+    for (int c = 0; c < D; ++c) z += qv[c] * kr[c];
+    p[a] = scale * z;
+    if (p[a] > zmax) zmax = p[a];
+  }
+  double sum = 0.0;
+  for (int a = 0; a < m; ++a) {
+    p[a] = exp(p[a] - zmax);
+    sum += p[a];
+  }
+  double dsum = 0.0;
+  for (int a = 0; a < m; ++a) {
+    p[a] /= sum;
+    const double* vr = V + (size_t)keys[a] * rs;
+    double x = 0.0;
+    for (int c = 0; c < D; ++c) {
+      o_out[c] += p[a] * vr[c];
+      x += vr[c] * dob[c];
+    }
+    dp[a] = x;
+    dsum += p[a] * x;
+  }
+  for (int a = 0; a < m; ++a) {
+    const double dz = p[a] * (dp[a] - dsum);
+    const double* kr = K + (size_t)keys[a] * rs;
+    double* dkr = dK + (size_t)keys[a] * rs;
+    double* dvr = dV + (size_t)keys[a] * rs;
+    for (int c = 0; c < D; ++c) {
+      dq[c] += scale * dz * kr[c];
+      if (shared) {
+#pragma omp atomic
+        dkr[c] += scale * dz * qv[c];
+#pragma omp atomic
+        dvr[c] += p[a] * dob[c];
+      } else {
+        dkr[c] += scale * dz * qv[c];
+        dvr[c] += p[a] * dob[c];
+      }
+    }
+  }
+}
+
+static int cmp_int(const void* a, const void* b) {
+  const int x = *(const int*)a, y = *(const int*)b;
+  return (x > y) - (x < y);
+}
+
+/* Gradients of sum(dout * out) for one sequence of T tokens.  q [T,Hq,D],
+ * k/v [T,Hkv,D], gates [T,Hq,3], w_k/w_v [Hkv,D,l*D], sel [T,Hkv,n] (-1
+ * padded), dout [T,Hq,D]; kc_in/vc_in [C,Hkv,D] the compressed tensors to
+ * attend to, or NULL for step 1 in fp64.  rows: the query rows whose terms
+ * are summed (NULL: all T).  Outputs (overwritten): dq, dk, dv, dgates,
+ * dw_k, dw_v, dkc, dvc.  Returns 0, or -1 for a geometry it cannot hold. */
+int oracle_backward(const nsa_oracle_params* P, int T, const double* q, const double* k,
+                    const double* v, const double* gates, const double* wk, const double* wv,
+                    const int* sel, const double* dout, const double* kc_in,
+                    const double* vc_in, const int* rows, int nrows, double* dq, double* dk,
+                    double* dv, double* dgates, double* dwk, double* dwv, double* dkc,
+                    double* dvc) {
+  const int D = P->D, Hq = P->Hq, Hkv = P->Hkv, l = P->l, d = P->d, ls = P->lsel, n = P->n;
+  if (Hkv <= 0 || Hq % Hkv != 0 || T < 0) return -1;
+  const int G = Hq / Hkv, C = oracle_num_cmp_blocks(P, T), LD = l * D;
+  const size_t rs = (size_t)Hkv * D;
+  const double scale = P->scale;
+  double* kc = (double*)malloc(sizeof(double) * ((size_t)C * rs + 1));
+  double* vc = (double*)malloc(sizeof(double) * ((size_t)C * rs + 1));
+  if (!kc || !vc) {
+    free(kc);
+    free(vc);
+    return -1;
+  }
+  for (int i = 0; i < C; ++i)
+    for (int g = 0; g < Hkv; ++g)
+      for (int r = 0; r < D; ++r) {
+        double sk = 0.0, sv = 0.0;
+        for (int e = 0; e < LD; ++e) {
+          const size_t x = ((size_t)(i * d + e / D) * Hkv + g) * D + e % D;
+          sk += wk[((size_t)g * D + r) * LD + e] * k[x];
+          sv += wv[((size_t)g * D + r) * LD + e] * v[x];
+        }
+        kc[((size_t)i * Hkv + g) * D + r] = kc_in ? kc_in[((size_t)i * Hkv + g) * D + r] : sk;
+        vc[((size_t)i * Hkv + g) * D + r] = vc_in ? vc_in[((size_t)i * Hkv + g) * D + r] : sv;
+      }
+  memset(dq, 0, sizeof(double) * (size_t)T * Hq * D);
+  memset(dk, 0, sizeof(double) * (size_t)T * rs);
+  memset(dv, 0, sizeof(double) * (size_t)T * rs);
+  memset(dgates, 0, sizeof(double) * (size_t)T * Hq * 3);
+  memset(dwk, 0, sizeof(double) * (size_t)Hkv * D * LD);
+  memset(dwv, 0, sizeof(double) * (size_t)Hkv * D * LD);
+  memset(dkc, 0, sizeof(double) * (size_t)C * rs);
+  memset(dvc, 0, sizeof(double) * (size_t)C * rs);
+  const int R = rows ? nrows : T;
+  int fail = 0;
+  /* key-side gradients: each thread sums into its own copy, merged at the
+   * end, when the copies fit in 2 GB; otherwise atomically into the result */
+  const size_t kv_elems = ((size_t)T + C) * rs;
+#pragma omp parallel
+  {
+    const int nthr = omp_get_num_threads();
+    const int priv = (double)nthr * 2.0 * (double)kv_elems * sizeof(double) <= 2e9;
+    double* pk = priv ? (double*)calloc(2 * kv_elems + 1, sizeof(double)) : NULL;
+    const int use_priv = pk != NULL;
+    double* tdk = use_priv ? pk : dk;
+    double* tdv = use_priv ? pk + (size_t)T * rs : dv;
+    double* tdkc = use_priv ? pk + 2 * (size_t)T * rs : dkc;
+    double* tdvc = use_priv ? pk + 2 * (size_t)T * rs + (size_t)C * rs : dvc;
+    const int cap = T + C + 1;
+    int* ck = (int*)malloc(sizeof(int) * cap);
+    int* sk = (int*)malloc(sizeof(int) * cap);
+    int* wkeys = (int*)malloc(sizeof(int) * cap);
+    double* p = (double*)malloc(sizeof(double) * cap);
+    double* dp = (double*)malloc(sizeof(double) * cap);
+    double* o = (double*)malloc(sizeof(double) * D);
+    double* dob = (double*)malloc(sizeof(double) * D);
+    const int ok = ck && sk && wkeys && p && dp && o && dob;
+    if (!ok) {
+#pragma omp atomic write
+      fail = 1;
+    }
+    /* every thread takes part in the loop; one without scratch skips its rows */
+#pragma omp for schedule(dynamic, 4)
+    for (int rr = 0; rr < R; ++rr) {
+      if (ok) {
+        const int t = rows ? rows[rr] : rr;
+        for (int h = 0; h < Hq; ++h) {
+          const int g = h / G;
+          int mc = 0, msl = 0, mw = 0;
+          for (int i = 0; i < C; ++i)
+            if (i * d + l - 1 <= t) ck[mc++] = i;
+          for (int s = 0; s < n; ++s) {
+            const int j = sel[((size_t)t * Hkv + g) * n + s];
+            if (j < 0) continue;
+            for (int u = j * ls; u < j * ls + ls && u <= t; ++u) sk[msl++] = u;
+          }
+          qsort(sk, msl, sizeof(int), cmp_int);
+          for (int u = (t - P->w + 1 > 0 ? t - P->w + 1 : 0); u <= t; ++u) wkeys[mw++] = u;
+          const double* qv = q + ((size_t)t * Hq + h) * D;
+          const double* dov = dout + ((size_t)t * Hq + h) * D;
+          double* dqv = dq + ((size_t)t * Hq + h) * D;
+          const double* gt = gates + ((size_t)t * Hq + h) * 3;
+          double* dg = dgates + ((size_t)t * Hq + h) * 3;
+          for (int b = 0; b < 3; ++b) {
+            for (int c = 0; c < D; ++c) dob[c] = gt[b] * dov[c];
+            if (b == 0)
+              bw_branch(D, scale, qv, kc + (size_t)g * D, vc + (size_t)g * D, rs, ck, mc, dob, dqv,
+                        tdkc + (size_t)g * D, tdvc + (size_t)g * D, o, p, dp, !use_priv);
+            else
+              bw_branch(D, scale, qv, k + (size_t)g * D, v + (size_t)g * D, rs, b == 1 ? sk : wkeys,
+                        b == 1 ? msl : mw, dob, dqv, tdk + (size_t)g * D, tdv + (size_t)g * D, o, p,
+                        dp, !use_priv);
+            double x = 0.0;
+            for (int c = 0; c < D; ++c) x += dov[c] * o[c];
+            dg[b] = x;
+          }
+        }
+      }
+    }
+    if (use_priv) {
+      /* atomic: a thread without a private copy may still be adding */
+      for (size_t e = 0; e < (size_t)T * rs; ++e) {
+#pragma omp atomic
+        dk[e] += tdk[e];
+#pragma omp atomic
+        dv[e] += tdv[e];
+      }
+      for (size_t e = 0; e < (size_t)C * rs; ++e) {
+#pragma omp atomic
+        dkc[e] += tdkc[e];
+#pragma omp atomic
+        dvc[e] += tdvc[e];
+      }
+    }
+    free(pk);
+    free(ck);
+    free(sk);
+    free(wkeys);
+    free(p);
+    free(dp);
+    free(o);
+    free(dob);
+  }
+  /* step 1: K~[i, g] = W[g] vec(x[i d : i d + l, g]) */
+  for (int i = 0; i < C && !fail; ++i)
+    for (int g = 0; g < Hkv; ++g)
+      for (int r = 0; r < D; ++r) {
+        const double gk = dkc[((size_t)i * Hkv + g) * D + r];
+        const double gv = dvc[((size_t)i * Hkv + g) * D + r];
+        for (int e = 0; e < LD; ++e) {
+          const size_t x = ((size_t)(i * d + e / D) * Hkv + g) * D + e % D;
+          dwk[((size_t)g * D + r) * LD + e] += gk * k[x];
+          dwv[((size_t)g * D + r) * LD + e] += gv * v[x];
+          dk[x] += wk[((size_t)g * D + r) * LD + e] * gk;
+          dv[x] += wv[((size_t)g * D + r) * LD + e] * gv;
+        }
+      }
+  free(kc);
+  free(vc);
+  return fail ? -1 : 0;
 }

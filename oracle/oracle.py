@@ -100,6 +100,8 @@ def _load():
             lib.oracle_dsa_rows.argtypes = [P, ctypes.POINTER(_DsaParams), ctypes.c_int, vp, vp, vp,
                                             vp, vp, vp, vp, ctypes.c_int, vp, vp, vp, vp]
             lib.oracle_dsa_rows.restype = ctypes.c_int
+            lib.oracle_backward.argtypes = [P, ctypes.c_int] + [vp] * 11 + [ctypes.c_int] + [vp] * 8
+            lib.oracle_backward.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -366,4 +368,33 @@ def dsa_rows(p: OracleParams, top_k: int, q, k, v, qi, w, ki, rows, with_index: 
         raise ValueError("oracle rejected the geometry or a row index")
     if with_index:
         res["index"] = idx
+    return res
+
+
+def backward_c(p: OracleParams, q, k, v, gates, w_k, w_v, sel, dout, kc=None, vc=None,
+               rows=None) -> dict:
+    """The backward of ``oracle.backward.backward`` (same arguments and
+    results: fp64 inputs, the selection held fixed) in C with OpenMP over
+    query rows, for sizes where the numpy loops are slow."""
+    D, Hq, Hkv = p.head_dim, p.num_q_heads, p.num_kv_heads
+    q, k, v = _c(q, np.float64), _c(k, np.float64), _c(v, np.float64)
+    gates, dout = _c(gates, np.float64), _c(dout, np.float64)
+    w_k, w_v = _c(w_k, np.float64), _c(w_v, np.float64)
+    sel = _c(sel, np.int32)
+    T = q.shape[0]
+    C = num_cmp_blocks(p, T)
+    kc = None if kc is None else _c(kc, np.float64)
+    vc = None if vc is None else _c(vc, np.float64)
+    rr = None if rows is None else _c(rows, np.int32)
+    res = {"dq": np.zeros((T, Hq, D)), "dk": np.zeros((T, Hkv, D)), "dv": np.zeros((T, Hkv, D)),
+           "dgates": np.zeros((T, Hq, 3)), "dw_k": np.zeros(w_k.shape), "dw_v": np.zeros(w_v.shape),
+           "dkc": np.zeros((C, Hkv, D)), "dvc": np.zeros((C, Hkv, D))}
+    none = ctypes.c_void_p(None)
+    rc = _load().oracle_backward(
+        ctypes.byref(p.c()), T, _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(w_k), _ptr(w_v),
+        _ptr(sel), _ptr(dout), none if kc is None else _ptr(kc), none if vc is None else _ptr(vc),
+        none if rr is None else _ptr(rr), 0 if rr is None else len(rr),
+        *[_ptr(res[name]) for name in ("dq", "dk", "dv", "dgates", "dw_k", "dw_v", "dkc", "dvc")])
+    if rc != 0:
+        raise ValueError("oracle rejected the geometry")
     return res

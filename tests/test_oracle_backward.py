@@ -13,7 +13,9 @@
     causal attention too: same check;
   - restricted to the query rows that read a key range (the form sampled
     parity at full sizes uses), dk and dv on that range and dq on those rows
-    equal the full backward's.
+    equal the full backward's;
+  - the C/OpenMP backward (``oracle.backward_c``) equals this numpy one, with
+    and without given compressed tensors and row restriction.
 """
 import numpy as np
 import pytest
@@ -159,3 +161,26 @@ def test_rows_touching_a_key_range_give_its_exact_gradients():
         # a row attending one key alone has p = 1 and adds nothing to dk)
         fewer = bw.backward(*args, rows=rows[1:])
         assert not np.allclose(fewer["dv"][lo:hi], full["dv"][lo:hi], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("geom", [
+    # D, Hq, Hkv, l, d, l', n, w, T
+    (8, 8, 2, 4, 4, 4, 3, 7, 40),
+    (8, 4, 1, 4, 2, 8, 2, 9, 37),  # d < l and l' = 2 l
+])
+def test_c_backward_equals_the_numpy_backward(geom):
+    D, Hq, Hkv, l, d, ls, n, w, T = geom
+    p = OracleParams(D, Hq, Hkv, l, d, ls, n, w)
+    c = _random_case(p, T, seed=200 + T)
+    args = (p, c["q"], c["k"], c["v"], c["gates"], c["w_k"], c["w_v"], c["sel"], c["dout"])
+    C = bw.num_blocks(p, T)
+    rng = np.random.default_rng(3)
+    kc = rng.standard_normal((C, Hkv, D))
+    vc = rng.standard_normal((C, Hkv, D))
+    rows = bw.rows_touching_keys(p, c["sel"], T, 12, 20)
+    for extra in ({}, {"kc": kc, "vc": vc}, {"rows": rows}):
+        a = bw.backward(*args, **extra)
+        b = oracle.backward_c(*args, **extra)
+        for name in ("dq", "dk", "dv", "dgates", "dw_k", "dw_v", "dkc", "dvc"):
+            np.testing.assert_allclose(b[name], a[name], rtol=0, atol=1e-12,
+                                       err_msg=f"{name} {sorted(extra)}")
